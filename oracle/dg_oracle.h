@@ -1,0 +1,120 @@
+/*
+ * dg_oracle.h -- plain CPU reference ("oracle") for the FP8 fine-grained-scaled
+ * GEMM family described on the DeepGEMM pages. TEST INFRASTRUCTURE ONLY: only
+ * tests, the smoke check and the benchmark's CPU-baseline leg may load it. It
+ * shares no code, header, table or helper with the CUDA library.
+ *
+ * Sources (page title, section):
+ *   - "DeepGEMM" README summary (ja.news.hada.io topic 19459), section
+ *     "GEMMインターフェースとレイアウト制約": D = C + A @ B.T with NT as the base
+ *     layout; LHS scaling factors TMA-aligned and transposed; FP32 scales.
+ *   - same page, section "DenseとGrouped GEMM": M-grouped contiguous layout
+ *     (segments aligned to the M block), masked layout (only rows below the
+ *     per-group count are computed), K-grouped TN for the MoE weight gradient.
+ *   - "DeepSeek開源新突破：DeepGEMM庫揭秘" (picoinsstore.com), paragraph 2:
+ *     two-level accumulation (promotion) because the FP8 tensor-core
+ *     accumulator is imprecise.
+ *   - E4M3 "FN" encoding: OCP 8-bit Floating Point Specification (OFP8) v1.0,
+ *     section 5.3 (bias 7, no infinities, S.1111.111 is NaN, max 448).
+ *
+ * All GEMM arithmetic is FP64 on decoded bytes. Every function here is
+ * "parity pinned" by CPU tests against closed forms, library routines and
+ * invariants (see tests/test_oracle_*.py).
+ */
+#ifndef DG_ORACLE_H
+#define DG_ORACLE_H
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* E4M3 (FN) byte -> value, from the OFP8 definition. NaN for 0x7F/0xFF. */
+double dgo_e4m3_decode(uint8_t code);
+
+/* Nearest finite E4M3 value to y, ties to even mantissa, |y| > 448 saturates
+ * to +-448, NaN -> 0x7F. Sign bit is copied from y (so -tiny -> 0x80). */
+uint8_t dgo_e4m3_encode(float y);
+
+/* bf16 bit pattern -> float (exact). */
+float dgo_bf16_to_f32(uint16_t bits);
+
+/* Quantisation modes (same numbering as the library ABI, re-declared here). */
+enum { DGO_ROW_1x128 = 0, DGO_BLOCK_128x128 = 1, DGO_COL_128x1 = 2 };
+
+/*
+ * Quantise x[batch][rows][cols] (float if in_is_bf16 == 0, bf16 bits
+ * otherwise) into E4M3 codes[batch][rows][cols] and FP32 scales:
+ *   ROW_1x128    : one scale per (row, 128-column strip); cols % 128 == 0;
+ *                  scales[b][cols/128][ld_scales] (transposed, "MN-major").
+ *   BLOCK_128x128: one scale per 128x128 block (rows may be ragged);
+ *                  scales[b][ceil(rows/128)][cols/128]; cols % 128 == 0.
+ *   COL_128x1    : one scale per (128-row strip, column); rows % 128 == 0;
+ *                  scales[b][rows/128][cols].
+ * scale = max(amax, 1e-4f) / 448.0f and code = E4M3(x / scale), both IEEE
+ * float divisions. Returns 0, or -1 on an invalid argument.
+ */
+int dgo_quantize(const void* x, int in_is_bf16, int batch, int rows, int cols,
+                 int mode, uint8_t* codes, float* scales, int ld_scales);
+
+/* C operand kinds for the GEMMs below. */
+enum { DGO_C_NONE = 0, DGO_C_BF16 = 1, DGO_C_F32 = 2 };
+
+/*
+ * Dense NT: R[i][n] = C[m][n] + sum_kb sfa[kb][m] * sfb[n/128][kb] *
+ *                     sum_{k in kb} dec(A[m][k]) * dec(B[n][k]),  m = rows[i]
+ * A [M][K], sfa [K/128][ld_sfa], B [N][K], sfb [ceil(N/128)][K/128],
+ * C [M][N] (kind c_kind), R [n_rows][N] double. rows == NULL means all M rows
+ * (n_rows must then equal M).
+ */
+int dgo_gemm_nt(const uint8_t* A, const float* sfa, int ld_sfa,
+                const uint8_t* B, const float* sfb,
+                const void* C, int c_kind, double* R,
+                int M, int N, int K, const int* rows, int n_rows);
+
+/*
+ * M-grouped contiguous: A [Mt][K], sfa [K/128][ld_sfa], B [G][N][K],
+ * sfb [G][ceil(N/128)][K/128], m_indices [Mt] (expert id, -1 = padding),
+ * C [Mt][N] (nullable), R [n_rows][N]. Padding rows come back as NaN.
+ */
+int dgo_m_grouped_contiguous(const uint8_t* A, const float* sfa, int ld_sfa,
+                             const uint8_t* B, const float* sfb,
+                             const int32_t* m_indices, const void* C, int c_kind,
+                             double* R, int Mt, int N, int K, int G,
+                             const int* rows, int n_rows);
+
+/*
+ * M-grouped masked: A [G][max_m][K], sfa [G][K/128][ld_sfa], B [G][N][K],
+ * sfb [G][ceil(N/128)][K/128], masked_m [G]; R [G][max_m][N] with rows
+ * m >= masked_m[g] set to NaN (not computed). If row_stride > 1 only every
+ * row_stride-th valid row (starting at row 0) is computed, the others NaN.
+ */
+int dgo_m_grouped_masked(const uint8_t* A, const float* sfa, int ld_sfa,
+                         const uint8_t* B, const float* sfb,
+                         const int32_t* masked_m, double* R,
+                         int G, int max_m, int N, int K, int row_stride);
+
+/*
+ * K-grouped TN: A [sumK][M], B [sumK][N] (both M/N contiguous),
+ * sfa [sumK/128][M], sfb [sumK/128][N], ks[G] (multiples of 128, may be 0).
+ * R_g[m][n] = C_g[m][n] + sum_{kb in g} sfa[kb][m] * sfb[kb][n] *
+ *             sum_{k in kb} dec(A[k][m]) * dec(B[k][n]).
+ * C [G][M][N] float (nullable); R [G][n_rows][N] for the selected rows.
+ */
+int dgo_k_grouped_tn(const uint8_t* A, const float* sfa, const uint8_t* B,
+                     const float* sfb, const int* ks, const float* C,
+                     double* R, int G, int M, int N,
+                     const int* rows, int n_rows);
+
+/* 1 - 2*sum(D*R) / sum(D^2 + R^2) over pairs where R is not NaN; 0 if the
+ * denominator is 0. */
+double dgo_calc_diff(const double* D, const double* R, size_t n);
+
+/* Threads the oracle's OpenMP loops use. */
+int dgo_num_threads(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
