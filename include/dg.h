@@ -1,0 +1,182 @@
+/*
+ * dg.h -- C ABI of libdg.so: FP8 (E4M3) GEMMs with fine-grained FP32 scaling
+ * and two-level (promoted) accumulation, for NVIDIA B200 (sm_100a).
+ *
+ * Operation (DeepGEMM README summary, ja.news.hada.io topic 19459, section
+ * "GEMMインターフェースとレイアウト制約"): D = C + A @ B.T, with NT as the base
+ * layout; scaling factors are FP32 and the LHS scales are stored transposed
+ * (MN-major) with a TMA-aligned leading dimension. Scale granularity: one
+ * scale per 1x128 K-strip of A and per 128x128 block of B; the per-K-block
+ * tensor-core partial sums are promoted into an FP32 accumulator with
+ * sfa * sfb applied ("DeepSeek開源新突破：DeepGEMM庫揭秘", paragraph 2: two-level
+ * accumulation because the FP8 tensor-core accumulator is imprecise).
+ *
+ * Conventions for every entry point below:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never frees or retains them. Row-major, densely packed, unless
+ *     a leading dimension is stated.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *     asynchronous on it: no host synchronisation, no device-to-host reads,
+ *     no memory allocation. They are therefore safe to capture in a CUDA graph.
+ *   - Every base pointer must be 16-byte aligned. Arguments are validated on
+ *     the host before anything is launched; a violation returns an error code
+ *     and launches nothing.
+ *   - Device-side waits are bounded: a wait that exceeds the timeout (default
+ *     2 s) records DG_ERR_TIMEOUT in a per-device error word, and the kernel
+ *     exits cleanly; read it with dg_get_last_device_error().
+ *   - E4M3 bytes are the OCP OFP8 "E4M3FN" encoding (torch.float8_e4m3fn).
+ */
+#ifndef DG_H
+#define DG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum */
+  DG_ERR_UNSUPPORTED_SHAPE = 2, /* K % 128 != 0, N % 8 != 0, too many groups, ... */
+  DG_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+  DG_ERR_CUDA = 4,              /* a CUDA runtime / driver call failed */
+  DG_ERR_TIMEOUT = 5            /* a bounded device wait ran out (see above) */
+} dg_status;
+
+/* Human-readable name of a status code (static string). */
+const char* dg_status_string(dg_status s);
+
+/* ---------------------------------------------------------------------------
+ * Quantiser: BF16/FP32 -> E4M3 codes + FP32 scales.
+ * Source: same README summary, section "GEMMインターフェースとレイアウト制約"
+ * (casting and scale layout are the caller's job; the library ships helpers),
+ * and the scale rule fixed for this library: scale = max(amax, 1e-4f) / 448,
+ * code = E4M3_RN_satfinite(x / scale), both IEEE FP32 divisions.
+ *
+ *   x       [batch][rows][cols], FP32 (in_dtype = DG_IN_F32) or BF16
+ *           (DG_IN_BF16). Read only.
+ *   codes   [batch][rows][cols] E4M3 bytes (written).
+ *   scales  written per mode:
+ *     DG_QUANT_ROW_1x128     one per (row, 128-col strip): cols % 128 == 0;
+ *                            scales[b][cols/128][ld_scales], transposed
+ *                            (MN-major); ld_scales >= rows, ld_scales % 4 == 0.
+ *                            This is the sfa layout every NT GEMM below reads.
+ *     DG_QUANT_BLOCK_128x128 one per 128x128 block, rows may be ragged:
+ *                            scales[b][ceil(rows/128)][cols/128]; cols % 128
+ *                            == 0; ld_scales ignored. This is the sfb layout.
+ *     DG_QUANT_COL_128x1     one per (128-row strip, column): rows % 128 == 0;
+ *                            scales[b][rows/128][cols]; ld_scales ignored.
+ *                            This is the layout the K-grouped TN GEMM reads.
+ *   amax is taken over the elements that exist (a ragged last block reads only
+ *   its real rows).
+ * ------------------------------------------------------------------------- */
+enum { DG_IN_F32 = 0, DG_IN_BF16 = 1 };
+enum { DG_QUANT_ROW_1x128 = 0, DG_QUANT_BLOCK_128x128 = 1, DG_QUANT_COL_128x1 = 2 };
+
+dg_status dg_quantize_fp8(const void* x, int in_dtype, int batch, int rows, int cols,
+                          int mode, void* codes, float* scales, int ld_scales,
+                          void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Dense NT GEMM: D[m][n] = C[m][n] + sum_kb sfa[kb][m] * sfb[n/128][kb] *
+ *                          sum_{k in kb} A[m][k] * B[n][k]
+ * Source: README summary, "GEMMインターフェースとレイアウト制約" (fp8_gemm_nt).
+ *
+ *   A    [M][K] E4M3            sfa [K/128][align4(M)] FP32 (ROW_1x128 layout)
+ *   B    [N][K] E4M3            sfb [ceil(N/128)][K/128] FP32 (BLOCK layout)
+ *   C    [M][N] BF16 or NULL (C may alias D)
+ *   D    [M][N] BF16, rounded to nearest even from the FP32 accumulator.
+ * Shapes: M >= 0, N >= 0 (either 0: no-op), K % 128 == 0 (K == 0: D = C),
+ * N % 8 == 0.
+ * ------------------------------------------------------------------------- */
+dg_status dg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb,
+                         const void* C, void* D, int M, int N, int K, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * M-grouped GEMM, contiguous layout (MoE prefill / training forward).
+ * Source: README summary, section "DenseとGrouped GEMM": experts share N and K;
+ * each expert's tokens are concatenated along M, each segment aligned to the
+ * M block size (dg_get_mk_alignment_for_contiguous_layout()).
+ *
+ *   A         [Mt][K] E4M3, Mt % 128 == 0
+ *   sfa       [K/128][align4(Mt)] FP32
+ *   B         [G][N][K] E4M3      sfb [G][ceil(N/128)][K/128] FP32
+ *   m_indices [Mt] int32 device array: expert id of each row, -1 on padding.
+ *             Each 128-row block must belong to a single expert (or be all
+ *             padding). A block whose first row is -1 is skipped entirely.
+ *   C         [Mt][N] BF16 or NULL     D [Mt][N] BF16
+ * Rows with m_indices == -1 (and rows whose id is >= G) are left untouched.
+ * ------------------------------------------------------------------------- */
+dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void* A, const float* sfa, const void* B,
+                                              const float* sfb, const int32_t* m_indices,
+                                              const void* C, void* D, int Mt, int N, int K,
+                                              int G, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * M-grouped GEMM, masked layout (MoE decode under CUDA graphs, where the host
+ * does not know per-expert token counts).
+ * Source: README summary, "DenseとGrouped GEMM" (m_grouped_fp8_gemm_nt_masked:
+ * given a mask tensor the kernel computes only the valid region).
+ *
+ *   A        [G][max_m][K] E4M3     sfa [G][K/128][align4(max_m)] FP32
+ *   B        [G][N][K] E4M3         sfb [G][ceil(N/128)][K/128] FP32
+ *   masked_m [G] int32 device array, read on the device; values are clamped
+ *            to [0, max_m].
+ *   D        [G][max_m][N] BF16; rows m >= masked_m[g] are left untouched.
+ * G <= 1024.
+ * ------------------------------------------------------------------------- */
+dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* A, const float* sfa, const void* B,
+                                          const float* sfb, const int32_t* masked_m, void* D,
+                                          int G, int max_m, int N, int K, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * K-grouped GEMM, TN, contiguous along K (MoE weight gradient).
+ * Source: README summary, "DenseとGrouped GEMM" (k_grouped_fp8_gemm_tn_contiguous:
+ * M and N fixed, groups along K). Reading of "TN": both operands are stored
+ * K-outer (M or N contiguous), groups concatenated along K.
+ *
+ *   A      [sumK][M] E4M3   sfa [sumK/128][M] FP32 (COL_128x1 layout)
+ *   B      [sumK][N] E4M3   sfb [sumK/128][N] FP32 (COL_128x1 layout)
+ *   ks     HOST array of G per-group K sizes, each a multiple of 128 (0
+ *          allowed); read during the call only.
+ *   C      [G][M][N] FP32 or NULL (may alias D)     D [G][M][N] FP32
+ *   D_g[m][n] = C_g[m][n] + sum_{kb in group g} sfa[kb][m] * sfb[kb][n] *
+ *               sum_{k in kb} A[k][m] * B[k][n]
+ * M % 16 == 0, N % 16 == 0, 1 <= G <= 256.
+ * ------------------------------------------------------------------------- */
+dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void* A, const float* sfa, const void* B,
+                                              const float* sfb, const int* ks, const float* C,
+                                              float* D, int G, int M, int N, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Utilities (README summary, section "ユーティリティと環境変数").
+ * ------------------------------------------------------------------------- */
+/* M alignment every contiguous-layout segment must have: 128. */
+int dg_get_mk_alignment_for_contiguous_layout(void);
+/* Smallest x >= mn with x * elem_bytes a multiple of 16 (TMA row alignment). */
+int dg_get_tma_aligned_size(int mn, int elem_bytes);
+/* Cap on the SMs the GEMM kernels use (0 = all SMs of the device). */
+void dg_set_num_sms(int n);
+int dg_get_num_sms(void);
+/* Bounded-wait limit in nanoseconds for subsequent launches (0 = default 2 s). */
+void dg_set_wait_timeout_ns(uint64_t ns);
+
+/* Synchronises `stream`, then reads and clears this device's error word.
+ * Returns DG_OK, DG_ERR_TIMEOUT (a bounded wait ran out; *site gets the code
+ * of the wait that gave up, if site != NULL) or DG_ERR_CUDA. Debug/test use. */
+dg_status dg_get_last_device_error(void* stream, int* site);
+
+/* Test hook: when nonzero, the next GEMM launch drops one producer arrive so
+ * that its consumers' bounded waits run out (used to test the timeout path).
+ * Reset to 0 after one launch. */
+void dg_debug_drop_next_arrive(int enable);
+
+/* Number of kernels this library has launched since load (all devices). */
+uint64_t dg_get_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DG_H */

@@ -1,0 +1,445 @@
+// dg_api.cu -- host side of libdg.so: argument validation, the per-shape
+// planner (tile width, grid size), TMA tensor-map encoding and kernel launch
+// for every entry point declared in include/dg.h. All device code of the
+// library is compiled in this one translation unit.
+#include <atomic>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/dg.h"
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
+
+namespace {
+
+using dg::GemmArgs;
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_num_sms_cap{0};
+std::atomic<unsigned long long> g_timeout_ns{0};
+std::atomic<int> g_drop_next{0};
+std::atomic<uint64_t> g_launches{0};
+
+int g_sm_count[kMaxDevices];
+std::once_flag g_sm_once[kMaxDevices];
+
+bool print_configs() {
+  static const bool on = [] {
+    const char* e = std::getenv("DG_PRINT_CONFIGS");
+    return e && e[0] && e[0] != '0';
+  }();
+  return on;
+}
+
+dg_status cuda_fail(cudaError_t e, const char* what) {
+  if (print_configs()) std::fprintf(stderr, "[dg] %s: %s\n", what, cudaGetErrorString(e));
+  return DG_ERR_CUDA;
+}
+
+dg_status device_sms(int* dev, int* sms) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (*dev < 0 || *dev >= kMaxDevices) return DG_ERR_CUDA;
+  std::call_once(g_sm_once[*dev], [d = *dev] {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d);
+    g_sm_count[d] = n;
+  });
+  int n = g_sm_count[*dev];
+  if (n <= 0) return DG_ERR_CUDA;
+  const int cap = g_num_sms_cap.load();
+  *sms = (cap > 0 && cap < n) ? cap : n;
+  return DG_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+unsigned long long timeout_ns() {
+  const unsigned long long t = g_timeout_ns.load();
+  return t ? t : 2000000000ull;
+}
+
+// ---------------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 2-D row-major tensor: `inner` contiguous elements per row, `outer` rows,
+// row pitch `pitch_bytes`; box {box_inner, box_outer}.
+dg_status make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner,
+                      uint64_t outer, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+                      CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return DG_ERR_CUDA;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    if (print_configs()) std::fprintf(stderr, "[dg] cuTensorMapEncodeTiled failed: %d\n", (int)r);
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
+}
+
+// ---------------------------------------------------------------- launches
+template <int MODE, int BN>
+dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
+                      const CUtensorMap& tsb, const GemmArgs& args, int grid, cudaStream_t st,
+                      int dev) {
+  using Cfg = dg::GemmCfg<MODE, BN>;
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t attr_err[kMaxDevices];
+  auto kern = dg::gemm_fp8_kernel<MODE, BN>;
+  std::call_once(once[dev], [&] {
+    attr_err[dev] =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+  });
+  if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(ta, tb, tsa, tsb, args);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  g_launches.fetch_add(1);
+  return DG_OK;
+}
+
+int take_drop_flag() { return g_drop_next.exchange(0); }
+
+// Tile width: 256 columns unless that leaves the GPU with clearly fewer
+// waves' worth of work than 128-column tiles (a 128-wide tile costs about half
+// of a 256-wide one, with ~15% lower per-tile efficiency).
+int choose_bn(long long m_blocks, int N, int sms) {
+  const long long t256 = m_blocks * ((N + 255) / 256);
+  const long long t128 = m_blocks * ((N + 127) / 128);
+  const double c256 = 2.0 * static_cast<double>((t256 + sms - 1) / sms);
+  const double c128 = 1.15 * static_cast<double>((t128 + sms - 1) / sms);
+  return c128 < c256 ? 128 : 256;
+}
+
+// D = C (or 0) for K == 0 / all-empty K-grouped problems.
+template <typename T>
+__global__ void copy_or_zero_kernel(const T* __restrict__ c, T* __restrict__ d, long long n) {
+  for (long long i = blockIdx.x * 1ll * blockDim.x + threadIdx.x; i < n;
+       i += 1ll * gridDim.x * blockDim.x)
+    d[i] = c ? c[i] : T(0);
+}
+
+template <typename T>
+dg_status copy_or_zero(const void* c, void* d, long long n, int sms, cudaStream_t st) {
+  if (n <= 0) return DG_OK;
+  if (c == d) return DG_OK;
+  const int grid = static_cast<int>(std::min<long long>((n + 255) / 256, 8ll * sms));
+  copy_or_zero_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(c), static_cast<T*>(d), n);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "copy launch");
+  g_launches.fetch_add(1);
+  return DG_OK;
+}
+
+struct Bf16Raw {
+  uint16_t v;
+  __host__ __device__ Bf16Raw() : v(0) {}
+  __host__ __device__ explicit Bf16Raw(int) : v(0) {}
+};
+
+// Shared NT launcher for dense / contiguous / masked.
+template <int MODE>
+dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, const float* sfb,
+                 const int32_t* m_indices, const int32_t* masked_m, const void* C, void* D,
+                 int rows_total, int M_logical, int N, int K, int G, long long m_blocks_bound,
+                 long long tiles_if_known, cudaStream_t st, const char* name) {
+  int dev = 0, sms = 0;
+  dg_status s = device_sms(&dev, &sms);
+  if (s != DG_OK) return s;
+  const int bn = choose_bn(m_blocks_bound, N, sms);
+  CUtensorMap ta, tb, dummy;
+  std::memset(&dummy, 0, sizeof dummy);
+  s = make_map_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, rows_total, K, 128, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != DG_OK) return s;
+  s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, static_cast<uint64_t>(G) * N, K, 128,
+                  bn, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != DG_OK) return s;
+  GemmArgs args;
+  std::memset(&args, 0, sizeof args);
+  args.M = M_logical;
+  args.N = N;
+  args.K = K;
+  args.G = G;
+  args.num_m_blocks = static_cast<int>((MODE == dg::MODE_MASKED) ? (M_logical + 127) / 128
+                                                                  : (rows_total + 127) / 128);
+  args.num_n_blocks = (N + bn - 1) / bn;
+  const long long tiles = tiles_if_known >= 0
+                              ? tiles_if_known * args.num_n_blocks
+                              : m_blocks_bound * args.num_n_blocks;
+  args.total_tiles = static_cast<int>(tiles);
+  args.sfa = sfa;
+  args.ld_sfa = ld_sfa;
+  args.sfb = sfb;
+  args.m_indices = m_indices;
+  args.masked_m = masked_m;
+  args.C = C;
+  args.D = D;
+  args.timeout_ns = timeout_ns();
+  args.drop_arrive = take_drop_flag();
+  const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(sms, tiles)));
+  if (print_configs())
+    std::fprintf(stderr, "[dg] %s M=%d N=%d K=%d G=%d: BM=128 BN=%d tiles=%lld grid=%d\n", name,
+                 M_logical, N, K, G, bn, tiles, grid);
+  if (bn == 256) return launch_gemm<MODE, 256>(ta, tb, dummy, dummy, args, grid, st, dev);
+  return launch_gemm<MODE, 128>(ta, tb, dummy, dummy, args, grid, st, dev);
+}
+
+}  // namespace
+
+// =============================================================== C ABI
+extern "C" {
+
+const char* dg_status_string(dg_status s) {
+  switch (s) {
+    case DG_OK: return "DG_OK";
+    case DG_ERR_INVALID_ARG: return "DG_ERR_INVALID_ARG";
+    case DG_ERR_UNSUPPORTED_SHAPE: return "DG_ERR_UNSUPPORTED_SHAPE";
+    case DG_ERR_MISALIGNED: return "DG_ERR_MISALIGNED";
+    case DG_ERR_CUDA: return "DG_ERR_CUDA";
+    case DG_ERR_TIMEOUT: return "DG_ERR_TIMEOUT";
+  }
+  return "DG_ERR_UNKNOWN";
+}
+
+int dg_get_mk_alignment_for_contiguous_layout(void) { return 128; }
+
+int dg_get_tma_aligned_size(int mn, int elem_bytes) {
+  if (mn < 0 || elem_bytes <= 0 || 16 % elem_bytes != 0) return -1;
+  const int a = 16 / elem_bytes;
+  return (mn + a - 1) / a * a;
+}
+
+void dg_set_num_sms(int n) { g_num_sms_cap.store(n > 0 ? n : 0); }
+
+int dg_get_num_sms(void) {
+  int dev = 0, sms = 0;
+  if (device_sms(&dev, &sms) != DG_OK) return g_num_sms_cap.load();
+  return sms;
+}
+
+void dg_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns); }
+
+void dg_debug_drop_next_arrive(int enable) { g_drop_next.store(enable ? 1 : 0); }
+
+uint64_t dg_get_launch_count(void) { return g_launches.load(); }
+
+dg_status dg_get_last_device_error(void* stream, int* site) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int w[2] = {0, 0};
+  e = cudaMemcpyFromSymbol(w, dg::g_error_word, sizeof w);
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  const unsigned int z[2] = {0, 0};
+  e = cudaMemcpyToSymbol(dg::g_error_word, z, sizeof z);
+  if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+  if (site) *site = static_cast<int>(w[1]);
+  if (w[0] == 0) return DG_OK;
+  if (w[0] == static_cast<unsigned int>(DG_ERR_TIMEOUT)) return DG_ERR_TIMEOUT;
+  return DG_ERR_CUDA;
+}
+
+dg_status dg_quantize_fp8(const void* x, int in_dtype, int batch, int rows, int cols, int mode,
+                          void* codes, float* scales, int ld_scales, void* stream) {
+  if (batch < 0 || rows < 0 || cols < 0) return DG_ERR_INVALID_ARG;
+  if (in_dtype != DG_IN_F32 && in_dtype != DG_IN_BF16) return DG_ERR_INVALID_ARG;
+  if (mode < DG_QUANT_ROW_1x128 || mode > DG_QUANT_COL_128x1) return DG_ERR_INVALID_ARG;
+  if (mode == DG_QUANT_ROW_1x128 || mode == DG_QUANT_BLOCK_128x128) {
+    if (cols % 128 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  } else {
+    if (rows % 128 != 0 || cols % 4 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (mode == DG_QUANT_ROW_1x128 && (ld_scales < rows || ld_scales % 4 != 0))
+    return DG_ERR_INVALID_ARG;
+  if (static_cast<long long>(batch) * rows * cols == 0) return DG_OK;
+  if (!x || !codes || !scales) return DG_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return DG_ERR_MISALIGNED;
+  int dev = 0, sms = 0;
+  dg_status s = device_sms(&dev, &sms);
+  if (s != DG_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* q = static_cast<uint8_t*>(codes);
+  const bool bf = in_dtype == DG_IN_BF16;
+  if (mode == DG_QUANT_ROW_1x128) {
+    const long long strips = static_cast<long long>(batch) * rows * (cols / 128);
+    const int grid = static_cast<int>(std::min<long long>((strips + 7) / 8, 8ll * sms));
+    if (bf) dg::quant_row_kernel<true><<<grid, 256, 0, st>>>(x, batch, rows, cols, q, scales, ld_scales);
+    else dg::quant_row_kernel<false><<<grid, 256, 0, st>>>(x, batch, rows, cols, q, scales, ld_scales);
+  } else if (mode == DG_QUANT_BLOCK_128x128) {
+    const long long blocks = static_cast<long long>(batch) * ((rows + 127) / 128) * (cols / 128);
+    if (blocks > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
+    if (bf) dg::quant_block_kernel<true><<<static_cast<int>(blocks), 256, 0, st>>>(x, batch, rows, cols, q, scales);
+    else dg::quant_block_kernel<false><<<static_cast<int>(blocks), 256, 0, st>>>(x, batch, rows, cols, q, scales);
+  } else {
+    const long long blocks = static_cast<long long>(batch) * (rows / 128) * ((cols + 63) / 64);
+    if (blocks > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
+    if (bf) dg::quant_col_kernel<true><<<static_cast<int>(blocks), 256, 0, st>>>(x, batch, rows, cols, q, scales);
+    else dg::quant_col_kernel<false><<<static_cast<int>(blocks), 256, 0, st>>>(x, batch, rows, cols, q, scales);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  g_launches.fetch_add(1);
+  return DG_OK;
+}
+
+dg_status dg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb,
+                         const void* C, void* D, int M, int N, int K, void* stream) {
+  if (M < 0 || N < 0 || K < 0) return DG_ERR_INVALID_ARG;
+  if (K % 128 != 0 || N % 8 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return DG_OK;
+  if (!D) return DG_ERR_INVALID_ARG;
+  if (!aligned16(D) || (C && !aligned16(C))) return DG_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (K == 0) {
+    int dev = 0, sms = 0;
+    dg_status s = device_sms(&dev, &sms);
+    if (s != DG_OK) return s;
+    return copy_or_zero<Bf16Raw>(C, D, static_cast<long long>(M) * N, sms, st);
+  }
+  if (!A || !B || !sfa || !sfb) return DG_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(sfa) || !aligned16(sfb))
+    return DG_ERR_MISALIGNED;
+  const int ld = (M + 3) / 4 * 4;
+  const long long mb = (M + 127) / 128;
+  return run_nt<dg::MODE_DENSE>(A, sfa, ld, B, sfb, nullptr, nullptr, C, D, M, M, N, K, 1, mb, mb,
+                                st, "fp8_gemm_nt");
+}
+
+dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void* A, const float* sfa, const void* B,
+                                              const float* sfb, const int32_t* m_indices,
+                                              const void* C, void* D, int Mt, int N, int K, int G,
+                                              void* stream) {
+  if (Mt < 0 || N < 0 || K < 0 || G < 1) return DG_ERR_INVALID_ARG;
+  if (Mt % 128 != 0 || K % 128 != 0 || N % 8 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  if (Mt == 0 || N == 0) return DG_OK;
+  if (!D || !m_indices) return DG_ERR_INVALID_ARG;
+  if (K == 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  if (!A || !B || !sfa || !sfb) return DG_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(sfa) || !aligned16(sfb) || !aligned16(D) ||
+      !aligned16(m_indices) || (C && !aligned16(C)))
+    return DG_ERR_MISALIGNED;
+  if (static_cast<long long>(G) * N > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
+  const long long mb = Mt / 128;
+  return run_nt<dg::MODE_CONTIG>(A, sfa, Mt, B, sfb, m_indices, nullptr, C, D, Mt, Mt, N, K, G, mb,
+                                 mb, static_cast<cudaStream_t>(stream),
+                                 "m_grouped_fp8_gemm_nt_contiguous");
+}
+
+dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* A, const float* sfa, const void* B,
+                                          const float* sfb, const int32_t* masked_m, void* D,
+                                          int G, int max_m, int N, int K, void* stream) {
+  if (G < 1 || max_m < 0 || N < 0 || K < 0) return DG_ERR_INVALID_ARG;
+  if (G > dg::kMaxMaskedGroups || K % 128 != 0 || N % 8 != 0 || K == 0)
+    return DG_ERR_UNSUPPORTED_SHAPE;
+  if (max_m == 0 || N == 0) return DG_OK;
+  if (!A || !B || !sfa || !sfb || !masked_m || !D) return DG_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(sfa) || !aligned16(sfb) || !aligned16(D) ||
+      !aligned16(masked_m))
+    return DG_ERR_MISALIGNED;
+  if (static_cast<long long>(G) * max_m > 0x7fffffffll ||
+      static_cast<long long>(G) * N > 0x7fffffffll)
+    return DG_ERR_UNSUPPORTED_SHAPE;
+  const int ld = (max_m + 3) / 4 * 4;
+  const long long mb_bound = static_cast<long long>(G) * ((max_m + 127) / 128);
+  return run_nt<dg::MODE_MASKED>(A, sfa, ld, B, sfb, nullptr, masked_m, nullptr, D, G * max_m,
+                                 max_m, N, K, G, mb_bound, -1, static_cast<cudaStream_t>(stream),
+                                 "m_grouped_fp8_gemm_nt_masked");
+}
+
+dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void* A, const float* sfa, const void* B,
+                                              const float* sfb, const int* ks, const float* C,
+                                              float* D, int G, int M, int N, void* stream) {
+  if (G < 1 || M < 0 || N < 0 || !ks) return DG_ERR_INVALID_ARG;
+  if (G > dg::kMaxKGroups || M % 16 != 0 || N % 16 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  long long sumK = 0;
+  for (int g = 0; g < G; ++g) {
+    if (ks[g] < 0) return DG_ERR_INVALID_ARG;
+    if (ks[g] % 128 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+    sumK += ks[g];
+  }
+  if (sumK > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return DG_OK;
+  if (!D) return DG_ERR_INVALID_ARG;
+  if (!aligned16(D) || (C && !aligned16(C))) return DG_ERR_MISALIGNED;
+  int dev = 0, sms = 0;
+  dg_status s = device_sms(&dev, &sms);
+  if (s != DG_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (sumK == 0) return copy_or_zero<float>(C, D, static_cast<long long>(G) * M * N, sms, st);
+  if (!A || !B || !sfa || !sfb) return DG_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(sfa) || !aligned16(sfb))
+    return DG_ERR_MISALIGNED;
+  const int mb = (M + 127) / 128;
+  const int bn = choose_bn(static_cast<long long>(G) * mb, N, sms);
+  const uint64_t sumKB = static_cast<uint64_t>(sumK / 128);
+  CUtensorMap ta, tb, tsa, tsb;
+  if ((s = make_map_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, M, sumK, M, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  if ((s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, sumK, N, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  if ((s = make_map_2d(&tsa, sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, sumKB, 4ull * M, 128, 1,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
+    return s;
+  if ((s = make_map_2d(&tsb, sfb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, sumKB, 4ull * N, bn, 1,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
+    return s;
+  GemmArgs args;
+  std::memset(&args, 0, sizeof args);
+  args.M = M;
+  args.N = N;
+  args.K = 0;
+  args.G = G;
+  args.num_m_blocks = mb;
+  args.num_n_blocks = (N + bn - 1) / bn;
+  const long long tiles = static_cast<long long>(G) * mb * args.num_n_blocks;
+  args.total_tiles = static_cast<int>(tiles);
+  args.C = C;
+  args.D = D;
+  args.timeout_ns = timeout_ns();
+  args.drop_arrive = take_drop_flag();
+  int acc = 0;
+  for (int g = 0; g < G; ++g) {
+    args.kb_off[g] = acc;
+    acc += ks[g] / 128;
+  }
+  args.kb_off[G] = acc;
+  const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(sms, tiles)));
+  if (print_configs())
+    std::fprintf(stderr, "[dg] k_grouped_fp8_gemm_tn M=%d N=%d sumK=%lld G=%d: BN=%d tiles=%lld grid=%d\n",
+                 M, N, sumK, G, bn, tiles, grid);
+  if (bn == 256) return launch_gemm<dg::MODE_KGROUPED, 256>(ta, tb, tsa, tsb, args, grid, st, dev);
+  return launch_gemm<dg::MODE_KGROUPED, 128>(ta, tb, tsa, tsb, args, grid, st, dev);
+}
+
+}  // extern "C"

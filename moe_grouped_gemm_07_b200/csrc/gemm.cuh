@@ -1,0 +1,573 @@
+// gemm.cuh -- persistent, warp-specialised FP8 GEMM with per-K-block FP32
+// promotion for sm_100a (B200).
+//
+// Operation (DeepGEMM README summary, section "GEMMインターフェースとレイアウト制約"):
+//   D = C + A @ B.T, E4M3 operands, FP32 scales per 1x128 strip of A and per
+//   128x128 block of B (or per column for the K-grouped TN variant).
+// Promotion (picoinsstore DeepGEMM article, paragraph 2): the tensor core's
+// partial sum over each 128-wide K-block is NOT carried across K-blocks;
+// it is read out of TMEM and accumulated in FP32 registers with the scales
+// applied: acc += sfa * sfb * P_kb.
+//
+// CTA = 320 threads, one CTA per SM, persistent over output tiles:
+//   warp 0      TMA producer: A/B tiles (128B-swizzled) into an S-stage ring
+//               (plus, for K-grouped, the per-K-block scale vectors).
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer: for each
+//               K-block, 4 x (M=128, N=BN, K=32) MMAs into one of two TMEM
+//               accumulator buffers (2 x BN columns), reset per K-block.
+//   warps 2..9  promotion / epilogue: warp w reads TMEM lane quadrant (w % 4)
+//               and column half ((w - 2) / 4); acc += s * P in registers;
+//               at tile end adds C, converts and stores D.
+// The MMA of K-block j+1 overlaps the promotion of K-block j (double-buffered
+// TMEM); the producer runs up to S K-blocks ahead.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace dg {
+
+enum GemmMode : int { MODE_DENSE = 0, MODE_CONTIG = 1, MODE_MASKED = 2, MODE_KGROUPED = 3 };
+
+constexpr int kMaxKGroups = 256;
+constexpr int kMaxMaskedGroups = 1024;
+
+struct GemmArgs {
+  int M, N, K;     // dense: M; contiguous: Mt; masked: max_m; K-grouped: M (K unused)
+  int G;
+  int num_m_blocks, num_n_blocks;
+  int total_tiles;  // host-known tile count (masked: upper bound, recomputed on device)
+  const float* sfa;
+  int ld_sfa;
+  const float* sfb;
+  const int32_t* m_indices;
+  const int32_t* masked_m;
+  const void* C;
+  void* D;
+  unsigned long long timeout_ns;
+  int drop_arrive;
+  int kb_off[kMaxKGroups + 1];  // K-grouped: prefix sums of K-blocks per group
+};
+
+template <int MODE, int BN_>
+struct GemmCfg {
+  static constexpr int BM = 128;
+  static constexpr int BN = BN_;
+  static constexpr int BK = 128;  // FP8 elements (= bytes) per K-block
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int SCALE_SLOTS = 8;  // K-grouped only
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int SCALE_BYTES = (BM + BN) * 4;
+  static constexpr int THREADS = 320;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int EPI_COLS = BN / 2;  // accumulator columns per promotion thread
+  static constexpr int GROUP_M = 16;       // tile rasterisation group (L2 reuse)
+  static constexpr bool KG = MODE == MODE_KGROUPED;
+  // shared memory carve-up (offsets from a 1024-byte aligned base)
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_SCALE = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_BAR = OFF_SCALE + (KG ? SCALE_SLOTS * SCALE_BYTES : 0);
+  static constexpr int NUM_BARS = 2 * STAGES + 4 + 2 * SCALE_SLOTS + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;       // tmem slot, abort flag
+  static constexpr int OFF_PREFIX = OFF_MISC + 16;              // masked: prefix + counts
+  static constexpr int PREFIX_BYTES = MODE == MODE_MASKED ? (2 * kMaxMaskedGroups + 1) * 4 : 0;
+  static constexpr int SMEM_BYTES = OFF_PREFIX + PREFIX_BYTES + 1024;  // + alignment slack
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(BN == 128 || BN == 256, "BN");
+};
+
+struct Tile {
+  int valid;
+  int g;
+  int m0;        // first row of the tile in its group's row space
+  int n0;        // first column
+  int a_row;     // NT: TMA row (y) of A; K-grouped: TMA x of A (= m0)
+  int b_row;     // NT: TMA row (y) of B; K-grouped: TMA x of B (= n0)
+  int kb0, nkb;  // K-blocks [kb0, kb0 + nkb) along the K axis of the operands
+  int rows;      // rows of this tile that may be written (before per-row checks)
+  long long out_row0;  // row of D holding tile row 0
+};
+
+// Tile t -> coordinates. Every role calls this with identical inputs, so all
+// roles walk the same tile sequence.
+template <int MODE, int BN>
+__device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int* prefix,
+                                            const int* mm_clamped) {
+  using Cfg = GemmCfg<MODE, BN>;
+  Tile tl;
+  tl.valid = 1;
+  tl.kb0 = 0;
+  tl.nkb = a.K / Cfg::BK;
+  if constexpr (MODE == MODE_DENSE || MODE == MODE_CONTIG) {
+    const int group_tiles = Cfg::GROUP_M * a.num_n_blocks;
+    const int grp = t / group_tiles;
+    const int first_m = grp * Cfg::GROUP_M;
+    const int gm = min(a.num_m_blocks - first_m, Cfg::GROUP_M);
+    const int local = t - grp * group_tiles;
+    const int mb = first_m + local % gm;
+    const int nb = local / gm;
+    tl.m0 = mb * Cfg::BM;
+    tl.n0 = nb * BN;
+    tl.a_row = tl.m0;
+    tl.out_row0 = tl.m0;
+    if constexpr (MODE == MODE_DENSE) {
+      tl.g = 0;
+      tl.b_row = tl.n0;
+      tl.rows = min(Cfg::BM, a.M - tl.m0);
+    } else {
+      const int g = __ldg(a.m_indices + tl.m0);
+      tl.g = g;
+      tl.valid = (g >= 0 && g < a.G);
+      tl.b_row = g * a.N + tl.n0;
+      tl.rows = Cfg::BM;
+    }
+  } else if constexpr (MODE == MODE_MASKED) {
+    // largest g with prefix[g] <= t
+    int lo = 0, hi = a.G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    const int g = lo;
+    const int cnt = (prefix[g + 1] - prefix[g]) / a.num_n_blocks;  // m-blocks of group g
+    const int local = t - prefix[g];
+    const int mb = local % cnt;
+    const int nb = local / cnt;
+    tl.g = g;
+    tl.m0 = mb * Cfg::BM;
+    tl.n0 = nb * BN;
+    tl.a_row = g * a.M + tl.m0;
+    tl.b_row = g * a.N + tl.n0;
+    tl.rows = min(Cfg::BM, mm_clamped[g] - tl.m0);
+    tl.out_row0 = static_cast<long long>(g) * a.M + tl.m0;
+  } else {  // K-grouped
+    const int per_g = a.num_m_blocks * a.num_n_blocks;
+    const int g = t / per_g;
+    const int local = t - g * per_g;
+    const int group_tiles = Cfg::GROUP_M * a.num_n_blocks;
+    const int grp = local / group_tiles;
+    const int first_m = grp * Cfg::GROUP_M;
+    const int gm = min(a.num_m_blocks - first_m, Cfg::GROUP_M);
+    const int l2 = local - grp * group_tiles;
+    const int mb = first_m + l2 % gm;
+    const int nb = l2 / gm;
+    tl.g = g;
+    tl.m0 = mb * Cfg::BM;
+    tl.n0 = nb * BN;
+    tl.a_row = tl.m0;
+    tl.b_row = tl.n0;
+    tl.kb0 = a.kb_off[g];
+    tl.nkb = a.kb_off[g + 1] - a.kb_off[g];
+    tl.rows = min(Cfg::BM, a.M - tl.m0);
+    tl.out_row0 = static_cast<long long>(g) * a.M + tl.m0;
+  }
+  return tl;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half)
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// Site codes reported with DG_ERR_TIMEOUT.
+enum : unsigned int {
+  SITE_PRODUCER_EMPTY = 1,
+  SITE_PRODUCER_SCALE_EMPTY = 2,
+  SITE_MMA_TMEM_EMPTY = 3,
+  SITE_MMA_FULL = 4,
+  SITE_EPI_TMEM_FULL = 5,
+  SITE_EPI_SCALE_FULL = 6,
+  SITE_TEARDOWN_TMA = 7,
+  SITE_TEARDOWN_MMA = 8,
+};
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(320, 1)
+    gemm_fp8_kernel(const __grid_constant__ CUtensorMap tm_a,
+                    const __grid_constant__ CUtensorMap tm_b,
+                    const __grid_constant__ CUtensorMap tm_sfa,
+                    const __grid_constant__ CUtensorMap tm_sfb,
+                    const __grid_constant__ GemmArgs args) {
+  using Cfg = GemmCfg<MODE, BN>;
+  constexpr int S = Cfg::STAGES;
+  constexpr int SS = Cfg::SCALE_SLOTS;
+  constexpr int EC = Cfg::EPI_COLS;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sA = smem + Cfg::OFF_A;
+  uint8_t* sB = smem + Cfg::OFF_B;
+  float* sScale = reinterpret_cast<float*>(smem + Cfg::OFF_SCALE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint64_t* sfull = bars + 2 * S + 4;
+  uint64_t* sempty = bars + 2 * S + 4 + SS;
+  uint64_t* mma_done = bars + 2 * S + 4 + 2 * SS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
+  int* prefix = reinterpret_cast<int*>(smem + Cfg::OFF_PREFIX);
+  int* mm_clamped = prefix + kMaxMaskedGroups + 1;
+
+  const uint32_t warp = warp_id_uniform();
+  const uint32_t lane = lane_id();
+  const uint64_t tmo = args.timeout_ns;
+
+  // ---------------------------------------------------------------- set-up
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);
+    }
+    for (int i = 0; i < SS; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&sempty[i], 8);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+    if constexpr (Cfg::KG) {
+      tma_prefetch_desc(&tm_sfa);
+      tma_prefetch_desc(&tm_sfb);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  int total_tiles = args.total_tiles;
+  if constexpr (MODE == MODE_MASKED) {
+    if (warp == 2) {
+      int carry = 0;
+      for (int base = 0; base < args.G; base += 32) {
+        const int g = base + lane;
+        int mm = 0, v = 0;
+        if (g < args.G) {
+          mm = min(max(__ldg(args.masked_m + g), 0), args.M);
+          v = ((mm + Cfg::BM - 1) / Cfg::BM) * args.num_n_blocks;
+          mm_clamped[g] = mm;
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= static_cast<uint32_t>(o)) v += y;
+        }
+        if (g < args.G) prefix[g + 1] = carry + v;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+      }
+      if (lane == 0) prefix[0] = 0;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  if constexpr (MODE == MODE_MASKED) total_tiles = prefix[args.G];
+
+  // ---------------------------------------------------------------- roles
+  if (warp == 0) {
+    // ======================= TMA producer (one thread) =======================
+    if (lane == 0) {
+      uint32_t it = 0, sit = 0;
+      int dropped = -1;
+      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped);
+        if (!tl.valid) continue;
+        for (int kb = 0; kb < tl.nkb; ++kb, ++it) {
+          const uint32_t s = it % S;
+          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort_flag, tmo, SITE_PRODUCER_EMPTY))
+            goto producer_done;
+          if constexpr (Cfg::KG) {
+            // take the scale slot before arming anything, so an abort here
+            // leaves no uncounted copy in flight
+            const uint32_t ss = sit % SS;
+            if (!mbar_wait(&sempty[ss], ((sit / SS) & 1) ^ 1, abort_flag, tmo,
+                           SITE_PRODUCER_SCALE_EMPTY))
+              goto producer_done;
+          }
+          if (args.drop_arrive && it == 0) {  // test hook: never arm stage 0
+            dropped = 0;
+          } else {
+            mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES);
+            const int kk = (tl.kb0 + kb) * Cfg::BK;
+            if constexpr (Cfg::KG) {
+              tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], tl.a_row, kk);
+#pragma unroll
+              for (int h = 0; h < BN / 128; ++h)
+                tma_load_2d(sB + s * Cfg::B_BYTES + h * 128 * Cfg::BK, &tm_b, &full[s],
+                            tl.b_row + h * 128, kk);
+            } else {
+              tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], kk, tl.a_row);
+              tma_load_2d(sB + s * Cfg::B_BYTES, &tm_b, &full[s], kk, tl.b_row);
+            }
+          }
+          if constexpr (Cfg::KG) {
+            const uint32_t ss = sit % SS;
+            mbar_arrive_expect_tx(&sfull[ss], Cfg::SCALE_BYTES);
+            float* slot = sScale + ss * (Cfg::BM + BN);
+            tma_load_2d(slot, &tm_sfa, &sfull[ss], tl.m0, tl.kb0 + kb);
+            tma_load_2d(slot + Cfg::BM, &tm_sfb, &sfull[ss], tl.n0, tl.kb0 + kb);
+            ++sit;
+          }
+        }
+      }
+    producer_done:
+      // Wait (bounded, regardless of abort) for every copy still in flight:
+      // the last min(it, S) stages and min(sit, SS) scale slots.
+      for (uint32_t j = (it > S ? it - S : 0); j < it; ++j) {
+        if (static_cast<int>(j) == dropped) continue;
+        volatile int never = 0;
+        mbar_wait(&full[j % S], (j / S) & 1, &never, tmo, SITE_TEARDOWN_TMA);
+      }
+      if constexpr (Cfg::KG) {
+        for (uint32_t j = (sit > SS ? sit - SS : 0); j < sit; ++j) {
+          volatile int never = 0;
+          mbar_wait(&sfull[j % SS], (j / SS) & 1, &never, tmo, SITE_TEARDOWN_TMA);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ======================= MMA issuer (one thread) ========================
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(Cfg::BM, BN, Cfg::KG ? 1 : 0, Cfg::KG ? 1 : 0);
+      uint32_t it = 0, acc_it = 0;
+      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped);
+        if (!tl.valid) continue;
+        for (int kb = 0; kb < tl.nkb; ++kb, ++it, ++acc_it) {
+          const uint32_t b = acc_it & 1;
+          if (!mbar_wait(&tempty[b], ((acc_it >> 1) & 1) ^ 1, abort_flag, tmo, SITE_MMA_TMEM_EMPTY))
+            goto mma_done_label;
+          tc_fence_after();
+          const uint32_t s = it % S;
+          if (!mbar_wait(&full[s], (it / S) & 1, abort_flag, tmo, SITE_MMA_FULL))
+            goto mma_done_label;
+          tc_fence_after();
+          const uint32_t a_base = smem_addr(sA + s * Cfg::A_BYTES);
+          const uint32_t b_base = smem_addr(sB + s * Cfg::B_BYTES);
+          const uint32_t d_tmem = tmem_base + b * BN;
+#pragma unroll
+          for (int k = 0; k < Cfg::BK / 32; ++k) {
+            uint64_t da, db;
+            if constexpr (Cfg::KG) {
+              // MN-major: 32 K-rows of 128 bytes per MMA; MN atoms 16 KB apart.
+              da = smem_desc_sw128(a_base + k * 32 * 128, 128 * Cfg::BK, 1024);
+              db = smem_desc_sw128(b_base + k * 32 * 128, 128 * Cfg::BK, 1024);
+            } else {
+              // K-major: 32 bytes of K per MMA inside the 128-byte swizzle row.
+              da = smem_desc_sw128(a_base + k * 32, 16, 1024);
+              db = smem_desc_sw128(b_base + k * 32, 16, 1024);
+            }
+            mma_f8f6f4(d_tmem, da, db, idesc, k > 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&tfull[b]);
+        }
+      }
+    mma_done_label:
+      mma_commit(mma_done);
+      {
+        volatile int never = 0;
+        mbar_wait(mma_done, 0, &never, tmo, SITE_TEARDOWN_MMA);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ======================= promotion + epilogue (8 warps) =================
+    const uint32_t q = warp & 3;              // TMEM lane quadrant
+    const uint32_t h = (warp - 2) >> 2;       // column half
+    const int r_in_tile = static_cast<int>(q * 32 + lane);
+    const uint32_t t_lane = tmem_base + ((q * 32) << 16);
+    uint32_t acc_it = 0, sit = 0;
+    const int KBn = args.K / Cfg::BK;  // NT: K-blocks per row of sfb
+    const int nbN = (args.N + 127) / 128;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+      const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped);
+      if (!tl.valid) continue;
+      float acc[EC];
+#pragma unroll
+      for (int j = 0; j < EC; ++j) acc[j] = 0.0f;
+
+      // NT scale streams: sfa for this thread's row, sfb for its column half,
+      // prefetched 4 K-blocks ahead in registers.
+      // (rows past M and column halves past N get zero scales; they are
+      // never stored, and their scale rows may not exist)
+      const float* pa = args.sfa;
+      const float* pb = args.sfb;
+      bool row_in = false, half_in = false;
+      if constexpr (!Cfg::KG) {
+        const int m_local = tl.m0 + r_in_tile;
+        row_in = m_local < args.M;
+        if constexpr (MODE == MODE_MASKED)
+          pa = args.sfa + static_cast<long long>(tl.g) * KBn * args.ld_sfa + m_local;
+        else
+          pa = args.sfa + m_local;
+        const int col_first = tl.n0 + static_cast<int>(h) * EC;
+        half_in = col_first < args.N;
+        pb = args.sfb + (static_cast<long long>(tl.g) * nbN + col_first / 128) * KBn;
+      }
+      float sa0 = 0.f, sa1 = 0.f, sa2 = 0.f, sa3 = 0.f;
+      float sb0 = 0.f, sb1 = 0.f, sb2 = 0.f, sb3 = 0.f;
+      if constexpr (!Cfg::KG) {
+        const int n = tl.nkb;
+        if (half_in) {
+          if (n > 0) sb0 = __ldg(pb + 0);
+          if (n > 1) sb1 = __ldg(pb + 1);
+          if (n > 2) sb2 = __ldg(pb + 2);
+          if (n > 3) sb3 = __ldg(pb + 3);
+        }
+        if (row_in) {
+          if (n > 0) sa0 = __ldg(pa);
+          if (n > 1) sa1 = __ldg(pa + 1LL * args.ld_sfa);
+          if (n > 2) sa2 = __ldg(pa + 2LL * args.ld_sfa);
+          if (n > 3) sa3 = __ldg(pa + 3LL * args.ld_sfa);
+        }
+      }
+
+      for (int kb = 0; kb < tl.nkb; ++kb, ++acc_it) {
+        const uint32_t b = acc_it & 1;
+        bool ok = mbar_wait(&tfull[b], (acc_it >> 1) & 1, abort_flag, tmo, SITE_EPI_TMEM_FULL);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) goto epi_done;
+        tc_fence_after();
+        if constexpr (!Cfg::KG) {
+          const float s = sa0 * sb0;
+          // rotate the prefetch window and fetch K-block kb + 4
+          sa0 = sa1; sa1 = sa2; sa2 = sa3;
+          sb0 = sb1; sb1 = sb2; sb2 = sb3;
+          if (kb + 4 < tl.nkb) {
+            sb3 = half_in ? __ldg(pb + kb + 4) : 0.f;
+            sa3 = row_in ? __ldg(pa + static_cast<long long>(kb + 4) * args.ld_sfa) : 0.f;
+          }
+#pragma unroll
+          for (int c = 0; c < EC / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
+            tmem_ld_wait();
+            if (c == EC / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[b]);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(s, __uint_as_float(r[i]), acc[c * 32 + i]);
+          }
+        } else {
+          const uint32_t ss = sit % SS;
+          bool ok2 = mbar_wait(&sfull[ss], (sit / SS) & 1, abort_flag, tmo, SITE_EPI_SCALE_FULL);
+          ok2 = __all_sync(0xffffffffu, ok2);
+          if (!ok2) goto epi_done;
+          const float* slot = sScale + ss * (Cfg::BM + BN);
+          const float sa = slot[r_in_tile];
+          const float* sbv = slot + Cfg::BM + h * EC;
+#pragma unroll
+          for (int c = 0; c < EC / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
+            tmem_ld_wait();
+            if (c == EC / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[b]);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 sb = *reinterpret_cast<const float4*>(sbv + c * 32 + i);
+              acc[c * 32 + i + 0] = fmaf(sa * sb.x, __uint_as_float(r[i + 0]), acc[c * 32 + i + 0]);
+              acc[c * 32 + i + 1] = fmaf(sa * sb.y, __uint_as_float(r[i + 1]), acc[c * 32 + i + 1]);
+              acc[c * 32 + i + 2] = fmaf(sa * sb.z, __uint_as_float(r[i + 2]), acc[c * 32 + i + 2]);
+              acc[c * 32 + i + 3] = fmaf(sa * sb.w, __uint_as_float(r[i + 3]), acc[c * 32 + i + 3]);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sempty[ss]);
+          ++sit;
+        }
+      }
+
+      // ------------------------------------------------ tile epilogue
+      {
+        bool write = r_in_tile < tl.rows;
+        const long long orow = tl.out_row0 + r_in_tile;
+        if constexpr (MODE == MODE_CONTIG) {
+          if (write) write = __ldg(args.m_indices + orow) == tl.g;
+        }
+        const int col0 = tl.n0 + static_cast<int>(h) * EC;
+        if (write) {
+          if constexpr (Cfg::KG) {
+            float* drow = static_cast<float*>(args.D) + orow * args.N;
+            const float* crow = args.C ? static_cast<const float*>(args.C) + orow * args.N : nullptr;
+#pragma unroll
+            for (int j = 0; j < EC; j += 4) {
+              const int n = col0 + j;
+              if (n < args.N) {
+                float4 v = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                if (crow) {
+                  const float4 c4 = *reinterpret_cast<const float4*>(crow + n);
+                  v.x += c4.x; v.y += c4.y; v.z += c4.z; v.w += c4.w;
+                }
+                *reinterpret_cast<float4*>(drow + n) = v;
+              }
+            }
+          } else {
+            __nv_bfloat16* drow = static_cast<__nv_bfloat16*>(args.D) + orow * args.N;
+            const __nv_bfloat16* crow =
+                args.C ? static_cast<const __nv_bfloat16*>(args.C) + orow * args.N : nullptr;
+#pragma unroll
+            for (int j = 0; j < EC; j += 8) {
+              const int n = col0 + j;
+              if (n < args.N) {
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = acc[j + i];
+                if (crow) {
+                  const uint4 c4 = *reinterpret_cast<const uint4*>(crow + n);
+                  v[0] += bf16_lo(c4.x); v[1] += bf16_hi(c4.x);
+                  v[2] += bf16_lo(c4.y); v[3] += bf16_hi(c4.y);
+                  v[4] += bf16_lo(c4.z); v[5] += bf16_hi(c4.z);
+                  v[6] += bf16_lo(c4.w); v[7] += bf16_hi(c4.w);
+                }
+                uint4 o;
+                o.x = pack_bf16x2(v[0], v[1]);
+                o.y = pack_bf16x2(v[2], v[3]);
+                o.z = pack_bf16x2(v[4], v[5]);
+                o.w = pack_bf16x2(v[6], v[7]);
+                *reinterpret_cast<uint4*>(drow + n) = o;
+              }
+            }
+          }
+        }
+      }
+    }
+  epi_done:;
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace dg

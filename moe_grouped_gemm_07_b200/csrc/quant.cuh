@@ -1,0 +1,184 @@
+// quant.cuh -- BF16/FP32 -> E4M3 quantisers with FP32 scales, sm_100a.
+//
+// scale = max(amax, 1e-4f) / 448 and code = E4M3_RN_satfinite(x / scale), both
+// IEEE single-precision divisions (this file must not be built with
+// --use_fast_math). Three scale granularities:
+//   ROW   one scale per (row, 128-column strip), stored transposed [cols/128][ld]
+//   BLOCK one scale per 128x128 block, [ceil(rows/128)][cols/128]
+//   COL   one scale per (128-row strip, column), [rows/128][cols]
+// All three are single-pass, HBM-bound kernels: every input byte is read once,
+// every code and scale written once.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+namespace dg {
+
+struct In4 {
+  float v[4];
+};
+
+template <bool BF16>
+__device__ __forceinline__ In4 load4(const void* x, int64_t i) {
+  In4 r;
+  if constexpr (BF16) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(x) + i));
+    r.v[0] = __uint_as_float(u.x << 16);
+    r.v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    r.v[2] = __uint_as_float(u.y << 16);
+    r.v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+  } else {
+    const float4 f = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(x) + i));
+    r.v[0] = f.x;
+    r.v[1] = f.y;
+    r.v[2] = f.z;
+    r.v[3] = f.w;
+  }
+  return r;
+}
+
+__device__ __forceinline__ float scale_from_amax(float amax) {
+  return fmaxf(amax, 1e-4f) / 448.0f;  // IEEE division (no fast-math)
+}
+
+// Four E4M3 codes packed little-endian (element 0 in the low byte).
+__device__ __forceinline__ uint32_t encode4(const float (&v)[4], float s) {
+  const float y0 = v[0] / s, y1 = v[1] / s, y2 = v[2] / s, y3 = v[3] / s;
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(y2, y3), __NV_SATFINITE, __NV_E4M3);
+  return (lo & 0xFFFFu) | (hi << 16);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// ROW_1x128: one warp per 128-element strip; strips enumerated (batch, row,
+// strip) with the strip index fastest so consecutive warps stream each row.
+template <bool BF16>
+__global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__ x, int batch,
+                                                        int rows, int cols,
+                                                        uint8_t* __restrict__ codes,
+                                                        float* __restrict__ scales, int ld) {
+  const int lane = threadIdx.x & 31;
+  const int kbs = cols >> 7;
+  const int64_t nstrips = static_cast<int64_t>(batch) * rows * kbs;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t s = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; s < nstrips;
+       s += nwarps) {
+    const int kb = static_cast<int>(s % kbs);
+    const int64_t br = s / kbs;  // batch * rows + row
+    const int64_t base = br * cols + (kb << 7) + (lane << 2);
+    const In4 in = load4<BF16>(x, base);
+    float amax = fmaxf(fmaxf(fabsf(in.v[0]), fabsf(in.v[1])), fmaxf(fabsf(in.v[2]), fabsf(in.v[3])));
+    amax = warp_max(amax);
+    const float sc = scale_from_amax(amax);
+    *reinterpret_cast<uint32_t*>(codes + base) = encode4(in.v, sc);
+    if (lane == 0) {
+      const int64_t b = br / rows;
+      const int r = static_cast<int>(br - b * rows);
+      scales[(b * kbs + kb) * ld + r] = sc;
+    }
+  }
+}
+
+// BLOCK_128x128: one 256-thread CTA per 128x128 block; warp w holds rows
+// [16w, 16w+16) of the block, lane l columns [4l, 4l+4).
+template <bool BF16>
+__global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict__ x, int batch,
+                                                          int rows, int cols,
+                                                          uint8_t* __restrict__ codes,
+                                                          float* __restrict__ scales) {
+  __shared__ float red[8];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int kbs = cols >> 7, nbs = (rows + 127) >> 7;
+  const int64_t blk = blockIdx.x;
+  const int kb = static_cast<int>(blk % kbs);
+  const int nb = static_cast<int>((blk / kbs) % nbs);
+  const int64_t b = blk / (static_cast<int64_t>(kbs) * nbs);
+  In4 v[16];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = (nb << 7) + (w << 4) + i;
+    if (r < rows) {
+      v[i] = load4<BF16>(x, (b * rows + r) * cols + (kb << 7) + (lane << 2));
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].v[0]), fabsf(v[i].v[1])),
+                               fmaxf(fabsf(v[i].v[2]), fabsf(v[i].v[3]))));
+    }
+  }
+  amax = warp_max(amax);
+  if (lane == 0) red[w] = amax;
+  __syncthreads();
+  float a = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
+  const float sc = scale_from_amax(a);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = (nb << 7) + (w << 4) + i;
+    if (r < rows)
+      *reinterpret_cast<uint32_t*>(codes + (b * rows + r) * cols + (kb << 7) + (lane << 2)) =
+          encode4(v[i].v, sc);
+  }
+  if (threadIdx.x == 0) scales[(b * nbs + nb) * kbs + kb] = sc;
+}
+
+// COL_128x1: one 256-thread CTA per (batch, 128-row strip, 64-column slab);
+// thread t holds columns [4(t%16), +4) of rows (t/16) + 16i, i < 8.
+template <bool BF16>
+__global__ void __launch_bounds__(256) quant_col_kernel(const void* __restrict__ x, int batch,
+                                                        int rows, int cols,
+                                                        uint8_t* __restrict__ codes,
+                                                        float* __restrict__ scales) {
+  __shared__ float red[16][64];
+  __shared__ float sc_s[64];
+  const int cg = threadIdx.x & 15, rg = threadIdx.x >> 4;
+  const int slabs = (cols + 63) >> 6, rbs = rows >> 7;
+  const int64_t blk = blockIdx.x;
+  const int slab = static_cast<int>(blk % slabs);
+  const int rb = static_cast<int>((blk / slabs) % rbs);
+  const int64_t b = blk / (static_cast<int64_t>(slabs) * rbs);
+  const int c = (slab << 6) + (cg << 2);
+  const bool col_ok = c < cols;
+  In4 v[8];
+  float m4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = (rb << 7) + rg + (i << 4);
+    if (col_ok) {
+      v[i] = load4<BF16>(x, (b * rows + r) * cols + c);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) m4[j] = fmaxf(m4[j], fabsf(v[i].v[j]));
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) red[rg][(cg << 2) + j] = m4[j];
+  __syncthreads();
+  if (threadIdx.x < 64) {
+    float a = red[0][threadIdx.x];
+#pragma unroll
+    for (int i = 1; i < 16; ++i) a = fmaxf(a, red[i][threadIdx.x]);
+    const float sc = scale_from_amax(a);
+    sc_s[threadIdx.x] = sc;
+    const int cc = (slab << 6) + threadIdx.x;
+    if (cc < cols) scales[(b * rbs + rb) * cols + cc] = sc;
+  }
+  __syncthreads();
+  if (!col_ok) return;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = (rb << 7) + rg + (i << 4);
+    const float y0 = v[i].v[0] / sc_s[(cg << 2) + 0], y1 = v[i].v[1] / sc_s[(cg << 2) + 1];
+    const float y2 = v[i].v[2] / sc_s[(cg << 2) + 2], y3 = v[i].v[3] / sc_s[(cg << 2) + 3];
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(y2, y3), __NV_SATFINITE, __NV_E4M3);
+    *reinterpret_cast<uint32_t*>(codes + (b * rows + r) * cols + c) = (lo & 0xFFFFu) | (hi << 16);
+  }
+}
+
+}  // namespace dg

@@ -1,0 +1,96 @@
+"""The C-ABI library loads without a GPU and exports every entry point that
+include/dg.h declares; host-side validation rejects bad arguments before any
+CUDA call (these paths never touch a device)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dg.h")
+LIB = os.path.join(ROOT, "moe_grouped_gemm_07_b200", "libdg.so")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dg_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_gemms_and_quantiser():
+    names = declared_functions()
+    for n in ["dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
+              "dg_m_grouped_fp8_gemm_nt_masked", "dg_k_grouped_fp8_gemm_tn_contiguous",
+              "dg_quantize_fp8"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    assert os.path.exists(LIB), "build libdg.so first (python moe_grouped_gemm_07_b200/build.py)"
+    out = subprocess.check_output(["nm", "-D", "--defined-only", LIB], text=True)
+    exported = set(l.split()[-1] for l in out.splitlines() if l.strip())
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(LIB)
+    for n in declared_functions():
+        assert getattr(lib, n) is not None
+
+
+def test_binding_exports_same_names():
+    import moe_grouped_gemm_07_b200 as dg
+    for n in declared_functions():
+        assert hasattr(dg, n), n
+        assert n in dg.EXPORTED
+
+
+def test_host_utilities_without_gpu():
+    import moe_grouped_gemm_07_b200 as dg
+    assert dg.dg_get_mk_alignment_for_contiguous_layout() == 128
+    assert dg.dg_get_tma_aligned_size(37, 4) == 40
+    assert dg.dg_get_tma_aligned_size(37, 2) == 40
+    assert dg.dg_get_tma_aligned_size(37, 1) == 48
+    assert dg.dg_get_tma_aligned_size(64, 4) == 64
+    assert dg.dg_get_tma_aligned_size(3, 3) == -1
+    assert dg.dg_status_string(dg.DG_ERR_TIMEOUT) == "DG_ERR_TIMEOUT"
+    assert dg.dg_status_string(99) == "DG_ERR_UNKNOWN"
+
+
+def test_host_validation_before_any_cuda_call():
+    import moe_grouped_gemm_07_b200 as dg
+    L, vp = dg._lib, ctypes.c_void_p
+    fake = vp(0x1000)
+    # shape errors are reported before pointers are touched or a device queried
+    assert L.dg_fp8_gemm_nt(fake, fake, fake, fake, None, fake, 8, 8, 100, None) == \
+        dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert L.dg_fp8_gemm_nt(fake, fake, fake, fake, None, fake, 8, 12, 128, None) == \
+        dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert L.dg_fp8_gemm_nt(fake, fake, fake, fake, None, fake, -1, 8, 128, None) == \
+        dg.DG_ERR_INVALID_ARG
+    assert L.dg_fp8_gemm_nt(None, None, None, None, None, None, 0, 8, 128, None) == dg.DG_OK
+    assert L.dg_m_grouped_fp8_gemm_nt_contiguous(fake, fake, fake, fake, fake, None, fake, 100,
+                                                 8, 128, 2, None) == dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert L.dg_m_grouped_fp8_gemm_nt_contiguous(fake, fake, fake, fake, fake, None, fake, 128,
+                                                 8, 128, 0, None) == dg.DG_ERR_INVALID_ARG
+    assert L.dg_m_grouped_fp8_gemm_nt_masked(fake, fake, fake, fake, fake, fake, 2000, 64, 8,
+                                             128, None) == dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert L.dg_m_grouped_fp8_gemm_nt_masked(fake, fake, fake, fake, fake, fake, 0, 64, 8,
+                                             128, None) == dg.DG_ERR_INVALID_ARG
+    ks = (ctypes.c_int * 2)(128, 100)
+    assert L.dg_k_grouped_fp8_gemm_tn_contiguous(fake, fake, fake, fake, ks, None, fake, 2, 16,
+                                                 16, None) == dg.DG_ERR_UNSUPPORTED_SHAPE
+    ks = (ctypes.c_int * 2)(128, -128)
+    assert L.dg_k_grouped_fp8_gemm_tn_contiguous(fake, fake, fake, fake, ks, None, fake, 2, 16,
+                                                 16, None) == dg.DG_ERR_INVALID_ARG
+    ks = (ctypes.c_int * 1)(128)
+    assert L.dg_k_grouped_fp8_gemm_tn_contiguous(fake, fake, fake, fake, ks, None, fake, 1, 24,
+                                                 16, None) == dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert L.dg_quantize_fp8(fake, 0, 1, 128, 100, 0, fake, fake, 128, None) == \
+        dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert L.dg_quantize_fp8(fake, 0, 1, 100, 128, 2, fake, fake, 0, None) == \
+        dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert L.dg_quantize_fp8(fake, 7, 1, 128, 128, 0, fake, fake, 128, None) == \
+        dg.DG_ERR_INVALID_ARG
+    assert L.dg_quantize_fp8(fake, 0, 1, 128, 128, 0, fake, fake, 126, None) == \
+        dg.DG_ERR_INVALID_ARG

@@ -1,0 +1,201 @@
+"""GPU GEMMs vs the CPU oracle on seeded inputs, element by element.
+
+Each case quantises the same float32 inputs on both sides (GPU kernels vs
+oracle), runs the GPU GEMM through the C ABI and the FP64 oracle GEMM, and
+checks calc_diff <= 1e-4 and |D - R| <= 1e-2 max|R|. Shapes span several tiles
+and ragged M/N tails; rows the method leaves alone (masked rows, padding rows)
+are checked bit-exactly against a sentinel fill.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_grouped_gemm_07_b200 as dg
+import oracle
+import synth
+import synth.workloads as wl
+from gpu_helpers import as_f64, bf16_dev, check_close, dev, to_dev
+
+pytestmark = pytest.mark.gpu
+
+SENTINEL = 0x7FBF  # a bf16 NaN pattern no computed value can produce
+
+
+def quant_nt_gpu(A, B):
+    qa, sa = dg.dg_quantize_fp8(to_dev(A), dg.DG_QUANT_ROW_1x128)
+    qb, sb = dg.dg_quantize_fp8(to_dev(B), dg.DG_QUANT_BLOCK_128x128)
+    return qa, sa, qb, sb
+
+
+def quant_nt_cpu(A, B):
+    oqa, osa = oracle.quantize(A, oracle.ROW_1x128)
+    oqb, osb = oracle.quantize(B, oracle.BLOCK_128x128)
+    return oqa, osa, oqb, osb
+
+
+def sentinel_bf16(shape):
+    t = torch.full(shape, SENTINEL, dtype=torch.int16, device=dev())
+    return t.view(torch.bfloat16)
+
+
+# ------------------------------------------------------------------ dense NT
+DENSE_CASES = [
+    (128, 256, 512, False),     # the correctness configuration (C = 0)
+    (1, 8, 128, False),
+    (77, 200, 384, True),
+    (130, 264, 512, True),
+    (256, 512, 1024, True),
+    (300, 2112, 256, False),    # ragged last N tile (2112 = 8.25 x 256)
+    (513, 136, 640, True),
+]
+
+
+@pytest.mark.parametrize("M,N,K,with_c", DENSE_CASES)
+def test_dense_nt_vs_oracle(M, N, K, with_c):
+    w = wl.dense(M, N, K, cfg=80, shape=M + N + K, with_c=with_c)
+    Cb = synth.to_bf16_bits(w.C) if with_c else None
+    qa, sa, qb, sb = quant_nt_gpu(w.A, w.B)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
+    dg.dg_fp8_gemm_nt(qa, sa, qb, sb, bf16_dev(Cb) if with_c else None, D)
+    R = oracle.gemm_nt(*quant_nt_cpu(w.A, w.B), Cb)
+    check_close(as_f64(D), R, f"dense {M}x{N}x{K}")
+
+
+def test_dense_c_aliases_d_and_is_added_once():
+    M, N, K = 200, 384, 512
+    w = wl.dense(M, N, K, cfg=81, with_c=True)
+    Cb = synth.to_bf16_bits(w.C)
+    qa, sa, qb, sb = quant_nt_gpu(w.A, w.B)
+    D = bf16_dev(Cb).clone()
+    dg.dg_fp8_gemm_nt(qa, sa, qb, sb, D, D)
+    R = oracle.gemm_nt(*quant_nt_cpu(w.A, w.B), Cb)
+    check_close(as_f64(D), R, "C aliases D")
+
+
+def test_dense_deterministic():
+    M, N, K = 384, 768, 1024
+    w = wl.dense(M, N, K, cfg=82)
+    qa, sa, qb, sb = quant_nt_gpu(w.A, w.B)
+    outs = []
+    for _ in range(3):
+        D = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
+        dg.dg_fp8_gemm_nt(qa, sa, qb, sb, None, D)
+        outs.append(D.view(torch.int16).cpu().numpy())
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+
+
+def test_dense_k_zero_copies_c_and_empty_is_noop():
+    M, N = 64, 128
+    C = torch.randn(M, N, device=dev()).to(torch.bfloat16)
+    D = torch.zeros(M, N, device=dev(), dtype=torch.bfloat16)
+    e = torch.empty(0, device=dev(), dtype=torch.uint8)
+    s = torch.zeros(1, device=dev(), dtype=torch.float32)
+    dg._check("k0", dg._lib.dg_fp8_gemm_nt(None, None, None, None, dg._ptr(C), dg._ptr(D), M, N, 0,
+                                           dg._stream()))
+    torch.cuda.synchronize()
+    assert torch.equal(D.view(torch.int16), C.view(torch.int16))
+    assert dg._lib.dg_fp8_gemm_nt(None, None, None, None, None, None, 0, N, 128,
+                                  dg._stream()) == dg.DG_OK
+    del e, s
+
+
+def test_dense_rejects_bad_args():
+    z = torch.zeros(16, device=dev(), dtype=torch.uint8)
+    p = dg._ptr(z)
+    st = dg._stream()
+    assert dg._lib.dg_fp8_gemm_nt(p, p, p, p, None, p, 8, 8, 100, st) == dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert dg._lib.dg_fp8_gemm_nt(p, p, p, p, None, p, 8, 12, 128, st) == dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert dg._lib.dg_fp8_gemm_nt(p, p, p, p, None, p, -1, 8, 128, st) == dg.DG_ERR_INVALID_ARG
+    bad = dg._vp(z.data_ptr() + 4)
+    assert dg._lib.dg_fp8_gemm_nt(bad, p, p, p, None, p, 8, 8, 128, st) == dg.DG_ERR_MISALIGNED
+    assert dg._lib.dg_fp8_gemm_nt(None, p, p, p, None, p, 8, 8, 128, st) == dg.DG_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------------ contiguous
+@pytest.mark.parametrize("G,N,K,lo,hi", [(3, 264, 256, 100, 300), (4, 512, 384, 1, 200)])
+def test_contiguous_vs_oracle(G, N, K, lo, hi):
+    w = wl.contiguous(G=G, N=N, K=K, lo=lo, hi=hi, cfg=83, shape=G)
+    Cb = synth.to_bf16_bits(synth.normal((w.Mt, N), synth.seed(83, G, 2)))
+    qa, sa = dg.dg_quantize_fp8(to_dev(w.A), dg.DG_QUANT_ROW_1x128)
+    qb, sb = dg.dg_quantize_fp8(to_dev(w.B), dg.DG_QUANT_BLOCK_128x128)
+    D = sentinel_bf16((w.Mt, N))
+    mi = to_dev(w.m_indices)
+    dg.dg_m_grouped_fp8_gemm_nt_contiguous(qa, sa, qb, sb, mi, bf16_dev(Cb), D)
+    oqa, osa = oracle.quantize(w.A, oracle.ROW_1x128)
+    oqb, osb = oracle.quantize(w.B, oracle.BLOCK_128x128)
+    R = oracle.m_grouped_contiguous(oqa, osa, oqb, osb, w.m_indices, Cb)
+    check_close(as_f64(D), R, "contiguous")
+    raw = D.view(torch.int16).cpu().numpy().view(np.uint16)
+    pad = w.m_indices < 0
+    assert np.all(raw[pad] == SENTINEL), "padding rows were written"
+
+
+# ------------------------------------------------------------------ masked
+@pytest.mark.parametrize("G,max_m,N,K", [(4, 192, 200, 384), (3, 256, 512, 256)])
+def test_masked_vs_oracle(G, max_m, N, K):
+    w = wl.masked(G=G, max_m=max_m, N=N, K=K, lo=0, hi=max_m, cfg=84, shape=G)
+    w.masked_m[0] = max_m
+    w.masked_m[-1] = 0
+    qa, sa = dg.dg_quantize_fp8(to_dev(w.A), dg.DG_QUANT_ROW_1x128)
+    qb, sb = dg.dg_quantize_fp8(to_dev(w.B), dg.DG_QUANT_BLOCK_128x128)
+    D = sentinel_bf16((G, max_m, N))
+    dg.dg_m_grouped_fp8_gemm_nt_masked(qa, sa, qb, sb, to_dev(w.masked_m), D)
+    oqa, osa = oracle.quantize(w.A, oracle.ROW_1x128)
+    oqb, osb = oracle.quantize(w.B, oracle.BLOCK_128x128)
+    R = oracle.m_grouped_masked(oqa, osa, oqb, osb, w.masked_m)
+    check_close(as_f64(D), R, "masked")
+    raw = D.view(torch.int16).cpu().numpy().view(np.uint16)
+    for g in range(G):
+        assert np.all(raw[g, w.masked_m[g]:] == SENTINEL), f"group {g}: masked rows written"
+
+
+def test_masked_counts_above_max_are_clamped():
+    G, max_m, N, K = 2, 128, 128, 128
+    w = wl.masked(G=G, max_m=max_m, N=N, K=K, cfg=85)
+    mm = np.array([1000, -5], dtype=np.int32)
+    qa, sa = dg.dg_quantize_fp8(to_dev(w.A), dg.DG_QUANT_ROW_1x128)
+    qb, sb = dg.dg_quantize_fp8(to_dev(w.B), dg.DG_QUANT_BLOCK_128x128)
+    D = sentinel_bf16((G, max_m, N))
+    dg.dg_m_grouped_fp8_gemm_nt_masked(qa, sa, qb, sb, to_dev(mm), D)
+    oqa, osa = oracle.quantize(w.A, oracle.ROW_1x128)
+    oqb, osb = oracle.quantize(w.B, oracle.BLOCK_128x128)
+    R = oracle.m_grouped_masked(oqa, osa, oqb, osb, np.array([max_m, 0], dtype=np.int32))
+    check_close(as_f64(D), R, "masked clamp")
+    raw = D.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.all(raw[1] == SENTINEL)
+
+
+# ------------------------------------------------------------------ K-grouped
+@pytest.mark.parametrize("G,M,N,ks,with_c", [
+    (3, 144, 272, [256, 0, 384], True),
+    (2, 128, 256, [128, 640], False),
+    (4, 256, 512, [384, 128, 256, 512], True),
+])
+def test_k_grouped_vs_oracle(G, M, N, ks, with_c):
+    w = wl.k_grouped(G=G, M=M, N=N, ks=ks, cfg=86, shape=G)
+    qa, sa = dg.dg_quantize_fp8(to_dev(w.A), dg.DG_QUANT_COL_128x1)
+    qb, sb = dg.dg_quantize_fp8(to_dev(w.B), dg.DG_QUANT_COL_128x1)
+    C = to_dev(w.C) if with_c else None
+    D = torch.full((G, M, N), float("nan"), device=dev())
+    dg.dg_k_grouped_fp8_gemm_tn_contiguous(qa, sa, qb, sb, w.ks, C, D)
+    oqa, osa = oracle.quantize(w.A, oracle.COL_128x1)
+    oqb, osb = oracle.quantize(w.B, oracle.COL_128x1)
+    R = oracle.k_grouped_tn(oqa, osa, oqb, osb, w.ks, w.C if with_c else None)
+    check_close(D.cpu().numpy().astype(np.float64), R, "k-grouped")
+    for g, k in enumerate(ks):
+        if k == 0:
+            expect = w.C[g] if with_c else np.zeros((M, N), np.float32)
+            assert np.array_equal(D[g].cpu().numpy(), expect)
+
+
+def test_k_grouped_accumulates_in_place():
+    G, M, N, ks = 2, 128, 256, [256, 384]
+    w = wl.k_grouped(G=G, M=M, N=N, ks=ks, cfg=87)
+    qa, sa = dg.dg_quantize_fp8(to_dev(w.A), dg.DG_QUANT_COL_128x1)
+    qb, sb = dg.dg_quantize_fp8(to_dev(w.B), dg.DG_QUANT_COL_128x1)
+    D = to_dev(w.C).clone()
+    dg.dg_k_grouped_fp8_gemm_tn_contiguous(qa, sa, qb, sb, ks, D, D)
+    oqa, osa = oracle.quantize(w.A, oracle.COL_128x1)
+    oqb, osb = oracle.quantize(w.B, oracle.COL_128x1)
+    R = oracle.k_grouped_tn(oqa, osa, oqb, osb, ks, w.C)
+    check_close(D.cpu().numpy().astype(np.float64), R, "k-grouped in place")
