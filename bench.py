@@ -266,6 +266,10 @@ def run_ours(args):
     def step(record=False):
         for i, (M, N, K) in enumerate(shapes):
             flush.fill_(i & 0xFF)
+            # ~50 us device spin (outside the per-shape events) so the host has
+            # queued the timed launches before the device reaches them: the
+            # events then bracket kernel time, not host submission gaps
+            torch.cuda._sleep(100_000)
             if record:
                 ev[i][0].record()
             qa, sa = qbufs[i]
@@ -399,6 +403,7 @@ def run_ours(args):
                    "NK": [list(x) for x in wl.DENSE_NK],
                    "step": "per shape: quantise A (1x128) + GEMM; B pre-quantised (128x128)",
                    "l2": "flushed (256 MiB write) before every shape, flush excluded from timing",
+                   "host_gap": "a ~50 us device spin precedes each shape so events time kernels only",
                    "parallelism": f"replicas x{world}"},
         "ms_per_step_incl_flush": round(ms_outer, 4),
         "fp8_pct_of_measured_peak": round(100 * flops_step / (ms_step * 1e-3) / 1e12 / fp8_peak, 2),

@@ -13,6 +13,7 @@
 
 #include "../../include/dg.h"
 #include "gemm.cuh"
+#include "gemm_decode.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 
@@ -213,6 +214,120 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
   return launch_gemm<MODE, 128>(ta, tb, dummy, dummy, args, grid, st, dev);
 }
 
+// ---------------------------------------------------------------- decode path
+// Largest cluster size (1..8, powers of two) that the device can co-schedule
+// for this kernel; cached per device and instantiation.
+template <int BNP>
+int max_cluster(int dev) {
+  using Cfg = dg::DecodeCfg<BNP>;
+  static std::once_flag once[kMaxDevices];
+  static int best[kMaxDevices];
+  std::call_once(once[dev], [&] {
+    auto kern = dg::gemm_decode_kernel<BNP>;
+    best[dev] = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM_BYTES) != cudaSuccess)
+      return;
+    for (int c = 8; c >= 1; c >>= 1) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(c, 1, 1);
+      cfg.blockDim = dim3(320, 1, 1);
+      cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = c;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) {
+        best[dev] = c;
+        return;
+      }
+      cudaGetLastError();
+    }
+  });
+  return best[dev];
+}
+
+// Split count: double the CTAs per N-tile while the launch still fits in two
+// CTAs per SM and every CTA keeps at least two K-blocks.
+int choose_splits(int n_tiles, int KB, int sms, int cap) {
+  int splits = 1;
+  while (splits * 2 <= cap && static_cast<long long>(n_tiles) * splits * 2 <= 2ll * sms &&
+         KB / (splits * 2) >= 2)
+    splits *= 2;
+  return splits;
+}
+
+template <int BNP>
+dg_status run_decode(const void* A, const float* sfa, const void* B, const float* sfb,
+                     const void* C, void* D, int M, int N, int K, int sms, int dev,
+                     cudaStream_t st) {
+  using Cfg = dg::DecodeCfg<BNP>;
+  const int cap = max_cluster<BNP>(dev);
+  if (cap <= 0) return DG_ERR_CUDA;
+  const int KB = K / 128;
+  const int n_tiles = (N + 127) / 128;
+  const int splits = choose_splits(n_tiles, KB, sms, cap);
+  const int ld = (M + 3) / 4 * 4;
+  CUtensorMap tw, tx, tsa;
+  dg_status s;
+  if ((s = make_map_2d(&tw, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  if ((s = make_map_2d(&tx, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, BNP,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  if ((s = make_map_2d(&tsa, sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ld, KB, 4ull * ld, BNP, 1,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
+    return s;
+  dg::DecodeArgs args;
+  std::memset(&args, 0, sizeof args);
+  args.M = M;
+  args.N = N;
+  args.K = K;
+  args.KB = KB;
+  args.splits = splits;
+  args.sfb = sfb;
+  args.C = C;
+  args.D = D;
+  args.timeout_ns = timeout_ns();
+  args.drop_arrive = take_drop_flag();
+  if (print_configs())
+    std::fprintf(stderr,
+                 "[dg] fp8_gemm_nt decode M=%d N=%d K=%d: swap-AB BNP=%d, n_tiles=%d x "
+                 "split-K %d (cluster), %d CTAs, %d stages\n",
+                 M, N, K, BNP, n_tiles, splits, n_tiles * splits, Cfg::STAGES);
+  auto kern = dg::gemm_decode_kernel<BNP>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(splits, n_tiles, 1);
+  cfg.blockDim = dim3(320, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, tsa, args);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  g_launches.fetch_add(1);
+  return DG_OK;
+}
+
+dg_status dispatch_decode(const void* A, const float* sfa, const void* B, const float* sfb,
+                          const void* C, void* D, int M, int N, int K, int sms, int dev,
+                          cudaStream_t st) {
+  if (M <= 16) return run_decode<16>(A, sfa, B, sfb, C, D, M, N, K, sms, dev, st);
+  if (M <= 32) return run_decode<32>(A, sfa, B, sfb, C, D, M, N, K, sms, dev, st);
+  if (M <= 64) return run_decode<64>(A, sfa, B, sfb, C, D, M, N, K, sms, dev, st);
+  return run_decode<128>(A, sfa, B, sfb, C, D, M, N, K, sms, dev, st);
+}
+
 }  // namespace
 
 // =============================================================== C ABI
@@ -330,6 +445,12 @@ dg_status dg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const f
     return DG_ERR_MISALIGNED;
   const int ld = (M + 3) / 4 * 4;
   const long long mb = (M + 127) / 128;
+  if (M <= 128) {
+    int dev = 0, sms = 0;
+    dg_status s = device_sms(&dev, &sms);
+    if (s != DG_OK) return s;
+    return dispatch_decode(A, sfa, B, sfb, C, D, M, N, K, sms, dev, st);
+  }
   return run_nt<dg::MODE_DENSE>(A, sfa, ld, B, sfb, nullptr, nullptr, C, D, M, M, N, K, 1, mb, mb,
                                 st, "fp8_gemm_nt");
 }

@@ -78,6 +78,9 @@ struct GemmCfg {
   static constexpr int PREFIX_BYTES = MODE == MODE_MASKED ? (2 * kMaxMaskedGroups + 1) * 4 : 0;
   static constexpr int SMEM_BYTES = OFF_PREFIX + PREFIX_BYTES + 1024;  // + alignment slack
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  // TMA destinations: 128-byte aligned; 128B-swizzled tiles 1024-byte aligned
+  static_assert(OFF_B % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "tiles");
+  static_assert(OFF_SCALE % 128 == 0 && SCALE_BYTES % 128 == 0 && (BM * 4) % 128 == 0, "scales");
   static_assert(BN == 128 || BN == 256, "BN");
 };
 
@@ -425,82 +428,87 @@ __global__ void __launch_bounds__(320, 1)
         half_in = col_first < args.N;
         pb = args.sfb + (static_cast<long long>(tl.g) * nbN + col_first / 128) * KBn;
       }
-      float sa0 = 0.f, sa1 = 0.f, sa2 = 0.f, sa3 = 0.f;
-      float sb0 = 0.f, sb1 = 0.f, sb2 = 0.f, sb3 = 0.f;
+      // Prefetch ring of 4 K-blocks; the K-block loop is unrolled by 4 so
+      // slot u is consumed and refilled in place (no register moves that
+      // would wait on an in-flight load).
+      float sa[4] = {0.f, 0.f, 0.f, 0.f};
+      float sb[4] = {0.f, 0.f, 0.f, 0.f};
       if constexpr (!Cfg::KG) {
-        const int n = tl.nkb;
-        if (half_in) {
-          if (n > 0) sb0 = __ldg(pb + 0);
-          if (n > 1) sb1 = __ldg(pb + 1);
-          if (n > 2) sb2 = __ldg(pb + 2);
-          if (n > 3) sb3 = __ldg(pb + 3);
-        }
-        if (row_in) {
-          if (n > 0) sa0 = __ldg(pa);
-          if (n > 1) sa1 = __ldg(pa + 1LL * args.ld_sfa);
-          if (n > 2) sa2 = __ldg(pa + 2LL * args.ld_sfa);
-          if (n > 3) sa3 = __ldg(pa + 3LL * args.ld_sfa);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (u < tl.nkb) {
+            if (half_in) sb[u] = __ldg(pb + u);
+            if (row_in) sa[u] = __ldg(pa + static_cast<long long>(u) * args.ld_sfa);
+          }
         }
       }
 
-      for (int kb = 0; kb < tl.nkb; ++kb, ++acc_it) {
-        const uint32_t b = acc_it & 1;
-        bool ok = mbar_wait(&tfull[b], (acc_it >> 1) & 1, abort_flag, tmo, SITE_EPI_TMEM_FULL);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) goto epi_done;
-        tc_fence_after();
-        if constexpr (!Cfg::KG) {
-          const float s = sa0 * sb0;
-          // rotate the prefetch window and fetch K-block kb + 4
-          sa0 = sa1; sa1 = sa2; sa2 = sa3;
-          sb0 = sb1; sb1 = sb2; sb2 = sb3;
-          if (kb + 4 < tl.nkb) {
-            sb3 = half_in ? __ldg(pb + kb + 4) : 0.f;
-            sa3 = row_in ? __ldg(pa + static_cast<long long>(kb + 4) * args.ld_sfa) : 0.f;
-          }
+      for (int kb0 = 0; kb0 < tl.nkb; kb0 += 4) {
 #pragma unroll
-          for (int c = 0; c < EC / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
-            tmem_ld_wait();
-            if (c == EC / 32 - 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&tempty[b]);
+        for (int u = 0; u < 4; ++u) {
+          const int kb = kb0 + u;
+          if (kb >= tl.nkb) break;
+          const uint32_t b = acc_it & 1;
+          bool ok = mbar_wait(&tfull[b], (acc_it >> 1) & 1, abort_flag, tmo, SITE_EPI_TMEM_FULL);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) goto epi_done;
+          tc_fence_after();
+          if constexpr (!Cfg::KG) {
+            const float sc = sa[u] * sb[u];
+            if (kb + 4 < tl.nkb) {
+              sb[u] = half_in ? __ldg(pb + kb + 4) : 0.f;
+              sa[u] = row_in ? __ldg(pa + static_cast<long long>(kb + 4) * args.ld_sfa) : 0.f;
             }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(s, __uint_as_float(r[i]), acc[c * 32 + i]);
-          }
-        } else {
-          const uint32_t ss = sit % SS;
-          bool ok2 = mbar_wait(&sfull[ss], (sit / SS) & 1, abort_flag, tmo, SITE_EPI_SCALE_FULL);
-          ok2 = __all_sync(0xffffffffu, ok2);
-          if (!ok2) goto epi_done;
-          const float* slot = sScale + ss * (Cfg::BM + BN);
-          const float sa = slot[r_in_tile];
-          const float* sbv = slot + Cfg::BM + h * EC;
+            for (int c = 0; c < EC / 32; ++c) {
+              uint32_t r[32];
+              tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
+              tmem_ld_wait();
+              if (c == EC / 32 - 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[b]);
+              }
 #pragma unroll
-          for (int c = 0; c < EC / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
-            tmem_ld_wait();
-            if (c == EC / 32 - 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&tempty[b]);
+              for (int i = 0; i < 32; i += 2)
+                fma2(acc[c * 32 + i], acc[c * 32 + i + 1], sc, sc, __uint_as_float(r[i]),
+                     __uint_as_float(r[i + 1]));
             }
+          } else {
+            const uint32_t ss = sit % SS;
+            bool ok2 = mbar_wait(&sfull[ss], (sit / SS) & 1, abort_flag, tmo, SITE_EPI_SCALE_FULL);
+            ok2 = __all_sync(0xffffffffu, ok2);
+            if (!ok2) goto epi_done;
+            const float* slot = sScale + ss * (Cfg::BM + BN);
+            const float sav = slot[r_in_tile];
+            const float* sbv = slot + Cfg::BM + h * EC;
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const float4 sb = *reinterpret_cast<const float4*>(sbv + c * 32 + i);
-              acc[c * 32 + i + 0] = fmaf(sa * sb.x, __uint_as_float(r[i + 0]), acc[c * 32 + i + 0]);
-              acc[c * 32 + i + 1] = fmaf(sa * sb.y, __uint_as_float(r[i + 1]), acc[c * 32 + i + 1]);
-              acc[c * 32 + i + 2] = fmaf(sa * sb.z, __uint_as_float(r[i + 2]), acc[c * 32 + i + 2]);
-              acc[c * 32 + i + 3] = fmaf(sa * sb.w, __uint_as_float(r[i + 3]), acc[c * 32 + i + 3]);
+            for (int c = 0; c < EC / 32; ++c) {
+              uint32_t r[32];
+              tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
+              tmem_ld_wait();
+              if (c == EC / 32 - 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[b]);
+              }
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
+                const float4 sb4 = *reinterpret_cast<const float4*>(sbv + c * 32 + i);
+                float t0, t1, t2, t3;
+                mul2(t0, t1, sav, sav, sb4.x, sb4.y);
+                mul2(t2, t3, sav, sav, sb4.z, sb4.w);
+                fma2(acc[c * 32 + i], acc[c * 32 + i + 1], t0, t1, __uint_as_float(r[i]),
+                     __uint_as_float(r[i + 1]));
+                fma2(acc[c * 32 + i + 2], acc[c * 32 + i + 3], t2, t3, __uint_as_float(r[i + 2]),
+                     __uint_as_float(r[i + 3]));
+              }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sempty[ss]);
+            ++sit;
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sempty[ss]);
-          ++sit;
+          ++acc_it;
         }
       }
 

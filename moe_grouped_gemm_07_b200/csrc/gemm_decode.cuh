@@ -1,0 +1,316 @@
+// gemm_decode.cuh -- FP8 fine-grained-scaled GEMM for small M (M <= 128,
+// decode), sm_100a. Same operation and promotion rule as gemm.cuh:
+//   D[m][n] = C[m][n] + sum_kb sfa[kb][m] * sfb[n/128][kb] * P_kb[m][n]
+// but arranged for the memory-bound regime (the DeepGEMM launch article notes
+// decode shapes are bandwidth-bound; the blog "从矩阵乘法为什么这么慢说起" §2.2,
+// §5.1 describes thin shapes starving the tensor cores):
+//
+//   * swap-AB: the 128 weight rows of an N-tile fill the MMA's M = 128 lanes
+//     and the tokens become the MMA's N (BNP = 16..128 columns), so one
+//     128-row weight block -- and therefore one sfb value per K-block --
+//     covers the whole tile;
+//   * split-K across a thread-block cluster: the `splits` CTAs of a cluster
+//     share one N-tile and each streams its own slice of K-blocks, so
+//     n_tiles x splits CTAs keep HBM busy even when N/128 is small;
+//   * the partial tiles are reduced through distributed shared memory: each
+//     CTA writes its FP32 partial to its own shared memory, the cluster
+//     synchronises, and CTA r sums rows [r*128/splits, (r+1)*128/splits) of
+//     all partials in rank order (deterministic), adds C and stores BF16.
+//
+// Roles per CTA (320 threads): warp 0 TMA producer, warp 1 TMEM allocator and
+// single-thread tcgen05.mma issuer, warps 2..9 promotion (TMEM lane quadrant
+// w % 4, column half (w - 2) / 4). All waits are bounded (see ptx.cuh); both
+// cluster barriers are reached unconditionally, also after a timeout.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+namespace dg {
+
+struct DecodeArgs {
+  int M, N, K;
+  int KB;       // K / 128
+  int splits;   // CTAs per cluster along K
+  const float* sfb;  // [ceil(N/128)][KB]
+  const void* C;     // [M][N] bf16 or null
+  void* D;           // [M][N] bf16
+  unsigned long long timeout_ns;
+  int drop_arrive;
+};
+
+template <int BNP_>
+struct DecodeCfg {
+  static constexpr int BNP = BNP_;              // token columns (MMA N)
+  static constexpr int BK = 128;
+  static constexpr int W_BYTES = 128 * BK;      // weight tile (MMA A operand)
+  static constexpr int X_BYTES = BNP * BK;      // token tile (MMA B operand)
+  static constexpr int RING = 96 * 1024;
+  static constexpr int STAGES_RAW = RING / (W_BYTES + X_BYTES);
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int SS = 8;                  // sfa slots
+  // a TMA destination in shared memory must be 128-byte aligned, so each
+  // slot holds at least 32 floats even when BNP = 16
+  static constexpr int SLOT_FLOATS = BNP < 32 ? 32 : BNP;
+  static constexpr int EC = BNP / 2;            // accumulator columns per promotion thread
+  static constexpr int CH = EC < 16 ? EC : 16;  // columns per tcgen05.ld
+  static constexpr int TMEM_COLS = 2 * BNP < 32 ? 32 : 2 * BNP;
+  static constexpr int OFF_W = 0;
+  static constexpr int OFF_X = OFF_W + STAGES * W_BYTES;
+  static constexpr int OFF_SCALE = OFF_X + STAGES * X_BYTES;
+  static constexpr int OFF_BAR = OFF_SCALE + SS * SLOT_FLOATS * 4;
+  static constexpr int NUM_BARS = 2 * STAGES + 4 + 2 * SS + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int RED_BYTES = BNP * 128 * 4;  // partial tile, overlays the ring
+  static_assert(RED_BYTES <= STAGES * (W_BYTES + X_BYTES), "reduction buffer fits the ring");
+  static_assert(BNP == 16 || BNP == 32 || BNP == 64 || BNP == 128, "BNP");
+  static_assert(OFF_SCALE % 1024 == 0 && (SLOT_FLOATS * 4) % 128 == 0, "TMA smem alignment");
+  static_assert(OFF_X % 1024 == 0 && X_BYTES % 1024 == 0, "SW128 tiles are 1024-byte aligned");
+  static_assert(SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
+};
+
+template <int BNP>
+__global__ void __launch_bounds__(320, 2)
+    gemm_decode_kernel(const __grid_constant__ CUtensorMap tm_w,    // B: [N][K] e4m3
+                       const __grid_constant__ CUtensorMap tm_x,    // A: [M][K] e4m3
+                       const __grid_constant__ CUtensorMap tm_sfa,  // sfa: [KB][ld] f32
+                       const __grid_constant__ DecodeArgs args) {
+  using Cfg = DecodeCfg<BNP>;
+  constexpr int S = Cfg::STAGES;
+  constexpr int SS = Cfg::SS;
+  constexpr int EC = Cfg::EC;
+  constexpr int CH = Cfg::CH;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sW = smem + Cfg::OFF_W;
+  uint8_t* sX = smem + Cfg::OFF_X;
+  float* sScale = reinterpret_cast<float*>(smem + Cfg::OFF_SCALE);
+  float* red = reinterpret_cast<float*>(smem);  // [BNP][128] partial, after the main loop
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint64_t* sfull = bars + 2 * S + 4;
+  uint64_t* sempty = bars + 2 * S + 4 + SS;
+  uint64_t* mma_done = bars + 2 * S + 4 + 2 * SS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
+
+  const uint32_t warp = warp_id_uniform();
+  const uint32_t lane = lane_id();
+  const uint64_t tmo = args.timeout_ns;
+  const uint32_t rank = cluster_ctarank();
+  const int splits = args.splits;
+  const int n_tile = blockIdx.y;
+  const int n0 = n_tile * 128;
+  const int kb_begin = static_cast<int>((static_cast<long long>(rank) * args.KB) / splits);
+  const int kb_end = static_cast<int>((static_cast<long long>(rank + 1) * args.KB) / splits);
+  const int nkb = kb_end - kb_begin;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);
+    }
+    for (int i = 0; i < SS; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&sempty[i], 8);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_sfa);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  float acc[EC];
+#pragma unroll
+  for (int j = 0; j < EC; ++j) acc[j] = 0.0f;
+  const uint32_t q = warp & 3;
+  const uint32_t h = (warp - 2) >> 2;
+
+  if (warp == 0) {
+    // ======================= TMA producer =======================
+    if (lane == 0) {
+      int it = 0;
+      int dropped = -1;
+      for (; it < nkb; ++it) {
+        const int s = it % S;
+        const int ss = it % SS;
+        if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort_flag, tmo, SITE_PRODUCER_EMPTY)) break;
+        if (!mbar_wait(&sempty[ss], ((it / SS) & 1) ^ 1, abort_flag, tmo,
+                       SITE_PRODUCER_SCALE_EMPTY))
+          break;
+        const int kb = kb_begin + it;
+        if (args.drop_arrive && it == 0) {
+          dropped = 0;  // test hook: never arm stage 0
+        } else {
+          mbar_arrive_expect_tx(&full[s], Cfg::W_BYTES + Cfg::X_BYTES);
+          tma_load_2d(sW + s * Cfg::W_BYTES, &tm_w, &full[s], kb * Cfg::BK, n0);
+          tma_load_2d(sX + s * Cfg::X_BYTES, &tm_x, &full[s], kb * Cfg::BK, 0);
+        }
+        mbar_arrive_expect_tx(&sfull[ss], BNP * 4);
+        tma_load_2d(sScale + ss * Cfg::SLOT_FLOATS, &tm_sfa, &sfull[ss], 0, kb);
+      }
+      // bounded wait for every copy still in flight
+      for (int j = (it > S ? it - S : 0); j < it; ++j) {
+        if (j == dropped) continue;
+        volatile int never = 0;
+        mbar_wait(&full[j % S], (j / S) & 1, &never, tmo, SITE_TEARDOWN_TMA);
+      }
+      for (int j = (it > SS ? it - SS : 0); j < it; ++j) {
+        volatile int never = 0;
+        mbar_wait(&sfull[j % SS], (j / SS) & 1, &never, tmo, SITE_TEARDOWN_TMA);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(128, BNP, 0, 0);
+      for (int it = 0; it < nkb; ++it) {
+        const uint32_t b = it & 1;
+        if (!mbar_wait(&tempty[b], ((it >> 1) & 1) ^ 1, abort_flag, tmo, SITE_MMA_TMEM_EMPTY)) break;
+        tc_fence_after();
+        const int s = it % S;
+        if (!mbar_wait(&full[s], (it / S) & 1, abort_flag, tmo, SITE_MMA_FULL)) break;
+        tc_fence_after();
+        const uint32_t w_base = smem_addr(sW + s * Cfg::W_BYTES);
+        const uint32_t x_base = smem_addr(sX + s * Cfg::X_BYTES);
+#pragma unroll
+        for (int k = 0; k < Cfg::BK / 32; ++k)
+          mma_f8f6f4(tmem_base + b * BNP, smem_desc_sw128(w_base + k * 32, 16, 1024),
+                     smem_desc_sw128(x_base + k * 32, 16, 1024), idesc, k > 0 ? 1u : 0u);
+        mma_commit(&empty[s]);
+        mma_commit(&tfull[b]);
+      }
+      mma_commit(mma_done);
+      volatile int never = 0;
+      mbar_wait(mma_done, 0, &never, tmo, SITE_TEARDOWN_MMA);
+    }
+    __syncwarp();
+  } else {
+    // ======================= promotion (8 warps) =======================
+    const uint32_t t_lane = tmem_base + ((q * 32) << 16);
+    const float* pb = args.sfb + static_cast<long long>(n_tile) * args.KB + kb_begin;
+    // sfb prefetch ring of 4 K-blocks, loop unrolled by 4 (slot u refilled in place)
+    float sbr[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (u < nkb) sbr[u] = __ldg(pb + u);
+    for (int it0 = 0; it0 < nkb; it0 += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int it = it0 + u;
+        if (it >= nkb) break;
+        const uint32_t b = it & 1;
+        bool ok = mbar_wait(&tfull[b], (it >> 1) & 1, abort_flag, tmo, SITE_EPI_TMEM_FULL);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) goto promo_done;
+        const int ss = it % SS;
+        bool ok2 = mbar_wait(&sfull[ss], (it / SS) & 1, abort_flag, tmo, SITE_EPI_SCALE_FULL);
+        ok2 = __all_sync(0xffffffffu, ok2);
+        if (!ok2) goto promo_done;
+        tc_fence_after();
+        const float sb = sbr[u];
+        if (it + 4 < nkb) sbr[u] = __ldg(pb + it + 4);
+        const float* sa = sScale + ss * Cfg::SLOT_FLOATS + h * EC;
+#pragma unroll
+        for (int c = 0; c < EC / CH; ++c) {
+          uint32_t r[CH];
+          tmem_ld_32x32b<CH>(t_lane + b * BNP + h * EC + c * CH, r);
+          tmem_ld_wait();
+          if (c == EC / CH - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[b]);
+          }
+#pragma unroll
+          for (int i = 0; i < CH; i += 4) {
+            const float4 s4 = *reinterpret_cast<const float4*>(sa + c * CH + i);
+            float t0, t1, t2, t3;
+            mul2(t0, t1, s4.x, s4.y, sb, sb);
+            mul2(t2, t3, s4.z, s4.w, sb, sb);
+            fma2(acc[c * CH + i], acc[c * CH + i + 1], t0, t1, __uint_as_float(r[i]),
+                 __uint_as_float(r[i + 1]));
+            fma2(acc[c * CH + i + 2], acc[c * CH + i + 3], t2, t3, __uint_as_float(r[i + 2]),
+                 __uint_as_float(r[i + 3]));
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty[ss]);
+      }
+    }
+  promo_done:;
+  }
+
+  // ---------------------------------------------------------- split-K reduction
+  // Every role is done and every copy / MMA has landed, so the ring is free.
+  tc_fence_before();
+  __syncthreads();
+  if (warp >= 2) {
+    const int n_local = static_cast<int>(q * 32 + lane);
+#pragma unroll
+    for (int j = 0; j < EC; ++j) red[(h * EC + j) * 128 + n_local] = acc[j];
+  }
+  cluster_sync_all();
+  {
+    const int rows = 128 / splits;            // n rows this CTA reduces
+    const int chunks = rows / 4;              // float4 chunks per token column
+    const int n_lo = static_cast<int>(rank) * rows;
+    const uint32_t red_base = smem_addr(red);
+    const int items = BNP * chunks;
+    for (int itm = threadIdx.x; itm < items; itm += blockDim.x) {
+      const int m = itm / chunks;
+      const int n = n_lo + (itm - m * chunks) * 4;
+      const int gn = n0 + n;
+      if (m >= args.M || gn >= args.N) continue;
+      const uint32_t off = red_base + static_cast<uint32_t>((m * 128 + n) * 4);
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int r = 0; r < splits; ++r) {  // fixed rank order: deterministic
+        const float4 v = ld_dsmem_f32x4(dsmem_addr(off, static_cast<uint32_t>(r)));
+        sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+      }
+      const long long o = static_cast<long long>(m) * args.N + gn;
+      if (args.C) {
+        const uint2 c2 = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(args.C) + o);
+        sum.x += bf16_lo(c2.x); sum.y += bf16_hi(c2.x);
+        sum.z += bf16_lo(c2.y); sum.w += bf16_hi(c2.y);
+      }
+      uint2 out;
+      out.x = pack_bf16x2(sum.x, sum.y);
+      out.y = pack_bf16x2(sum.z, sum.w);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(args.D) + o) = out;
+    }
+  }
+  cluster_sync_all();  // no CTA leaves while others still read its partial
+
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace dg

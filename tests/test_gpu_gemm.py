@@ -61,6 +61,46 @@ def test_dense_nt_vs_oracle(M, N, K, with_c):
     check_close(as_f64(D), R, f"dense {M}x{N}x{K}")
 
 
+# M <= 128 runs the swap-AB split-K cluster kernel (token widths 16/32/64/128)
+DECODE_CASES = [
+    (1, 256, 7168, False),
+    (16, 2112, 7168, True),
+    (17, 200, 1024, False),
+    (33, 1024, 2048, True),
+    (64, 384, 512, False),
+    (100, 2112, 3072, True),
+    (128, 4096, 1408, False),   # 11 K-blocks: uneven split
+    (128, 136, 128, True),      # a single K-block
+]
+
+
+@pytest.mark.parametrize("M,N,K,with_c", DECODE_CASES)
+def test_dense_decode_path_vs_oracle(M, N, K, with_c):
+    w = wl.dense(M, N, K, cfg=88, shape=M + N + K, with_c=with_c)
+    Cb = synth.to_bf16_bits(w.C) if with_c else None
+    qa, sa, qb, sb = quant_nt_gpu(w.A, w.B)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
+    dg.dg_fp8_gemm_nt(qa, sa, qb, sb, bf16_dev(Cb) if with_c else None, D)
+    R = oracle.gemm_nt(*quant_nt_cpu(w.A, w.B), Cb)
+    check_close(as_f64(D), R, f"decode {M}x{N}x{K}")
+
+
+def test_decode_deterministic_and_c_alias():
+    M, N, K = 128, 2112, 7168
+    w = wl.dense(M, N, K, cfg=89, with_c=True)
+    Cb = synth.to_bf16_bits(w.C)
+    qa, sa, qb, sb = quant_nt_gpu(w.A, w.B)
+    outs = []
+    for _ in range(3):
+        D = bf16_dev(Cb).clone()
+        dg.dg_fp8_gemm_nt(qa, sa, qb, sb, D, D)
+        outs.append(D.view(torch.int16).cpu().numpy())
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+    R = oracle.gemm_nt(*quant_nt_cpu(w.A, w.B), Cb)
+    check_close(synth.bf16_bits_to_f32(outs[0].view(np.uint16)).astype(np.float64), R,
+                "decode C alias")
+
+
 def test_dense_c_aliases_d_and_is_added_once():
     M, N, K = 200, 384, 512
     w = wl.dense(M, N, K, cfg=81, with_c=True)
