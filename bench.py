@@ -241,7 +241,7 @@ def run_ours(args):
     device = torch.device("cuda", local)
     shapes = wl.dense_shapes()
     if args.shape:
-        shapes = [tuple(int(x) for x in args.shape.split(","))]
+        shapes = [tuple(int(x) for x in sh.split(",")) for sh in args.shape.split(";") if sh]
 
     # ---- set-up: weights quantised once, activations resident in HBM
     weights = {}
@@ -442,7 +442,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--shape", default="", help="M,N,K: time one shape only (profiling)")
+    ap.add_argument("--shape", default="",
+                    help="M,N,K[;M,N,K...]: time only these shapes (profiling)")
     ap.add_argument("--quick", action="store_true",
                     help="timed device loop only: no e2e leg, CPU baseline or clock sampling")
     args = ap.parse_args()

@@ -129,10 +129,16 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
 
 int take_drop_flag() { return g_drop_next.exchange(0); }
 
-// Tile width: 256 columns unless that leaves the GPU with clearly fewer
+// Tile width (DG_FORCE_BN=128|256 overrides it, for tuning): 256 columns
+// unless that leaves the GPU with clearly fewer
 // waves' worth of work than 128-column tiles (a 128-wide tile costs about half
 // of a 256-wide one, with ~15% lower per-tile efficiency).
 int choose_bn(long long m_blocks, int N, int sms) {
+  static const int forced = [] {
+    const char* e = std::getenv("DG_FORCE_BN");
+    return e ? std::atoi(e) : 0;
+  }();
+  if (forced == 128 || forced == 256) return forced;
   const long long t256 = m_blocks * ((N + 255) / 256);
   const long long t128 = m_blocks * ((N + 127) / 128);
   const double c256 = 2.0 * static_cast<double>((t256 + sms - 1) / sms);

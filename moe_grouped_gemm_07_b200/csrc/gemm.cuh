@@ -13,13 +13,13 @@
 //   warp 0      TMA producer: A/B tiles (128B-swizzled) into an S-stage ring
 //               (plus, for K-grouped, the per-K-block scale vectors).
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer: for each
-//               K-block, 4 x (M=128, N=BN, K=32) MMAs into one of two TMEM
-//               accumulator buffers (2 x BN columns), reset per K-block.
+//               K-block, 4 x (M=128, N=BN, K=32) MMAs into one of 512/BN TMEM
+//               accumulator buffers (all 512 columns), reset per K-block.
 //   warps 2..9  promotion / epilogue: warp w reads TMEM lane quadrant (w % 4)
 //               and column half ((w - 2) / 4); acc += s * P in registers;
 //               at tile end adds C, converts and stores D.
-// The MMA of K-block j+1 overlaps the promotion of K-block j (double-buffered
-// TMEM); the producer runs up to S K-blocks ahead.
+// The MMA runs up to 512/BN - 1 K-blocks ahead of the promotion (2 buffers at
+// BN=256, 4 at BN=128); the producer runs up to S K-blocks ahead.
 #pragma once
 
 #include <cstdint>
@@ -63,16 +63,24 @@ struct GemmCfg {
   static constexpr int B_BYTES = BN * BK;
   static constexpr int SCALE_BYTES = (BM + BN) * 4;
   static constexpr int THREADS = 320;
-  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int NACC = 512 / BN;  // TMEM accumulator buffers (all 512 columns)
+  static constexpr int TMEM_COLS = NACC * BN;
   static constexpr int EPI_COLS = BN / 2;  // accumulator columns per promotion thread
+
   static constexpr int GROUP_M = 16;       // tile rasterisation group (L2 reuse)
   static constexpr bool KG = MODE == MODE_KGROUPED;
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_SCALE = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_BAR = OFF_SCALE + (KG ? SCALE_SLOTS * SCALE_BYTES : 0);
-  static constexpr int NUM_BARS = 2 * STAGES + 4 + 2 * SCALE_SLOTS + 1;
+  // NT modes: per promotion warp, a ring of SRING K-blocks of scales (32 sfa
+  // values for the warp's rows + 1 sfb value for its column half), filled by
+  // cp.async SRING K-blocks ahead
+  static constexpr int SRING = 8;
+  static constexpr int SRING_FLOATS = 8 * SRING * 33;
+  static constexpr int OFF_BAR =
+      OFF_SCALE + (KG ? SCALE_SLOTS * SCALE_BYTES : ((SRING_FLOATS * 4 + 127) / 128) * 128);
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * NACC + 2 * SCALE_SLOTS + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;       // tmem slot, abort flag
   static constexpr int OFF_PREFIX = OFF_MISC + 16;              // masked: prefix + counts
   static constexpr int PREFIX_BYTES = MODE == MODE_MASKED ? (2 * kMaxMaskedGroups + 1) * 4 : 0;
@@ -212,11 +220,12 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
+  constexpr int NA = Cfg::NACC;
   uint64_t* tfull = bars + 2 * S;
-  uint64_t* tempty = bars + 2 * S + 2;
-  uint64_t* sfull = bars + 2 * S + 4;
-  uint64_t* sempty = bars + 2 * S + 4 + SS;
-  uint64_t* mma_done = bars + 2 * S + 4 + 2 * SS;
+  uint64_t* tempty = bars + 2 * S + NA;
+  uint64_t* sfull = bars + 2 * S + 2 * NA;
+  uint64_t* sempty = bars + 2 * S + 2 * NA + SS;
+  uint64_t* mma_done = bars + 2 * S + 2 * NA + 2 * SS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
   int* prefix = reinterpret_cast<int*>(smem + Cfg::OFF_PREFIX);
@@ -232,7 +241,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NA; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 8);
     }
@@ -357,8 +366,8 @@ __global__ void __launch_bounds__(320, 1)
         const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped);
         if (!tl.valid) continue;
         for (int kb = 0; kb < tl.nkb; ++kb, ++it, ++acc_it) {
-          const uint32_t b = acc_it & 1;
-          if (!mbar_wait(&tempty[b], ((acc_it >> 1) & 1) ^ 1, abort_flag, tmo, SITE_MMA_TMEM_EMPTY))
+          const uint32_t b = acc_it % NA;
+          if (!mbar_wait(&tempty[b], ((acc_it / NA) & 1) ^ 1, abort_flag, tmo, SITE_MMA_TMEM_EMPTY))
             goto mma_done_label;
           tc_fence_after();
           const uint32_t s = it % S;
@@ -428,89 +437,90 @@ __global__ void __launch_bounds__(320, 1)
         half_in = col_first < args.N;
         pb = args.sfb + (static_cast<long long>(tl.g) * nbN + col_first / 128) * KBn;
       }
-      // Prefetch ring of 4 K-blocks; the K-block loop is unrolled by 4 so
-      // slot u is consumed and refilled in place (no register moves that
-      // would wait on an in-flight load).
-      float sa[4] = {0.f, 0.f, 0.f, 0.f};
-      float sb[4] = {0.f, 0.f, 0.f, 0.f};
-      if constexpr (!Cfg::KG) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (u < tl.nkb) {
-            if (half_in) sb[u] = __ldg(pb + u);
-            if (row_in) sa[u] = __ldg(pa + static_cast<long long>(u) * args.ld_sfa);
-          }
+      // NT scales stream through this warp's shared-memory ring by cp.async,
+      // SRING K-blocks ahead: lane l copies sfa for its row, lane 0 also the
+      // sfb value of the warp's column half. Every iteration commits exactly
+      // one cp.async group, so wait_group<SRING-1> means "K-block kb landed".
+      constexpr int SR = Cfg::SRING;
+      float* ring = reinterpret_cast<float*>(sScale) + (warp - 2) * (SR * 33);
+      auto issue_scales = [&](int kb) {
+        if (kb < tl.nkb) {
+          float* slot = ring + (kb % SR) * 33;
+          if (row_in) cp_async_4(slot + lane, pa + static_cast<long long>(kb) * args.ld_sfa);
+          if (lane == 0 && half_in) cp_async_4(slot + 32, pb + kb);
         }
+        cp_async_commit();
+      };
+      if constexpr (!Cfg::KG) {
+#pragma unroll 1
+        for (int u = 0; u < SR; ++u) issue_scales(u);
       }
 
-      for (int kb0 = 0; kb0 < tl.nkb; kb0 += 4) {
+      for (int kb = 0; kb < tl.nkb; ++kb) {
+        const uint32_t b = acc_it % NA;
+        bool ok = mbar_wait(&tfull[b], (acc_it / NA) & 1, abort_flag, tmo, SITE_EPI_TMEM_FULL);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) goto epi_done;
+        tc_fence_after();
+        if constexpr (!Cfg::KG) {
+          cp_async_wait<SR - 1>();
+          __syncwarp();
+          const float* slot = ring + (kb % SR) * 33;
+          const float sc = (row_in ? slot[lane] : 0.f) * (half_in ? slot[32] : 0.f);
+          __syncwarp();
+          issue_scales(kb + SR);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int kb = kb0 + u;
-          if (kb >= tl.nkb) break;
-          const uint32_t b = acc_it & 1;
-          bool ok = mbar_wait(&tfull[b], (acc_it >> 1) & 1, abort_flag, tmo, SITE_EPI_TMEM_FULL);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) goto epi_done;
-          tc_fence_after();
-          if constexpr (!Cfg::KG) {
-            const float sc = sa[u] * sb[u];
-            if (kb + 4 < tl.nkb) {
-              sb[u] = half_in ? __ldg(pb + kb + 4) : 0.f;
-              sa[u] = row_in ? __ldg(pa + static_cast<long long>(kb + 4) * args.ld_sfa) : 0.f;
+          for (int c = 0; c < EC / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
+            tmem_ld_wait();
+            if (c == EC / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[b]);
             }
 #pragma unroll
-            for (int c = 0; c < EC / 32; ++c) {
-              uint32_t r[32];
-              tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
-              tmem_ld_wait();
-              if (c == EC / 32 - 1) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[b]);
-              }
-#pragma unroll
-              for (int i = 0; i < 32; i += 2)
-                fma2(acc[c * 32 + i], acc[c * 32 + i + 1], sc, sc, __uint_as_float(r[i]),
-                     __uint_as_float(r[i + 1]));
-            }
-          } else {
-            const uint32_t ss = sit % SS;
-            bool ok2 = mbar_wait(&sfull[ss], (sit / SS) & 1, abort_flag, tmo, SITE_EPI_SCALE_FULL);
-            ok2 = __all_sync(0xffffffffu, ok2);
-            if (!ok2) goto epi_done;
-            const float* slot = sScale + ss * (Cfg::BM + BN);
-            const float sav = slot[r_in_tile];
-            const float* sbv = slot + Cfg::BM + h * EC;
-#pragma unroll
-            for (int c = 0; c < EC / 32; ++c) {
-              uint32_t r[32];
-              tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
-              tmem_ld_wait();
-              if (c == EC / 32 - 1) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[b]);
-              }
-#pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                const float4 sb4 = *reinterpret_cast<const float4*>(sbv + c * 32 + i);
-                float t0, t1, t2, t3;
-                mul2(t0, t1, sav, sav, sb4.x, sb4.y);
-                mul2(t2, t3, sav, sav, sb4.z, sb4.w);
-                fma2(acc[c * 32 + i], acc[c * 32 + i + 1], t0, t1, __uint_as_float(r[i]),
-                     __uint_as_float(r[i + 1]));
-                fma2(acc[c * 32 + i + 2], acc[c * 32 + i + 3], t2, t3, __uint_as_float(r[i + 2]),
-                     __uint_as_float(r[i + 3]));
-              }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sempty[ss]);
-            ++sit;
+            for (int i = 0; i < 32; i += 2)
+              fma2(acc[c * 32 + i], acc[c * 32 + i + 1], sc, sc, __uint_as_float(r[i]),
+                   __uint_as_float(r[i + 1]));
           }
-          ++acc_it;
+        } else {
+          const uint32_t ss = sit % SS;
+          bool ok2 = mbar_wait(&sfull[ss], (sit / SS) & 1, abort_flag, tmo, SITE_EPI_SCALE_FULL);
+          ok2 = __all_sync(0xffffffffu, ok2);
+          if (!ok2) goto epi_done;
+          const float* slot = sScale + ss * (Cfg::BM + BN);
+          const float sav = slot[r_in_tile];
+          const float* sbv = slot + Cfg::BM + h * EC;
+#pragma unroll
+          for (int c = 0; c < EC / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
+            tmem_ld_wait();
+            if (c == EC / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[b]);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 sb4 = *reinterpret_cast<const float4*>(sbv + c * 32 + i);
+              float t0, t1, t2, t3;
+              mul2(t0, t1, sav, sav, sb4.x, sb4.y);
+              mul2(t2, t3, sav, sav, sb4.z, sb4.w);
+              fma2(acc[c * 32 + i], acc[c * 32 + i + 1], t0, t1, __uint_as_float(r[i]),
+                   __uint_as_float(r[i + 1]));
+              fma2(acc[c * 32 + i + 2], acc[c * 32 + i + 3], t2, t3, __uint_as_float(r[i + 2]),
+                   __uint_as_float(r[i + 3]));
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sempty[ss]);
+          ++sit;
         }
+        ++acc_it;
       }
+      if constexpr (!Cfg::KG) cp_async_wait<0>();
 
       // ------------------------------------------------ tile epilogue
       {
@@ -566,7 +576,8 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
     }
-  epi_done:;
+  epi_done:
+    cp_async_wait<0>();  // no shared-memory copy may land after the CTA exits
   }
 
   // ---------------------------------------------------------------- teardown
