@@ -109,8 +109,8 @@ dg_status make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, 
 // ---------------------------------------------------------------- launches
 template <int MODE, int BN>
 dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
-                      const CUtensorMap& tsb, const GemmArgs& args, int grid, cudaStream_t st,
-                      int dev) {
+                      const CUtensorMap& tsb, const CUtensorMap& td, const GemmArgs& args,
+                      int grid, cudaStream_t st, int dev) {
   using Cfg = dg::GemmCfg<MODE, BN>;
   static std::once_flag once[kMaxDevices];
   static cudaError_t attr_err[kMaxDevices];
@@ -120,7 +120,7 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
   });
   if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(ta, tb, tsa, tsb, args);
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(ta, tb, tsa, tsb, td, args);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   g_launches.fetch_add(1);
@@ -190,12 +190,18 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
   s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, static_cast<uint64_t>(G) * N, K, 128,
                   bn, CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DG_OK) return s;
+  // D as [rows_total][N] bf16; 32x32 boxes, 64-byte swizzle (TMA-store epilogue)
+  CUtensorMap td;
+  s = make_map_2d(&td, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, rows_total, 2ull * N, 32, 32,
+                  CU_TENSOR_MAP_SWIZZLE_64B);
+  if (s != DG_OK) return s;
   GemmArgs args;
   std::memset(&args, 0, sizeof args);
   args.M = M_logical;
   args.N = N;
   args.K = K;
   args.G = G;
+  args.d_rows = rows_total;
   args.num_m_blocks = static_cast<int>((MODE == dg::MODE_MASKED) ? (M_logical + 127) / 128
                                                                   : (rows_total + 127) / 128);
   args.num_n_blocks = (N + bn - 1) / bn;
@@ -216,8 +222,8 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
   if (print_configs())
     std::fprintf(stderr, "[dg] %s M=%d N=%d K=%d G=%d: BM=128 BN=%d tiles=%lld grid=%d\n", name,
                  M_logical, N, K, G, bn, tiles, grid);
-  if (bn == 256) return launch_gemm<MODE, 256>(ta, tb, dummy, dummy, args, grid, st, dev);
-  return launch_gemm<MODE, 128>(ta, tb, dummy, dummy, args, grid, st, dev);
+  if (bn == 256) return launch_gemm<MODE, 256>(ta, tb, dummy, dummy, td, args, grid, st, dev);
+  return launch_gemm<MODE, 128>(ta, tb, dummy, dummy, td, args, grid, st, dev);
 }
 
 // ---------------------------------------------------------------- decode path
@@ -541,12 +547,17 @@ dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void* A, const float* sfa, c
   if ((s = make_map_2d(&tsb, sfb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, sumKB, 4ull * N, bn, 1,
                        CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
     return s;
+  CUtensorMap td;  // D as [G*M][N] fp32; 16x32 boxes, 64-byte swizzle
+  if ((s = make_map_2d(&td, D, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, static_cast<uint64_t>(G) * M,
+                       4ull * N, 16, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != DG_OK)
+    return s;
   GemmArgs args;
   std::memset(&args, 0, sizeof args);
   args.M = M;
   args.N = N;
   args.K = 0;
   args.G = G;
+  args.d_rows = static_cast<long long>(G) * M;
   args.num_m_blocks = mb;
   args.num_n_blocks = (N + bn - 1) / bn;
   const long long tiles = static_cast<long long>(G) * mb * args.num_n_blocks;
@@ -565,8 +576,9 @@ dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void* A, const float* sfa, c
   if (print_configs())
     std::fprintf(stderr, "[dg] k_grouped_fp8_gemm_tn M=%d N=%d sumK=%lld G=%d: BN=%d tiles=%lld grid=%d\n",
                  M, N, sumK, G, bn, tiles, grid);
-  if (bn == 256) return launch_gemm<dg::MODE_KGROUPED, 256>(ta, tb, tsa, tsb, args, grid, st, dev);
-  return launch_gemm<dg::MODE_KGROUPED, 128>(ta, tb, tsa, tsb, args, grid, st, dev);
+  if (bn == 256)
+    return launch_gemm<dg::MODE_KGROUPED, 256>(ta, tb, tsa, tsb, td, args, grid, st, dev);
+  return launch_gemm<dg::MODE_KGROUPED, 128>(ta, tb, tsa, tsb, td, args, grid, st, dev);
 }
 
 }  // extern "C"

@@ -47,6 +47,7 @@ struct GemmArgs {
   const int32_t* masked_m;
   const void* C;
   void* D;
+  long long d_rows;  // rows of D viewed as [d_rows][N] (the store tensor map's outer extent)
   unsigned long long timeout_ns;
   int drop_arrive;
   int kb_off[kMaxKGroups + 1];  // K-grouped: prefix sums of K-blocks per group
@@ -78,8 +79,13 @@ struct GemmCfg {
   // cp.async SRING K-blocks ahead
   static constexpr int SRING = 8;
   static constexpr int SRING_FLOATS = 8 * SRING * 33;
-  static constexpr int OFF_BAR =
-      OFF_SCALE + (KG ? SCALE_SLOTS * SCALE_BYTES : ((SRING_FLOATS * 4 + 127) / 128) * 128);
+  static constexpr int OFF_STAGE =
+      ((OFF_SCALE + (KG ? SCALE_SLOTS * SCALE_BYTES : SRING_FLOATS * 4) + 1023) / 1024) * 1024;
+  // output staging for the TMA-store epilogue: one 32-row x 64-byte chunk
+  // (32 bf16 or 16 fp32 columns) per promotion warp, 64-byte swizzled
+  static constexpr int STAGE_BYTES_PER_WARP = 32 * 64;
+  static constexpr int STORE_COLS = KG ? 16 : 32;
+  static constexpr int OFF_BAR = OFF_STAGE + 8 * STAGE_BYTES_PER_WARP;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NACC + 2 * SCALE_SLOTS + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;       // tmem slot, abort flag
   static constexpr int OFF_PREFIX = OFF_MISC + 16;              // masked: prefix + counts
@@ -89,6 +95,7 @@ struct GemmCfg {
   // TMA destinations: 128-byte aligned; 128B-swizzled tiles 1024-byte aligned
   static_assert(OFF_B % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "tiles");
   static_assert(OFF_SCALE % 128 == 0 && SCALE_BYTES % 128 == 0 && (BM * 4) % 128 == 0, "scales");
+  static_assert(OFF_STAGE % 1024 == 0, "swizzled staging");
   static_assert(BN == 128 || BN == 256, "BN");
 };
 
@@ -206,6 +213,7 @@ __global__ void __launch_bounds__(320, 1)
                     const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_sfa,
                     const __grid_constant__ CUtensorMap tm_sfb,
+                    const __grid_constant__ CUtensorMap tm_d,
                     const __grid_constant__ GemmArgs args) {
   using Cfg = GemmCfg<MODE, BN>;
   constexpr int S = Cfg::STAGES;
@@ -217,6 +225,7 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sA = smem + Cfg::OFF_A;
   uint8_t* sB = smem + Cfg::OFF_B;
   float* sScale = reinterpret_cast<float*>(smem + Cfg::OFF_SCALE);
+  uint8_t* sStage = smem + Cfg::OFF_STAGE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
@@ -523,14 +532,69 @@ __global__ void __launch_bounds__(320, 1)
       if constexpr (!Cfg::KG) cp_async_wait<0>();
 
       // ------------------------------------------------ tile epilogue
+      // A warp whose 32 rows may all be written (or lie past the end of D,
+      // where the store clips them) stages 32-column chunks in shared memory
+      // and stores them with TMA; a warp holding rows that must stay untouched
+      // (masked rows, padding rows, another group's rows) stores directly.
       {
         bool write = r_in_tile < tl.rows;
         const long long orow = tl.out_row0 + r_in_tile;
         if constexpr (MODE == MODE_CONTIG) {
           if (write) write = __ldg(args.m_indices + orow) == tl.g;
         }
+        const bool clipped = orow >= args.d_rows;
         const int col0 = tl.n0 + static_cast<int>(h) * EC;
-        if (write) {
+        const bool use_tma = __all_sync(0xffffffffu, write || clipped);
+        if (use_tma) {
+          constexpr int CW = Cfg::STORE_COLS;
+          uint8_t* stg = sStage + (warp - 2) * Cfg::STAGE_BYTES_PER_WARP;
+          const int swz = static_cast<int>((lane >> 1) & 3);  // 64-byte swizzle of row `lane`
+#pragma unroll
+          for (int c = 0; c < EC / CW; ++c) {
+            const int n = col0 + c * CW;
+            if (n >= args.N) break;
+            if (lane == 0) bulk_wait_read0();  // previous chunk has left the staging buffer
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 o;
+              if constexpr (Cfg::KG) {
+                float v0 = acc[c * CW + j * 4 + 0], v1 = acc[c * CW + j * 4 + 1];
+                float v2 = acc[c * CW + j * 4 + 2], v3 = acc[c * CW + j * 4 + 3];
+                if (args.C && !clipped && n + j * 4 < args.N) {
+                  const float4 c4 = *reinterpret_cast<const float4*>(
+                      static_cast<const float*>(args.C) + orow * args.N + n + j * 4);
+                  v0 += c4.x; v1 += c4.y; v2 += c4.z; v3 += c4.w;
+                }
+                o = make_uint4(__float_as_uint(v0), __float_as_uint(v1), __float_as_uint(v2),
+                               __float_as_uint(v3));
+              } else {
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = acc[c * CW + j * 8 + i];
+                if (args.C && !clipped && n + j * 8 < args.N) {
+                  const uint4 c4 = *reinterpret_cast<const uint4*>(
+                      static_cast<const __nv_bfloat16*>(args.C) + orow * args.N + n + j * 8);
+                  v[0] += bf16_lo(c4.x); v[1] += bf16_hi(c4.x);
+                  v[2] += bf16_lo(c4.y); v[3] += bf16_hi(c4.y);
+                  v[4] += bf16_lo(c4.z); v[5] += bf16_hi(c4.z);
+                  v[6] += bf16_lo(c4.w); v[7] += bf16_hi(c4.w);
+                }
+                o.x = pack_bf16x2(v[0], v[1]);
+                o.y = pack_bf16x2(v[2], v[3]);
+                o.z = pack_bf16x2(v[4], v[5]);
+                o.w = pack_bf16x2(v[6], v[7]);
+              }
+              *reinterpret_cast<uint4*>(stg + lane * 64 + ((j ^ swz) << 4)) = o;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tm_d, stg, n, static_cast<int>(tl.out_row0 + q * 32));
+              bulk_commit();
+            }
+          }
+        } else if (write) {
           if constexpr (Cfg::KG) {
             float* drow = static_cast<float*>(args.D) + orow * args.N;
             const float* crow = args.C ? static_cast<const float*>(args.C) + orow * args.N : nullptr;
@@ -578,6 +642,8 @@ __global__ void __launch_bounds__(320, 1)
     }
   epi_done:
     cp_async_wait<0>();  // no shared-memory copy may land after the CTA exits
+    if (lane == 0) bulk_wait0();  // every TMA store of this warp has completed
+    __syncwarp();
   }
 
   // ---------------------------------------------------------------- teardown
