@@ -418,7 +418,7 @@ dg_status dg_quantize_fp8(const void* x, int in_dtype, int batch, int rows, int 
   const bool bf = in_dtype == DG_IN_BF16;
   if (mode == DG_QUANT_ROW_1x128) {
     const long long strips = static_cast<long long>(batch) * rows * (cols / 128);
-    const int grid = static_cast<int>(std::min<long long>((strips + 7) / 8, 8ll * sms));
+    const int grid = static_cast<int>(std::min<long long>((strips + 31) / 32, 8ll * sms));
     if (bf) dg::quant_row_kernel<true><<<grid, 256, 0, st>>>(x, batch, rows, cols, q, scales, ld_scales);
     else dg::quant_row_kernel<false><<<grid, 256, 0, st>>>(x, batch, rows, cols, q, scales, ld_scales);
   } else if (mode == DG_QUANT_BLOCK_128x128) {

@@ -1,8 +1,9 @@
 // quant.cuh -- BF16/FP32 -> E4M3 quantisers with FP32 scales, sm_100a.
 //
-// scale = max(amax, 1e-4f) / 448 and code = E4M3_RN_satfinite(x / scale), both
-// IEEE single-precision divisions (this file must not be built with
-// --use_fast_math). Three scale granularities:
+// scale = max(amax, 1e-4f) / 448 (IEEE division) and
+// code = E4M3_RN_satfinite(x / scale) with the quotient rounded exactly as the
+// IEEE division would round it (see quotient()); this file must not be built
+// with --use_fast_math. Three scale granularities:
 //   ROW   one scale per (row, 128-column strip), stored transposed [cols/128][ld]
 //   BLOCK one scale per 128x128 block, [ceil(rows/128)][cols/128]
 //   COL   one scale per (128-row strip, column), [rows/128][cols]
@@ -43,9 +44,25 @@ __device__ __forceinline__ float scale_from_amax(float amax) {
   return fmaxf(amax, 1e-4f) / 448.0f;  // IEEE division (no fast-math)
 }
 
+// x / s rounded to nearest (the IEEE quotient), from r = 1/s correctly rounded
+// and one FMA correction step (Markstein, "Computation of elementary functions
+// on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990: if r is
+// 1/s within half an ulp and q0 is within one ulp of x/s, q0 + r*(x - s*q0)
+// rounds to the correctly rounded quotient). The residual is exact unless
+// |x| < 2^-103; with s >= 1e-4/448 such quotients are below 2^-81 and encode
+// to a signed zero either way, so the E4M3 code always equals that of the
+// IEEE division. The sign is taken from x so that -0 / s = -0.
+__device__ __forceinline__ float quotient(float x, float s, float r) {
+  const float ax = fabsf(x);
+  const float q0 = __fmul_rn(ax, r);
+  const float e = fmaf(-q0, s, ax);
+  return copysignf(fmaf(e, r, q0), x);
+}
+
 // Four E4M3 codes packed little-endian (element 0 in the low byte).
-__device__ __forceinline__ uint32_t encode4(const float (&v)[4], float s) {
-  const float y0 = v[0] / s, y1 = v[1] / s, y2 = v[2] / s, y3 = v[3] / s;
+__device__ __forceinline__ uint32_t encode4(const float (&v)[4], float s, float r) {
+  const float y0 = quotient(v[0], s, r), y1 = quotient(v[1], s, r);
+  const float y2 = quotient(v[2], s, r), y3 = quotient(v[3], s, r);
   const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
   const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(y2, y3), __NV_SATFINITE, __NV_E4M3);
   return (lo & 0xFFFFu) | (hi << 16);
@@ -57,31 +74,42 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// ROW_1x128: one warp per 128-element strip; strips enumerated (batch, row,
-// strip) with the strip index fastest so consecutive warps stream each row.
+// ROW_1x128: strips enumerated (batch, row, strip) with the strip index
+// fastest, so strip s covers elements [128 s, 128 s + 128) of x. Each warp
+// takes 4 consecutive strips per step (2 KB of input in flight per warp).
 template <bool BF16>
 __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__ x, int batch,
                                                         int rows, int cols,
                                                         uint8_t* __restrict__ codes,
                                                         float* __restrict__ scales, int ld) {
+  constexpr int U = 4;
   const int lane = threadIdx.x & 31;
   const int kbs = cols >> 7;
   const int64_t nstrips = static_cast<int64_t>(batch) * rows * kbs;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t s = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; s < nstrips;
-       s += nwarps) {
-    const int kb = static_cast<int>(s % kbs);
-    const int64_t br = s / kbs;  // batch * rows + row
-    const int64_t base = br * cols + (kb << 7) + (lane << 2);
-    const In4 in = load4<BF16>(x, base);
-    float amax = fmaxf(fmaxf(fabsf(in.v[0]), fabsf(in.v[1])), fmaxf(fabsf(in.v[2]), fabsf(in.v[3])));
-    amax = warp_max(amax);
-    const float sc = scale_from_amax(amax);
-    *reinterpret_cast<uint32_t*>(codes + base) = encode4(in.v, sc);
-    if (lane == 0) {
-      const int64_t b = br / rows;
-      const int r = static_cast<int>(br - b * rows);
-      scales[(b * kbs + kb) * ld + r] = sc;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  for (int64_t s0 = warp0 * U; s0 < nstrips; s0 += nwarps * U) {
+    In4 in[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (s0 + u < nstrips) in[u] = load4<BF16>(x, (s0 + u) * 128 + (lane << 2));
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t st = s0 + u;
+      if (st >= nstrips) break;
+      float amax = fmaxf(fmaxf(fabsf(in[u].v[0]), fabsf(in[u].v[1])),
+                         fmaxf(fabsf(in[u].v[2]), fabsf(in[u].v[3])));
+      amax = warp_max(amax);
+      const float sc = scale_from_amax(amax);
+      const float rc = __frcp_rn(sc);
+      *reinterpret_cast<uint32_t*>(codes + st * 128 + (lane << 2)) = encode4(in[u].v, sc, rc);
+      if (lane == 0) {
+        const int kb = static_cast<int>(st % kbs);
+        const int64_t br = st / kbs;  // batch * rows + row
+        const int64_t b = br / rows;
+        const int r = static_cast<int>(br - b * rows);
+        scales[(b * kbs + kb) * ld + r] = sc;
+      }
     }
   }
 }
@@ -118,12 +146,13 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
 #pragma unroll
   for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
   const float sc = scale_from_amax(a);
+  const float rc = __frcp_rn(sc);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int r = (nb << 7) + (w << 4) + i;
     if (r < rows)
       *reinterpret_cast<uint32_t*>(codes + (b * rows + r) * cols + (kb << 7) + (lane << 2)) =
-          encode4(v[i].v, sc);
+          encode4(v[i].v, sc, rc);
   }
   if (threadIdx.x == 0) scales[(b * nbs + nb) * kbs + kb] = sc;
 }
@@ -137,6 +166,7 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const void* __restrict__
                                                         float* __restrict__ scales) {
   __shared__ float red[16][64];
   __shared__ float sc_s[64];
+  __shared__ float rc_s[64];
   const int cg = threadIdx.x & 15, rg = threadIdx.x >> 4;
   const int slabs = (cols + 63) >> 6, rbs = rows >> 7;
   const int64_t blk = blockIdx.x;
@@ -165,6 +195,7 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const void* __restrict__
     for (int i = 1; i < 16; ++i) a = fmaxf(a, red[i][threadIdx.x]);
     const float sc = scale_from_amax(a);
     sc_s[threadIdx.x] = sc;
+    rc_s[threadIdx.x] = __frcp_rn(sc);
     const int cc = (slab << 6) + threadIdx.x;
     if (cc < cols) scales[(b * rbs + rb) * cols + cc] = sc;
   }
@@ -173,8 +204,11 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const void* __restrict__
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int r = (rb << 7) + rg + (i << 4);
-    const float y0 = v[i].v[0] / sc_s[(cg << 2) + 0], y1 = v[i].v[1] / sc_s[(cg << 2) + 1];
-    const float y2 = v[i].v[2] / sc_s[(cg << 2) + 2], y3 = v[i].v[3] / sc_s[(cg << 2) + 3];
+    const int c0 = cg << 2;
+    const float y0 = quotient(v[i].v[0], sc_s[c0 + 0], rc_s[c0 + 0]);
+    const float y1 = quotient(v[i].v[1], sc_s[c0 + 1], rc_s[c0 + 1]);
+    const float y2 = quotient(v[i].v[2], sc_s[c0 + 2], rc_s[c0 + 2]);
+    const float y3 = quotient(v[i].v[3], sc_s[c0 + 3], rc_s[c0 + 3]);
     const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
     const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(y2, y3), __NV_SATFINITE, __NV_E4M3);
     *reinterpret_cast<uint32_t*>(codes + (b * rows + r) * cols + c) = (lo & 0xFFFFu) | (hi << 16);

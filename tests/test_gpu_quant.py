@@ -109,3 +109,31 @@ def test_quant_rejects_bad_shapes():
     with pytest.raises(dg.DGError) as e:
         dg.dg_quantize_fp8(x, dg.DG_QUANT_ROW_1x128)
     assert e.value.status == dg.DG_ERR_UNSUPPORTED_SHAPE
+
+
+def test_quotient_near_rounding_boundaries():
+    """Every strip gets a random amax (so a random scale s), and its other 127
+    values sit within a few float32 ulps of s times an E4M3 rounding boundary
+    (a midpoint between neighbouring codes), either sign. The codes must match
+    the oracle, which divides with IEEE float division."""
+    t = oracle.e4m3_table()
+    pos = np.array(sorted(set(float(v) for v in t[:0x7F])))
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)
+    strips = 8192
+    u = synth.u64(strips * 130, synth.seed(73, 1))
+    amax = np.ldexp(0.5 + (u[:strips] >> np.uint64(11)).astype(np.float64) / 2.0 ** 53,
+                    (u[strips:2 * strips] % np.uint64(50)).astype(np.int64) - 30).astype(np.float32)
+    amax[::97] = np.float32(3e-5)              # below the 1e-4 floor
+    s = (np.maximum(amax, np.float32(1e-4)) / np.float32(448.0)).astype(np.float32)
+    pick = (u[2 * strips:2 * strips + strips * 127] % np.uint64(mids.size)).astype(np.int64)
+    base = (mids[pick].reshape(strips, 127) * s[:, None]).astype(np.float32)
+    nudge = (u[:strips * 127] % np.uint64(9)).astype(np.int64).reshape(strips, 127) - 4
+    bits = base.view(np.int32) + nudge.astype(np.int32)
+    vals = bits.view(np.float32)
+    vals = np.minimum(vals, amax[:, None])      # keep amax the strip maximum
+    sign = np.where((u[:strips * 127] >> np.uint64(7)) & np.uint64(1), -1.0, 1.0).astype(np.float32)
+    x = np.empty((strips, 128), dtype=np.float32)
+    x[:, 0] = amax
+    x[:, 1:] = vals * sign.reshape(strips, 127)
+    gc, gsf, oc, osf = run_both(x, "row")
+    assert_bit_exact(gc, gsf, oc, osf)
