@@ -162,6 +162,12 @@ void dg_set_num_sms(int n);
 int dg_get_num_sms(void);
 /* Bounded-wait limit in nanoseconds for subsequent launches (0 = default 2 s). */
 void dg_set_wait_timeout_ns(uint64_t ns);
+/* Programmatic dependent launch (default on): each launch may start its
+ * prologue while the previous kernel on the stream finishes; every kernel of
+ * this library waits for its predecessor before reading global memory.
+ * Source: README summary, section "ユーティリティと環境変数" (set_pdl / get_pdl). */
+void dg_set_pdl(int enable);
+int dg_get_pdl(void);
 
 /* Synchronises `stream`, then reads and clears this device's error word.
  * Returns DG_OK, DG_ERR_TIMEOUT (a bounded wait ran out; *site gets the code

@@ -11,7 +11,8 @@ Functions keep the C names:
   dg_m_grouped_fp8_gemm_nt_masked, dg_k_grouped_fp8_gemm_tn_contiguous,
   dg_get_mk_alignment_for_contiguous_layout, dg_get_tma_aligned_size,
   dg_set_num_sms, dg_get_num_sms, dg_set_wait_timeout_ns,
-  dg_get_last_device_error, dg_debug_drop_next_arrive, dg_get_launch_count.
+  dg_get_last_device_error, dg_debug_drop_next_arrive, dg_get_launch_count,
+  dg_set_pdl, dg_get_pdl.
 """
 from __future__ import annotations
 
@@ -40,6 +41,7 @@ EXPORTED = (
     "dg_k_grouped_fp8_gemm_tn_contiguous", "dg_get_mk_alignment_for_contiguous_layout",
     "dg_get_tma_aligned_size", "dg_set_num_sms", "dg_get_num_sms", "dg_set_wait_timeout_ns",
     "dg_get_last_device_error", "dg_debug_drop_next_arrive", "dg_get_launch_count",
+    "dg_set_pdl", "dg_get_pdl",
 )
 
 _vp, _i32 = _C.c_void_p, _C.c_int
@@ -66,6 +68,8 @@ _lib.dg_get_last_device_error.argtypes = [_vp, _C.POINTER(_C.c_int)]
 _lib.dg_get_last_device_error.restype = _i32
 _lib.dg_debug_drop_next_arrive.argtypes = [_i32]
 _lib.dg_get_launch_count.restype = _C.c_uint64
+_lib.dg_set_pdl.argtypes = [_i32]
+_lib.dg_get_pdl.restype = _i32
 
 
 class DGError(RuntimeError):
@@ -257,3 +261,11 @@ def dg_debug_drop_next_arrive(enable: bool = True) -> None:
 
 def dg_get_launch_count() -> int:
     return int(_lib.dg_get_launch_count())
+
+
+def dg_set_pdl(enable: bool) -> None:
+    _lib.dg_set_pdl(1 if enable else 0)
+
+
+def dg_get_pdl() -> bool:
+    return bool(_lib.dg_get_pdl())

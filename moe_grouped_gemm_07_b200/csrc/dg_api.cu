@@ -26,6 +26,36 @@ std::atomic<int> g_num_sms_cap{0};
 std::atomic<unsigned long long> g_timeout_ns{0};
 std::atomic<int> g_drop_next{0};
 std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_pdl{1};
+
+// Launches `kern` on `st`, with programmatic dependent launch when enabled
+// (dg_set_pdl) and with a 1-D cluster of `cluster` CTAs when cluster > 1.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   int cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (g_pdl.load()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 int g_sm_count[kMaxDevices];
 std::once_flag g_sm_once[kMaxDevices];
@@ -120,8 +150,8 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
   });
   if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(ta, tb, tsa, tsb, td, args);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, 1, ta, tb, tsa,
+                         tsb, td, args);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   g_launches.fetch_add(1);
   return DG_OK;
@@ -149,6 +179,8 @@ int choose_bn(long long m_blocks, int N, int sms) {
 // D = C (or 0) for K == 0 / all-empty K-grouped problems.
 template <typename T>
 __global__ void copy_or_zero_kernel(const T* __restrict__ c, T* __restrict__ d, long long n) {
+  dg::pdl_wait();
+  dg::pdl_trigger();
   for (long long i = blockIdx.x * 1ll * blockDim.x + threadIdx.x; i < n;
        i += 1ll * gridDim.x * blockDim.x)
     d[i] = c ? c[i] : T(0);
@@ -159,8 +191,8 @@ dg_status copy_or_zero(const void* c, void* d, long long n, int sms, cudaStream_
   if (n <= 0) return DG_OK;
   if (c == d) return DG_OK;
   const int grid = static_cast<int>(std::min<long long>((n + 255) / 256, 8ll * sms));
-  copy_or_zero_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(c), static_cast<T*>(d), n);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch(copy_or_zero_kernel<T>, dim3(grid), dim3(256), 0, st, 1,
+                         static_cast<const T*>(c), static_cast<T*>(d), n);
   if (e != cudaSuccess) return cuda_fail(e, "copy launch");
   g_launches.fetch_add(1);
   return DG_OK;
@@ -227,8 +259,9 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
 }
 
 // ---------------------------------------------------------------- decode path
-// Largest cluster size (1..8, powers of two) that the device can co-schedule
-// for this kernel; cached per device and instantiation.
+// Largest cluster size (1..16) that the device can co-schedule for this
+// kernel (above 8 only where non-portable cluster sizes are allowed); cached
+// per device and instantiation.
 template <int BNP>
 int max_cluster(int dev) {
   using Cfg = dg::DecodeCfg<BNP>;
@@ -240,7 +273,11 @@ int max_cluster(int dev) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM_BYTES) != cudaSuccess)
       return;
-    for (int c = 8; c >= 1; c >>= 1) {
+    const bool nonportable =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+        cudaSuccess;
+    cudaGetLastError();
+    for (int c = nonportable ? 16 : 8; c >= 1; --c) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(c, 1, 1);
       cfg.blockDim = dim3(320, 1, 1);
@@ -253,7 +290,8 @@ int max_cluster(int dev) {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) {
+      // enough co-resident clusters of this size to fill most of the GPU
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n * c >= 64) {
         best[dev] = c;
         return;
       }
@@ -263,12 +301,14 @@ int max_cluster(int dev) {
   return best[dev];
 }
 
-// Split count: double the CTAs per N-tile while the launch still fits in two
-// CTAs per SM and every CTA keeps at least two K-blocks.
+// Split count: double the CTAs per N-tile (up to 8, a cluster size every
+// GPC can co-schedule many times over) while the launch still fits in two
+// CTAs per SM and every CTA keeps at least two K-blocks. Measured: 16-CTA
+// clusters do not all fit at once, and uneven splits lengthen the reduction.
 int choose_splits(int n_tiles, int KB, int sms, int cap) {
   int splits = 1;
-  while (splits * 2 <= cap && static_cast<long long>(n_tiles) * splits * 2 <= 2ll * sms &&
-         KB / (splits * 2) >= 2)
+  while (splits * 2 <= (cap < 8 ? cap : 8) &&
+         static_cast<long long>(n_tiles) * splits * 2 <= 2ll * sms && KB / (splits * 2) >= 2)
     splits *= 2;
   return splits;
 }
@@ -312,20 +352,8 @@ dg_status run_decode(const void* A, const float* sfa, const void* B, const float
                  "[dg] fp8_gemm_nt decode M=%d N=%d K=%d: swap-AB BNP=%d, n_tiles=%d x "
                  "split-K %d (cluster), %d CTAs, %d stages\n",
                  M, N, K, BNP, n_tiles, splits, n_tiles * splits, Cfg::STAGES);
-  auto kern = dg::gemm_decode_kernel<BNP>;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(splits, n_tiles, 1);
-  cfg.blockDim = dim3(320, 1, 1);
-  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = splits;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, tsa, args);
+  cudaError_t e = launch(dg::gemm_decode_kernel<BNP>, dim3(splits, n_tiles, 1), dim3(320),
+                         Cfg::SMEM_BYTES, st, splits, tw, tx, tsa, args);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   g_launches.fetch_add(1);
   return DG_OK;
@@ -375,6 +403,10 @@ int dg_get_num_sms(void) {
 
 void dg_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns); }
 
+void dg_set_pdl(int enable) { g_pdl.store(enable ? 1 : 0); }
+
+int dg_get_pdl(void) { return g_pdl.load(); }
+
 void dg_debug_drop_next_arrive(int enable) { g_drop_next.store(enable ? 1 : 0); }
 
 uint64_t dg_get_launch_count(void) { return g_launches.load(); }
@@ -416,23 +448,30 @@ dg_status dg_quantize_fp8(const void* x, int in_dtype, int batch, int rows, int 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* q = static_cast<uint8_t*>(codes);
   const bool bf = in_dtype == DG_IN_BF16;
+  cudaError_t e = cudaSuccess;
   if (mode == DG_QUANT_ROW_1x128) {
     const long long strips = static_cast<long long>(batch) * rows * (cols / 128);
+    if (strips >= 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
     const int grid = static_cast<int>(std::min<long long>((strips + 31) / 32, 8ll * sms));
-    if (bf) dg::quant_row_kernel<true><<<grid, 256, 0, st>>>(x, batch, rows, cols, q, scales, ld_scales);
-    else dg::quant_row_kernel<false><<<grid, 256, 0, st>>>(x, batch, rows, cols, q, scales, ld_scales);
+    e = bf ? launch(dg::quant_row_kernel<true>, dim3(grid), dim3(256), 0, st, 1, x, batch, rows,
+                    cols, q, scales, ld_scales)
+           : launch(dg::quant_row_kernel<false>, dim3(grid), dim3(256), 0, st, 1, x, batch, rows,
+                    cols, q, scales, ld_scales);
   } else if (mode == DG_QUANT_BLOCK_128x128) {
     const long long blocks = static_cast<long long>(batch) * ((rows + 127) / 128) * (cols / 128);
     if (blocks > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
-    if (bf) dg::quant_block_kernel<true><<<static_cast<int>(blocks), 256, 0, st>>>(x, batch, rows, cols, q, scales);
-    else dg::quant_block_kernel<false><<<static_cast<int>(blocks), 256, 0, st>>>(x, batch, rows, cols, q, scales);
+    e = bf ? launch(dg::quant_block_kernel<true>, dim3(static_cast<int>(blocks)), dim3(256), 0, st,
+                    1, x, batch, rows, cols, q, scales)
+           : launch(dg::quant_block_kernel<false>, dim3(static_cast<int>(blocks)), dim3(256), 0, st,
+                    1, x, batch, rows, cols, q, scales);
   } else {
     const long long blocks = static_cast<long long>(batch) * (rows / 128) * ((cols + 63) / 64);
     if (blocks > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
-    if (bf) dg::quant_col_kernel<true><<<static_cast<int>(blocks), 256, 0, st>>>(x, batch, rows, cols, q, scales);
-    else dg::quant_col_kernel<false><<<static_cast<int>(blocks), 256, 0, st>>>(x, batch, rows, cols, q, scales);
+    e = bf ? launch(dg::quant_col_kernel<true>, dim3(static_cast<int>(blocks)), dim3(256), 0, st, 1,
+                    x, batch, rows, cols, q, scales)
+           : launch(dg::quant_col_kernel<false>, dim3(static_cast<int>(blocks)), dim3(256), 0, st, 1,
+                    x, batch, rows, cols, q, scales);
   }
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   g_launches.fetch_add(1);
   return DG_OK;

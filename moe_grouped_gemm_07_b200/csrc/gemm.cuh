@@ -274,6 +274,13 @@ __global__ void __launch_bounds__(320, 1)
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // inputs may come from the previous launch on the stream: wait for it
+  // (everything above touched only shared memory, TMEM and kernel params)
+  pdl_wait();
   int total_tiles = args.total_tiles;
   if constexpr (MODE == MODE_MASKED) {
     if (warp == 2) {
@@ -297,11 +304,10 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) prefix[0] = 0;
     }
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  if constexpr (MODE == MODE_MASKED) total_tiles = prefix[args.G];
+  if constexpr (MODE == MODE_MASKED) {
+    __syncthreads();
+    total_tiles = prefix[args.G];
+  }
 
   // ---------------------------------------------------------------- roles
   if (warp == 0) {
@@ -647,6 +653,7 @@ __global__ void __launch_bounds__(320, 1)
   }
 
   // ---------------------------------------------------------------- teardown
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -14,13 +14,15 @@
 //     n_tiles x splits CTAs keep HBM busy even when N/128 is small;
 //   * the partial tiles are reduced through distributed shared memory: each
 //     CTA writes its FP32 partial to its own shared memory, the cluster
-//     synchronises, and CTA r sums rows [r*128/splits, (r+1)*128/splits) of
-//     all partials in rank order (deterministic), adds C and stores BF16.
+//     synchronises, and CTA r sums its slice of 8-row units (the 16 units of
+//     the tile spread over the splits) of all partials in rank order
+//     (deterministic), adds C and stores BF16.
 //
 // Roles per CTA (320 threads): warp 0 TMA producer, warp 1 TMEM allocator and
 // single-thread tcgen05.mma issuer, warps 2..9 promotion (TMEM lane quadrant
 // w % 4, column half (w - 2) / 4). All waits are bounded (see ptx.cuh); both
-// cluster barriers are reached unconditionally, also after a timeout.
+// cluster barriers are reached unconditionally, also after a timeout. With a
+// single split the launch has no cluster and a CTA barrier replaces them.
 #pragma once
 
 #include <cstdint>
@@ -66,7 +68,11 @@ struct DecodeCfg {
   static constexpr int NUM_BARS = 2 * STAGES + 4 + 2 * SS + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static constexpr int RED_BYTES = BNP * 128 * 4;  // partial tile, overlays the ring
+  // partial tile [BNP][RED_PITCH] floats, overlaying the ring; the pitch is
+  // padded from 128 so that the column slices the reduction reads fall into
+  // distinct shared-memory banks for consecutive tokens
+  static constexpr int RED_PITCH = 132;
+  static constexpr int RED_BYTES = BNP * RED_PITCH * 4;
   static_assert(RED_BYTES <= STAGES * (W_BYTES + X_BYTES), "reduction buffer fits the ring");
   static_assert(BNP == 16 || BNP == 32 || BNP == 64 || BNP == 128, "BNP");
   static_assert(OFF_SCALE % 1024 == 0 && (SLOT_FLOATS * 4) % 128 == 0, "TMA smem alignment");
@@ -91,7 +97,7 @@ __global__ void __launch_bounds__(320, 2)
   uint8_t* sW = smem + Cfg::OFF_W;
   uint8_t* sX = smem + Cfg::OFF_X;
   float* sScale = reinterpret_cast<float*>(smem + Cfg::OFF_SCALE);
-  float* red = reinterpret_cast<float*>(smem);  // [BNP][128] partial, after the main loop
+  float* red = reinterpret_cast<float*>(smem);  // [BNP][RED_PITCH] partial, after the main loop
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
@@ -144,6 +150,7 @@ __global__ void __launch_bounds__(320, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // inputs may come from the previous launch on the stream
 
   float acc[EC];
 #pragma unroll
@@ -273,39 +280,69 @@ __global__ void __launch_bounds__(320, 2)
   if (warp >= 2) {
     const int n_local = static_cast<int>(q * 32 + lane);
 #pragma unroll
-    for (int j = 0; j < EC; ++j) red[(h * EC + j) * 128 + n_local] = acc[j];
+    for (int j = 0; j < EC; ++j) red[(h * EC + j) * Cfg::RED_PITCH + n_local] = acc[j];
   }
-  cluster_sync_all();
+  pdl_trigger();
+  if (splits > 1) cluster_sync_all(); else __syncthreads();
   {
-    const int rows = 128 / splits;            // n rows this CTA reduces
-    const int chunks = rows / 4;              // float4 chunks per token column
-    const int n_lo = static_cast<int>(rank) * rows;
+    // CTA `rank` owns rows [8 lo, 8 hi) of the 128-row tile, lo/hi spreading
+    // the 16 eight-row units over the splits; item = (token m, unit u).
+    const int lo = (static_cast<int>(rank) * 16) / splits;
+    const int hi = ((static_cast<int>(rank) + 1) * 16) / splits;
+    const int units = hi - lo;
+    const int items = BNP * units;
     const uint32_t red_base = smem_addr(red);
-    const int items = BNP * chunks;
     for (int itm = threadIdx.x; itm < items; itm += blockDim.x) {
-      const int m = itm / chunks;
-      const int n = n_lo + (itm - m * chunks) * 4;
+      const int m = static_cast<int>(static_cast<uint32_t>(itm) / static_cast<uint32_t>(units));
+      const int u = itm - m * units;
+      const int n = (lo + u) * 8;
       const int gn = n0 + n;
       if (m >= args.M || gn >= args.N) continue;
-      const uint32_t off = red_base + static_cast<uint32_t>((m * 128 + n) * 4);
-      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int r = 0; r < splits; ++r) {  // fixed rank order: deterministic
-        const float4 v = ld_dsmem_f32x4(dsmem_addr(off, static_cast<uint32_t>(r)));
-        sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+      const uint32_t off = red_base + static_cast<uint32_t>((m * Cfg::RED_PITCH + n) * 4);
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (splits == 1) {
+        const float4 a = *reinterpret_cast<const float4*>(red + m * Cfg::RED_PITCH + n);
+        const float4 b = *reinterpret_cast<const float4*>(red + m * Cfg::RED_PITCH + n + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+      } else {
+        // partials of 4 ranks in flight at a time, summed in rank order
+        for (int r0 = 0; r0 < splits; r0 += 4) {
+          float4 pa[4], pb[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (r0 + j < splits) {
+              const uint32_t a = dsmem_addr(off, static_cast<uint32_t>(r0 + j));
+              pa[j] = ld_dsmem_f32x4(a);
+              pb[j] = ld_dsmem_f32x4(a + 16);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (r0 + j < splits) {
+              v[0] += pa[j].x; v[1] += pa[j].y; v[2] += pa[j].z; v[3] += pa[j].w;
+              v[4] += pb[j].x; v[5] += pb[j].y; v[6] += pb[j].z; v[7] += pb[j].w;
+            }
+          }
+        }
       }
       const long long o = static_cast<long long>(m) * args.N + gn;
       if (args.C) {
-        const uint2 c2 = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(args.C) + o);
-        sum.x += bf16_lo(c2.x); sum.y += bf16_hi(c2.x);
-        sum.z += bf16_lo(c2.y); sum.w += bf16_hi(c2.y);
+        const uint4 c4 = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(args.C) + o);
+        v[0] += bf16_lo(c4.x); v[1] += bf16_hi(c4.x);
+        v[2] += bf16_lo(c4.y); v[3] += bf16_hi(c4.y);
+        v[4] += bf16_lo(c4.z); v[5] += bf16_hi(c4.z);
+        v[6] += bf16_lo(c4.w); v[7] += bf16_hi(c4.w);
       }
-      uint2 out;
-      out.x = pack_bf16x2(sum.x, sum.y);
-      out.y = pack_bf16x2(sum.z, sum.w);
-      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(args.D) + o) = out;
+      uint4 out;
+      out.x = pack_bf16x2(v[0], v[1]);
+      out.y = pack_bf16x2(v[2], v[3]);
+      out.z = pack_bf16x2(v[4], v[5]);
+      out.w = pack_bf16x2(v[6], v[7]);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.D) + o) = out;
     }
   }
-  cluster_sync_all();  // no CTA leaves while others still read its partial
+  if (splits > 1) cluster_sync_all();  // no CTA leaves while others still read its partial
 
   if (warp == 1) {
     tc_fence_after();

@@ -37,6 +37,17 @@ __device__ __forceinline__ uint32_t warp_id_uniform() {
   return __shfl_sync(0xffffffffu, threadIdx.x >> 5, 0);
 }
 
+// ---------------------------------------------------------------- PDL
+// Programmatic dependent launch. Every kernel of this library calls pdl_wait()
+// in every CTA before its first global-memory access, so it never reads data
+// of a still-running predecessor, and the ordering stays transitive along a
+// chain of such launches. pdl_trigger() lets the next launch start its
+// prologue early. Both are no-ops for a launch without the PDL attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)

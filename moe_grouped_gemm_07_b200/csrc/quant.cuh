@@ -15,6 +15,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include "ptx.cuh"
+
 namespace dg {
 
 struct In4 {
@@ -40,10 +42,6 @@ __device__ __forceinline__ In4 load4(const void* x, int64_t i) {
   return r;
 }
 
-__device__ __forceinline__ float scale_from_amax(float amax) {
-  return fmaxf(amax, 1e-4f) / 448.0f;  // IEEE division (no fast-math)
-}
-
 // x / s rounded to nearest (the IEEE quotient), from r = 1/s correctly rounded
 // and one FMA correction step (Markstein, "Computation of elementary functions
 // on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990: if r is
@@ -57,6 +55,13 @@ __device__ __forceinline__ float quotient(float x, float s, float r) {
   const float q0 = __fmul_rn(ax, r);
   const float e = fmaf(-q0, s, ax);
   return copysignf(fmaf(e, r, q0), x);
+}
+
+// max(amax, 1e-4f) / 448 rounded exactly as the IEEE division (same method:
+// the dividend is >= 1e-4, far from underflow).
+__device__ __forceinline__ float scale_from_amax(float amax) {
+  constexpr float kInv448 = 1.0f / 448.0f;  // correctly rounded at compile time
+  return quotient(fmaxf(amax, 1e-4f), 448.0f, kInv448);
 }
 
 // Four E4M3 codes packed little-endian (element 0 in the low byte).
@@ -76,40 +81,46 @@ __device__ __forceinline__ float warp_max(float v) {
 
 // ROW_1x128: strips enumerated (batch, row, strip) with the strip index
 // fastest, so strip s covers elements [128 s, 128 s + 128) of x. Each warp
-// takes 4 consecutive strips per step (2 KB of input in flight per warp).
+// takes 4 consecutive strips per step (2 KB of input in flight per warp); the
+// (row, strip) position of the first one is found with one 32-bit division per
+// step and advanced incrementally. Requires batch * rows * (cols/128) < 2^31.
 template <bool BF16>
 __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__ x, int batch,
                                                         int rows, int cols,
                                                         uint8_t* __restrict__ codes,
                                                         float* __restrict__ scales, int ld) {
   constexpr int U = 4;
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
-  const int kbs = cols >> 7;
-  const int64_t nstrips = static_cast<int64_t>(batch) * rows * kbs;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  for (int64_t s0 = warp0 * U; s0 < nstrips; s0 += nwarps * U) {
+  const uint32_t kbs = static_cast<uint32_t>(cols) >> 7;
+  const uint32_t nstrips = static_cast<uint32_t>(batch) * static_cast<uint32_t>(rows) * kbs;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  const uint32_t warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  for (uint32_t s0 = warp0 * U; s0 < nstrips; s0 += nwarps * U) {
     In4 in[U];
 #pragma unroll
     for (int u = 0; u < U; ++u)
-      if (s0 + u < nstrips) in[u] = load4<BF16>(x, (s0 + u) * 128 + (lane << 2));
+      if (s0 + u < nstrips) in[u] = load4<BF16>(x, (static_cast<int64_t>(s0) + u) * 128 + (lane << 2));
+    uint32_t br = s0 / kbs;            // batch * rows + row of strip s0
+    uint32_t kb = s0 - br * kbs;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t st = s0 + u;
+      const uint32_t st = s0 + u;
       if (st >= nstrips) break;
       float amax = fmaxf(fmaxf(fabsf(in[u].v[0]), fabsf(in[u].v[1])),
                          fmaxf(fabsf(in[u].v[2]), fabsf(in[u].v[3])));
       amax = warp_max(amax);
       const float sc = scale_from_amax(amax);
       const float rc = __frcp_rn(sc);
-      *reinterpret_cast<uint32_t*>(codes + st * 128 + (lane << 2)) = encode4(in[u].v, sc, rc);
+      *reinterpret_cast<uint32_t*>(codes + static_cast<int64_t>(st) * 128 + (lane << 2)) =
+          encode4(in[u].v, sc, rc);
       if (lane == 0) {
-        const int kb = static_cast<int>(st % kbs);
-        const int64_t br = st / kbs;  // batch * rows + row
-        const int64_t b = br / rows;
-        const int r = static_cast<int>(br - b * rows);
-        scales[(b * kbs + kb) * ld + r] = sc;
+        const uint32_t b = br / static_cast<uint32_t>(rows);
+        const uint32_t r = br - b * static_cast<uint32_t>(rows);
+        scales[(static_cast<int64_t>(b) * kbs + kb) * ld + r] = sc;
       }
+      if (++kb == kbs) { kb = 0; ++br; }
     }
   }
 }
@@ -122,6 +133,8 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
                                                           uint8_t* __restrict__ codes,
                                                           float* __restrict__ scales) {
   __shared__ float red[8];
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int kbs = cols >> 7, nbs = (rows + 127) >> 7;
   const int64_t blk = blockIdx.x;
@@ -167,6 +180,8 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const void* __restrict__
   __shared__ float red[16][64];
   __shared__ float sc_s[64];
   __shared__ float rc_s[64];
+  pdl_wait();
+  pdl_trigger();
   const int cg = threadIdx.x & 15, rg = threadIdx.x >> 4;
   const int slabs = (cols + 63) >> 6, rbs = rows >> 7;
   const int64_t blk = blockIdx.x;

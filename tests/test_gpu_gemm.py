@@ -239,3 +239,58 @@ def test_k_grouped_accumulates_in_place():
     oqb, osb = oracle.quantize(w.B, oracle.COL_128x1)
     R = oracle.k_grouped_tn(oqa, osa, oqb, osb, ks, w.C)
     check_close(D.cpu().numpy().astype(np.float64), R, "k-grouped in place")
+
+
+def test_cuda_graph_capture_and_replay():
+    """The calls do no host synchronisation or allocation, so quantise + GEMM
+    (decode path, persistent path, masked) can be captured in a CUDA graph and
+    replayed on new inputs. The first calls (one-time per-device set-up) are
+    made before capture."""
+    Ms, N, K = (64, 256), 512, 1024
+    dense = {M: wl.dense(M, N, K, cfg=79, shape=M) for M in Ms}
+    B = dense[Ms[0]].B
+    qb, sb = dg.dg_quantize_fp8(to_dev(B), dg.DG_QUANT_BLOCK_128x128)
+    bufs = {}
+    for M in Ms:
+        A = to_dev(dense[M].A)
+        qa = torch.empty((M, K), dtype=torch.uint8, device=dev())
+        sa = torch.zeros((K // 128, (M + 3) // 4 * 4), dtype=torch.float32, device=dev())
+        D = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
+        bufs[M] = (A, qa, sa, D)
+    mw = wl.masked(G=3, max_m=128, N=N, K=K, lo=1, hi=128, cfg=79, shape=9)
+    mA, mmm = to_dev(mw.A), to_dev(mw.masked_m)
+    mqa = torch.empty(mw.A.shape, dtype=torch.uint8, device=dev())
+    msa = torch.zeros((3, K // 128, 128), dtype=torch.float32, device=dev())
+    mqb, msb = dg.dg_quantize_fp8(to_dev(mw.B), dg.DG_QUANT_BLOCK_128x128)
+    mD = torch.zeros((3, 128, N), dtype=torch.bfloat16, device=dev())
+
+    def work():
+        for M in Ms:
+            A, qa, sa, D = bufs[M]
+            dg.dg_quantize_fp8(A, dg.DG_QUANT_ROW_1x128, codes=qa, scales=sa)
+            dg.dg_fp8_gemm_nt(qa, sa, qb, sb, None, D)
+        dg.dg_quantize_fp8(mA, dg.DG_QUANT_ROW_1x128, codes=mqa, scales=msa)
+        dg.dg_m_grouped_fp8_gemm_nt_masked(mqa, msa, mqb, msb, mmm, mD)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        work()  # warm-up: one-time set-up happens outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        work()
+    oqb, osb = oracle.quantize(B, oracle.BLOCK_128x128)
+    for rep in range(2):
+        new = {M: synth.normal((M, K), synth.seed(79, 50 + rep, M)) for M in Ms}
+        for M in Ms:
+            bufs[M][0].copy_(to_dev(new[M]))
+        g.replay()
+        torch.cuda.synchronize()
+        for M in Ms:
+            oqa, osa = oracle.quantize(new[M], oracle.ROW_1x128)
+            check_close(as_f64(bufs[M][3]), oracle.gemm_nt(oqa, osa, oqb, osb), f"graph M={M}")
+    oqa, osa = oracle.quantize(mw.A, oracle.ROW_1x128)
+    oqb2, osb2 = oracle.quantize(mw.B, oracle.BLOCK_128x128)
+    check_close(as_f64(mD), oracle.m_grouped_masked(oqa, osa, oqb2, osb2, mw.masked_m), "graph masked")
