@@ -140,7 +140,7 @@ dg_status make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, 
 template <int MODE, int BN>
 dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
                       const CUtensorMap& tsb, const CUtensorMap& td, const GemmArgs& args,
-                      int grid, cudaStream_t st, int dev) {
+                      int grid, cudaStream_t st, int dev, int cluster = 1) {
   using Cfg = dg::GemmCfg<MODE, BN>;
   static std::once_flag once[kMaxDevices];
   static cudaError_t attr_err[kMaxDevices];
@@ -150,8 +150,8 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
   });
   if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
-  cudaError_t e = launch(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, 1, ta, tb, tsa,
-                         tsb, td, args);
+  cudaError_t e = launch(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, cluster, ta,
+                         tb, tsa, tsb, td, args);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   g_launches.fetch_add(1);
   return DG_OK;
@@ -256,6 +256,75 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
                  M_logical, N, K, G, bn, tiles, grid);
   if (bn == 256) return launch_gemm<MODE, 256>(ta, tb, dummy, dummy, td, args, grid, st, dev);
   return launch_gemm<MODE, 128>(ta, tb, dummy, dummy, td, args, grid, st, dev);
+}
+
+// ---------------------------------------------------------------- CTA pairs
+// Dense GEMM with M > 128 on CTA pairs (256 x BN tiles, cta_group::2 MMAs;
+// each CTA loads half of the B tile). Opt-in with DG_PAIR=1: measured on B200
+// it runs at the speed of the single-CTA kernel (the per-SM operand bytes
+// halve for B, but the shared L2-to-SM path stays the limit), so the
+// single-CTA kernel remains the default.
+bool use_pairs() {
+  static const bool on = [] {
+    const char* e = std::getenv("DG_PAIR");
+    return e && e[0] == '1';
+  }();
+  return on;
+}
+
+// Columns of a pair tile: 256, or 128 with DG_PAIR_BN=128.
+int pair_bn() {
+  static const int bn = [] {
+    const char* e = std::getenv("DG_PAIR_BN");
+    return (e && std::atoi(e) == 128) ? 128 : 256;
+  }();
+  return bn;
+}
+
+dg_status run_pair(const void* A, const float* sfa, int ld_sfa, const void* B, const float* sfb,
+                   const void* C, void* D, int M, int N, int K, cudaStream_t st) {
+  int dev = 0, sms = 0;
+  dg_status s = device_sms(&dev, &sms);
+  if (s != DG_OK) return s;
+  CUtensorMap ta, tb, td, dummy;
+  std::memset(&dummy, 0, sizeof dummy);
+  if ((s = make_map_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  // pair tiles are 256 x bn; each CTA of a pair loads half (bn/2 rows) of B
+  const int bn = pair_bn();
+  if ((s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, 128, bn / 2,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  if ((s = make_map_2d(&td, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, 2ull * N, 32, 32,
+                       CU_TENSOR_MAP_SWIZZLE_64B)) != DG_OK)
+    return s;
+  GemmArgs args;
+  std::memset(&args, 0, sizeof args);
+  args.M = M;
+  args.N = N;
+  args.K = K;
+  args.G = 1;
+  args.num_m_blocks = (M + 255) / 256;
+  args.num_n_blocks = (N + bn - 1) / bn;
+  const long long tiles = static_cast<long long>(args.num_m_blocks) * args.num_n_blocks;
+  args.total_tiles = static_cast<int>(tiles);
+  args.sfa = sfa;
+  args.ld_sfa = ld_sfa;
+  args.sfb = sfb;
+  args.C = C;
+  args.D = D;
+  args.d_rows = M;
+  args.timeout_ns = timeout_ns();
+  args.drop_arrive = take_drop_flag();
+  const int pairs = static_cast<int>(std::max<long long>(1, std::min<long long>(sms / 2, tiles)));
+  if (print_configs())
+    std::fprintf(stderr,
+                 "[dg] fp8_gemm_nt pairs M=%d N=%d K=%d: 256x%d tiles=%lld on %d CTA pairs\n", M,
+                 N, K, bn, tiles, pairs);
+  if (bn == 256)
+    return launch_gemm<dg::MODE_PAIR, 256>(ta, tb, dummy, dummy, td, args, 2 * pairs, st, dev, 2);
+  return launch_gemm<dg::MODE_PAIR, 128>(ta, tb, dummy, dummy, td, args, 2 * pairs, st, dev, 2);
 }
 
 // ---------------------------------------------------------------- decode path
@@ -502,6 +571,7 @@ dg_status dg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const f
     if (s != DG_OK) return s;
     return dispatch_decode(A, sfa, B, sfb, C, D, M, N, K, sms, dev, st);
   }
+  if (use_pairs()) return run_pair(A, sfa, ld, B, sfb, C, D, M, N, K, st);
   return run_nt<dg::MODE_DENSE>(A, sfa, ld, B, sfb, nullptr, nullptr, C, D, M, M, N, K, 1, mb, mb,
                                 st, "fp8_gemm_nt");
 }

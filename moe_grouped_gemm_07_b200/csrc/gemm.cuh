@@ -30,7 +30,13 @@
 
 namespace dg {
 
-enum GemmMode : int { MODE_DENSE = 0, MODE_CONTIG = 1, MODE_MASKED = 2, MODE_KGROUPED = 3 };
+// MODE_PAIR is the dense GEMM on CTA pairs: a 2-CTA cluster computes a
+// 256 x BN tile with tcgen05 cta_group::2 MMAs (each CTA holds 128 rows of A,
+// half of the B tile and the accumulator of its 128 rows): the same operand
+// traffic per SM as a 128 x 2BN single-CTA tile with half the accumulator.
+enum GemmMode : int {
+  MODE_DENSE = 0, MODE_CONTIG = 1, MODE_MASKED = 2, MODE_KGROUPED = 3, MODE_PAIR = 4
+};
 
 constexpr int kMaxKGroups = 256;
 constexpr int kMaxMaskedGroups = 1024;
@@ -58,10 +64,12 @@ struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
   static constexpr int BK = 128;  // FP8 elements (= bytes) per K-block
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr bool PAIR = MODE == MODE_PAIR;
+  // ring depth from the stage size (A + this CTA's B): 48 KB -> 4, 32 KB -> 6, 24 KB -> 8
+  static constexpr int STAGES = PAIR ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6);
   static constexpr int SCALE_SLOTS = 8;  // K-grouped only
   static constexpr int A_BYTES = BM * BK;
-  static constexpr int B_BYTES = BN * BK;
+  static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * BK;  // this CTA's part of the B tile
   static constexpr int SCALE_BYTES = (BM + BN) * 4;
   static constexpr int THREADS = 320;
   static constexpr int NACC = 512 / BN;  // TMEM accumulator buffers (all 512 columns)
@@ -115,13 +123,29 @@ struct Tile {
 // roles walk the same tile sequence.
 template <int MODE, int BN>
 __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int* prefix,
-                                            const int* mm_clamped) {
+                                            const int* mm_clamped, int rank = 0) {
   using Cfg = GemmCfg<MODE, BN>;
   Tile tl;
   tl.valid = 1;
   tl.kb0 = 0;
   tl.nkb = a.K / Cfg::BK;
-  if constexpr (MODE == MODE_DENSE || MODE == MODE_CONTIG) {
+  if constexpr (MODE == MODE_PAIR) {
+    // pair tile (256 rows x BN): CTA `rank` of the pair owns rows [128 rank, +128)
+    const int group_tiles = Cfg::GROUP_M * a.num_n_blocks;
+    const int grp = t / group_tiles;
+    const int first_m = grp * Cfg::GROUP_M;
+    const int gm = min(a.num_m_blocks - first_m, Cfg::GROUP_M);
+    const int local = t - grp * group_tiles;
+    const int mb = first_m + local % gm;
+    const int nb = local / gm;
+    tl.g = 0;
+    tl.m0 = mb * 256 + rank * 128;
+    tl.n0 = nb * BN;
+    tl.a_row = tl.m0;
+    tl.b_row = tl.n0 + rank * (BN / 2);
+    tl.rows = min(Cfg::BM, a.M - tl.m0);  // may be <= 0 for the second CTA
+    tl.out_row0 = tl.m0;
+  } else if constexpr (MODE == MODE_DENSE || MODE == MODE_CONTIG) {
     const int group_tiles = Cfg::GROUP_M * a.num_n_blocks;
     const int grp = t / group_tiles;
     const int first_m = grp * Cfg::GROUP_M;
@@ -243,6 +267,11 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t warp = warp_id_uniform();
   const uint32_t lane = lane_id();
   const uint64_t tmo = args.timeout_ns;
+  constexpr bool PAIR = Cfg::PAIR;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = leader of the pair
+  const bool leader = rank == 0;
+  const int cta_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int cta_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
@@ -252,7 +281,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int i = 0; i < NA; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 8);
+      mbar_init(&tempty[i], PAIR ? 16 : 8);  // pair: promotion warps of both CTAs
     }
     for (int i = 0; i < SS; ++i) {
       mbar_init(&sfull[i], 1);
@@ -271,11 +300,19 @@ __global__ void __launch_bounds__(320, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // inputs may come from the previous launch on the stream: wait for it
@@ -315,8 +352,8 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       uint32_t it = 0, sit = 0;
       int dropped = -1;
-      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-        const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped);
+      for (int t = cta_first; t < total_tiles; t += cta_step) {
+        const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped, rank);
         if (!tl.valid) continue;
         for (int kb = 0; kb < tl.nkb; ++kb, ++it) {
           const uint32_t s = it % S;
@@ -332,6 +369,13 @@ __global__ void __launch_bounds__(320, 1)
           }
           if (args.drop_arrive && it == 0) {  // test hook: never arm stage 0
             dropped = 0;
+          } else if constexpr (PAIR) {
+            // the leader's barrier counts the bytes of both CTAs' loads
+            if (leader) mbar_arrive_expect_tx(&full[s], 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
+            const uint32_t fb = dsmem_addr(smem_addr(&full[s]), 0);
+            const int kk = kb * Cfg::BK;
+            tma_load_2d_pair(sA + s * Cfg::A_BYTES, &tm_a, fb, kk, tl.a_row);
+            tma_load_2d_pair(sB + s * Cfg::B_BYTES, &tm_b, fb, kk, tl.b_row);
           } else {
             mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES);
             const int kk = (tl.kb0 + kb) * Cfg::BK;
@@ -359,7 +403,9 @@ __global__ void __launch_bounds__(320, 1)
     producer_done:
       // Wait (bounded, regardless of abort) for every copy still in flight:
       // the last min(it, S) stages and min(sit, SS) scale slots.
-      for (uint32_t j = (it > S ? it - S : 0); j < it; ++j) {
+      // (pair: the leader's barriers count both CTAs' copies; the follower
+      // leaves only after the leader, at the closing cluster barrier)
+      for (uint32_t j = (it > S ? it - S : 0); j < it && leader; ++j) {
         if (static_cast<int>(j) == dropped) continue;
         volatile int never = 0;
         mbar_wait(&full[j % S], (j / S) & 1, &never, tmo, SITE_TEARDOWN_TMA);
@@ -374,11 +420,12 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ======================= MMA issuer (one thread) ========================
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(Cfg::BM, BN, Cfg::KG ? 1 : 0, Cfg::KG ? 1 : 0);
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc =
+          idesc_e4m3_f32(PAIR ? 2 * Cfg::BM : Cfg::BM, BN, Cfg::KG ? 1 : 0, Cfg::KG ? 1 : 0);
       uint32_t it = 0, acc_it = 0;
-      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-        const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped);
+      for (int t = cta_first; t < total_tiles; t += cta_step) {
+        const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped, rank);
         if (!tl.valid) continue;
         for (int kb = 0; kb < tl.nkb; ++kb, ++it, ++acc_it) {
           const uint32_t b = acc_it % NA;
@@ -404,14 +451,25 @@ __global__ void __launch_bounds__(320, 1)
               da = smem_desc_sw128(a_base + k * 32, 16, 1024);
               db = smem_desc_sw128(b_base + k * 32, 16, 1024);
             }
-            mma_f8f6f4(d_tmem, da, db, idesc, k > 0 ? 1u : 0u);
+            if constexpr (PAIR)
+              mma_f8f6f4_pair(d_tmem, da, db, idesc, k > 0 ? 1u : 0u);
+            else
+              mma_f8f6f4(d_tmem, da, db, idesc, k > 0 ? 1u : 0u);
           }
-          mma_commit(&empty[s]);
-          mma_commit(&tfull[b]);
+          if constexpr (PAIR) {
+            mma_commit_pair_mc(&empty[s], 0x3);  // frees the stage in both CTAs
+            mma_commit_pair_mc(&tfull[b], 0x3);  // both accumulators are ready
+          } else {
+            mma_commit(&empty[s]);
+            mma_commit(&tfull[b]);
+          }
         }
       }
     mma_done_label:
-      mma_commit(mma_done);
+      if constexpr (PAIR)
+        mma_commit_pair_mc(mma_done, 0x1);
+      else
+        mma_commit(mma_done);
       {
         volatile int never = 0;
         mbar_wait(mma_done, 0, &never, tmo, SITE_TEARDOWN_MMA);
@@ -427,8 +485,8 @@ __global__ void __launch_bounds__(320, 1)
     uint32_t acc_it = 0, sit = 0;
     const int KBn = args.K / Cfg::BK;  // NT: K-blocks per row of sfb
     const int nbN = (args.N + 127) / 128;
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-      const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped);
+    for (int t = cta_first; t < total_tiles; t += cta_step) {
+      const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped, rank);
       if (!tl.valid) continue;
       float acc[EC];
 #pragma unroll
@@ -484,20 +542,43 @@ __global__ void __launch_bounds__(320, 1)
           const float sc = (row_in ? slot[lane] : 0.f) * (half_in ? slot[32] : 0.f);
           __syncwarp();
           issue_scales(kb + SR);
-#pragma unroll
-          for (int c = 0; c < EC / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
-            tmem_ld_wait();
-            if (c == EC / 32 - 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&tempty[b]);
+          auto release_tmem = [&]() {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              if constexpr (PAIR)
+                mbar_arrive_cluster(dsmem_addr(smem_addr(&tempty[b]), 0));
+              else
+                mbar_arrive(&tempty[b]);
             }
+          };
+          if constexpr (EC <= 64) {
+            // all chunks of this thread's columns in flight, one wait
+            uint32_t r[EC / 32][32];
 #pragma unroll
-            for (int i = 0; i < 32; i += 2)
-              fma2(acc[c * 32 + i], acc[c * 32 + i + 1], sc, sc, __uint_as_float(r[i]),
-                   __uint_as_float(r[i + 1]));
+            for (int c = 0; c < EC / 32; ++c)
+              tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r[c]);
+            tmem_ld_wait();
+            release_tmem();
+#pragma unroll
+            for (int c = 0; c < EC / 32; ++c)
+#pragma unroll
+              for (int i = 0; i < 32; i += 2)
+                fma2(acc[c * 32 + i], acc[c * 32 + i + 1], sc, sc, __uint_as_float(r[c][i]),
+                     __uint_as_float(r[c][i + 1]));
+          } else {
+            // 128 accumulator registers leave room for one chunk at a time
+#pragma unroll
+            for (int c = 0; c < EC / 32; ++c) {
+              uint32_t r[32];
+              tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
+              tmem_ld_wait();
+              if (c == EC / 32 - 1) release_tmem();
+#pragma unroll
+              for (int i = 0; i < 32; i += 2)
+                fma2(acc[c * 32 + i], acc[c * 32 + i + 1], sc, sc, __uint_as_float(r[i]),
+                     __uint_as_float(r[i + 1]));
+            }
           }
         } else {
           const uint32_t ss = sit % SS;
@@ -551,7 +632,9 @@ __global__ void __launch_bounds__(320, 1)
         const bool clipped = orow >= args.d_rows;
         const int col0 = tl.n0 + static_cast<int>(h) * EC;
         const bool use_tma = __all_sync(0xffffffffu, write || clipped);
-        if (use_tma) {
+        if (tl.rows <= 0) {
+          // pair: this CTA's half of the tile lies entirely past M
+        } else if (use_tma) {
           constexpr int CW = Cfg::STORE_COLS;
           uint8_t* stg = sStage + (warp - 2) * Cfg::STAGE_BYTES_PER_WARP;
           const int swz = static_cast<int>((lane >> 1) & 3);  // 64-byte swizzle of row `lane`
@@ -655,10 +738,16 @@ __global__ void __launch_bounds__(320, 1)
   // ---------------------------------------------------------------- teardown
   pdl_trigger();
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();  // the leader's MMAs into both CTAs' TMEM are done
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
 }
 
