@@ -11,8 +11,10 @@
 //
 // CTA = 320 threads, one CTA per SM, persistent over output tiles:
 //   warp 0      TMA producer: A/B tiles (128B-swizzled) into an S-stage ring
-//               (plus, for K-grouped, the per-K-block scale vectors).
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer: for each
+//               (plus, for K-grouped, the per-K-block scale vectors); the
+//               warp runs the loop, lane 0 issues.
+//   warp 1      TMEM allocator + tcgen05.mma issuer (lane 0 of the converged
+//               warp): for each
 //               K-block, 4 x (M=128, N=BN, K=32) MMAs into one of 512/BN TMEM
 //               accumulator buffers (all 512 columns), reset per K-block.
 //   warps 2..9  promotion / epilogue: warp w reads TMEM lane quadrant (w % 4)
@@ -348,8 +350,10 @@ __global__ void __launch_bounds__(320, 1)
 
   // ---------------------------------------------------------------- roles
   if (warp == 0) {
-    // ======================= TMA producer (one thread) =======================
-    if (lane == 0) {
+    // ======================= TMA producer ====================================
+    // The whole warp runs the loop and waits (converged, as in the MMA
+    // issuer); lane 0 arms the barriers and issues the copies.
+    {
       uint32_t it = 0, sit = 0;
       int dropped = -1;
       for (int t = cta_first; t < total_tiles; t += cta_step) {
@@ -357,50 +361,56 @@ __global__ void __launch_bounds__(320, 1)
         if (!tl.valid) continue;
         for (int kb = 0; kb < tl.nkb; ++kb, ++it) {
           const uint32_t s = it % S;
-          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort_flag, tmo, SITE_PRODUCER_EMPTY))
-            goto producer_done;
+          bool ok = mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort_flag, tmo, SITE_PRODUCER_EMPTY);
+          if (!__all_sync(0xffffffffu, ok)) goto producer_done;
           if constexpr (Cfg::KG) {
             // take the scale slot before arming anything, so an abort here
             // leaves no uncounted copy in flight
             const uint32_t ss = sit % SS;
-            if (!mbar_wait(&sempty[ss], ((sit / SS) & 1) ^ 1, abort_flag, tmo,
-                           SITE_PRODUCER_SCALE_EMPTY))
-              goto producer_done;
+            ok = mbar_wait(&sempty[ss], ((sit / SS) & 1) ^ 1, abort_flag, tmo,
+                           SITE_PRODUCER_SCALE_EMPTY);
+            if (!__all_sync(0xffffffffu, ok)) goto producer_done;
           }
           if (args.drop_arrive && it == 0) {  // test hook: never arm stage 0
             dropped = 0;
-          } else if constexpr (PAIR) {
-            // the leader's barrier counts the bytes of both CTAs' loads
-            if (leader) mbar_arrive_expect_tx(&full[s], 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
-            const uint32_t fb = dsmem_addr(smem_addr(&full[s]), 0);
-            const int kk = kb * Cfg::BK;
-            tma_load_2d_pair(sA + s * Cfg::A_BYTES, &tm_a, fb, kk, tl.a_row);
-            tma_load_2d_pair(sB + s * Cfg::B_BYTES, &tm_b, fb, kk, tl.b_row);
-          } else {
-            mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES);
-            const int kk = (tl.kb0 + kb) * Cfg::BK;
-            if constexpr (Cfg::KG) {
-              tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], tl.a_row, kk);
-#pragma unroll
-              for (int h = 0; h < BN / 128; ++h)
-                tma_load_2d(sB + s * Cfg::B_BYTES + h * 128 * Cfg::BK, &tm_b, &full[s],
-                            tl.b_row + h * 128, kk);
+          } else if (lane == 0) {
+            if constexpr (PAIR) {
+              // the leader's barrier counts the bytes of both CTAs' loads
+              if (leader) mbar_arrive_expect_tx(&full[s], 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
+              const uint32_t fb = dsmem_addr(smem_addr(&full[s]), 0);
+              const int kk = kb * Cfg::BK;
+              tma_load_2d_pair(sA + s * Cfg::A_BYTES, &tm_a, fb, kk, tl.a_row);
+              tma_load_2d_pair(sB + s * Cfg::B_BYTES, &tm_b, fb, kk, tl.b_row);
             } else {
-              tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], kk, tl.a_row);
-              tma_load_2d(sB + s * Cfg::B_BYTES, &tm_b, &full[s], kk, tl.b_row);
+              mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES);
+              const int kk = (tl.kb0 + kb) * Cfg::BK;
+              if constexpr (Cfg::KG) {
+                tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], tl.a_row, kk);
+#pragma unroll
+                for (int h = 0; h < BN / 128; ++h)
+                  tma_load_2d(sB + s * Cfg::B_BYTES + h * 128 * Cfg::BK, &tm_b, &full[s],
+                              tl.b_row + h * 128, kk);
+              } else {
+                tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], kk, tl.a_row);
+                tma_load_2d(sB + s * Cfg::B_BYTES, &tm_b, &full[s], kk, tl.b_row);
+              }
             }
           }
           if constexpr (Cfg::KG) {
             const uint32_t ss = sit % SS;
-            mbar_arrive_expect_tx(&sfull[ss], Cfg::SCALE_BYTES);
-            float* slot = sScale + ss * (Cfg::BM + BN);
-            tma_load_2d(slot, &tm_sfa, &sfull[ss], tl.m0, tl.kb0 + kb);
-            tma_load_2d(slot + Cfg::BM, &tm_sfb, &sfull[ss], tl.n0, tl.kb0 + kb);
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&sfull[ss], Cfg::SCALE_BYTES);
+              float* slot = sScale + ss * (Cfg::BM + BN);
+              tma_load_2d(slot, &tm_sfa, &sfull[ss], tl.m0, tl.kb0 + kb);
+              tma_load_2d(slot + Cfg::BM, &tm_sfb, &sfull[ss], tl.n0, tl.kb0 + kb);
+            }
             ++sit;
           }
+          __syncwarp();
         }
       }
     producer_done:
+      __syncwarp();
       // Wait (bounded, regardless of abort) for every copy still in flight:
       // the last min(it, S) stages and min(sit, SS) scale slots.
       // (pair: the leader's barriers count both CTAs' copies; the follower
@@ -419,57 +429,68 @@ __global__ void __launch_bounds__(320, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ======================= MMA issuer (one thread) ========================
-    if (lane == 0 && leader) {
+    // ======================= MMA issuer ======================================
+    // The whole warp runs the loop and waits; lane 0 issues the MMAs and
+    // commits. Keeping the issuing thread converged with its warp matters on
+    // sm_100a: bookkeeping run by a lone diverged thread between MMA groups
+    // measurably stalls the tensor pipe (about 20% per K-block here), the
+    // same work in a converged warp does not.
+    if (leader) {
       constexpr uint32_t idesc =
           idesc_e4m3_f32(PAIR ? 2 * Cfg::BM : Cfg::BM, BN, Cfg::KG ? 1 : 0, Cfg::KG ? 1 : 0);
-      uint32_t it = 0, acc_it = 0;
+      uint32_t s = 0, full_ph = 0, b = 0, tmem_ph = 0;
       for (int t = cta_first; t < total_tiles; t += cta_step) {
         const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped, rank);
         if (!tl.valid) continue;
-        for (int kb = 0; kb < tl.nkb; ++kb, ++it, ++acc_it) {
-          const uint32_t b = acc_it % NA;
-          if (!mbar_wait(&tempty[b], ((acc_it / NA) & 1) ^ 1, abort_flag, tmo, SITE_MMA_TMEM_EMPTY))
-            goto mma_done_label;
+        for (int kb = 0; kb < tl.nkb; ++kb) {
+          bool ok = mbar_wait(&tempty[b], tmem_ph ^ 1, abort_flag, tmo, SITE_MMA_TMEM_EMPTY);
+          if (!__all_sync(0xffffffffu, ok)) goto mma_done_label;
           tc_fence_after();
-          const uint32_t s = it % S;
-          if (!mbar_wait(&full[s], (it / S) & 1, abort_flag, tmo, SITE_MMA_FULL))
-            goto mma_done_label;
+          ok = mbar_wait(&full[s], full_ph, abort_flag, tmo, SITE_MMA_FULL);
+          if (!__all_sync(0xffffffffu, ok)) goto mma_done_label;
           tc_fence_after();
-          const uint32_t a_base = smem_addr(sA + s * Cfg::A_BYTES);
-          const uint32_t b_base = smem_addr(sB + s * Cfg::B_BYTES);
-          const uint32_t d_tmem = tmem_base + b * BN;
+          if (lane == 0) {
+            const uint32_t a_base = smem_addr(sA + s * Cfg::A_BYTES);
+            const uint32_t b_base = smem_addr(sB + s * Cfg::B_BYTES);
+            const uint32_t d_tmem = tmem_base + b * BN;
 #pragma unroll
-          for (int k = 0; k < Cfg::BK / 32; ++k) {
-            uint64_t da, db;
-            if constexpr (Cfg::KG) {
-              // MN-major: 32 K-rows of 128 bytes per MMA; MN atoms 16 KB apart.
-              da = smem_desc_sw128(a_base + k * 32 * 128, 128 * Cfg::BK, 1024);
-              db = smem_desc_sw128(b_base + k * 32 * 128, 128 * Cfg::BK, 1024);
-            } else {
-              // K-major: 32 bytes of K per MMA inside the 128-byte swizzle row.
-              da = smem_desc_sw128(a_base + k * 32, 16, 1024);
-              db = smem_desc_sw128(b_base + k * 32, 16, 1024);
+            for (int k = 0; k < Cfg::BK / 32; ++k) {
+              uint64_t da, db;
+              if constexpr (Cfg::KG) {
+                // MN-major: 32 K-rows of 128 bytes per MMA; MN atoms 16 KB apart.
+                da = smem_desc_sw128(a_base + k * 32 * 128, 128 * Cfg::BK, 1024);
+                db = smem_desc_sw128(b_base + k * 32 * 128, 128 * Cfg::BK, 1024);
+              } else {
+                // K-major: 32 bytes of K per MMA inside the 128-byte swizzle row.
+                da = smem_desc_sw128(a_base + k * 32, 16, 1024);
+                db = smem_desc_sw128(b_base + k * 32, 16, 1024);
+              }
+              if constexpr (PAIR)
+                mma_f8f6f4_pair(d_tmem, da, db, idesc, k > 0 ? 1u : 0u);
+              else
+                mma_f8f6f4(d_tmem, da, db, idesc, k > 0 ? 1u : 0u);
             }
-            if constexpr (PAIR)
-              mma_f8f6f4_pair(d_tmem, da, db, idesc, k > 0 ? 1u : 0u);
-            else
-              mma_f8f6f4(d_tmem, da, db, idesc, k > 0 ? 1u : 0u);
+            if constexpr (PAIR) {
+              mma_commit_pair_mc(&empty[s], 0x3);  // frees the stage in both CTAs
+              mma_commit_pair_mc(&tfull[b], 0x3);  // both accumulators are ready
+            } else {
+              mma_commit(&empty[s]);
+              mma_commit(&tfull[b]);
+            }
           }
-          if constexpr (PAIR) {
-            mma_commit_pair_mc(&empty[s], 0x3);  // frees the stage in both CTAs
-            mma_commit_pair_mc(&tfull[b], 0x3);  // both accumulators are ready
-          } else {
-            mma_commit(&empty[s]);
-            mma_commit(&tfull[b]);
-          }
+          __syncwarp();
+          if (++s == S) { s = 0; full_ph ^= 1; }
+          if (++b == NA) { b = 0; tmem_ph ^= 1; }
         }
       }
     mma_done_label:
-      if constexpr (PAIR)
-        mma_commit_pair_mc(mma_done, 0x1);
-      else
-        mma_commit(mma_done);
+      if (lane == 0) {
+        if constexpr (PAIR)
+          mma_commit_pair_mc(mma_done, 0x1);
+        else
+          mma_commit(mma_done);
+      }
+      __syncwarp();
       {
         volatile int never = 0;
         mbar_wait(mma_done, 0, &never, tmo, SITE_TEARDOWN_MMA);
