@@ -373,7 +373,8 @@ int max_cluster(int dev) {
 // Split count: double the CTAs per N-tile (up to 8, a cluster size every
 // GPC can co-schedule many times over) while the launch still fits in two
 // CTAs per SM and every CTA keeps at least two K-blocks. Measured: 16-CTA
-// clusters do not all fit at once, and uneven splits lengthen the reduction.
+// clusters do not all fit at once. The result is a power of two <= 8, so it
+// divides the 16 eight-row units of a tile that the reduction hands out.
 int choose_splits(int n_tiles, int KB, int sms, int cap) {
   int splits = 1;
   while (splits * 2 <= (cap < 8 ? cap : 8) &&

@@ -12,17 +12,23 @@
 //   * split-K across a thread-block cluster: the `splits` CTAs of a cluster
 //     share one N-tile and each streams its own slice of K-blocks, so
 //     n_tiles x splits CTAs keep HBM busy even when N/128 is small;
-//   * the partial tiles are reduced through distributed shared memory: each
-//     CTA writes its FP32 partial to its own shared memory, the cluster
-//     synchronises, and CTA r sums its slice of 8-row units (the 16 units of
-//     the tile spread over the splits) of all partials in rank order
-//     (deterministic), adds C and stores BF16.
+//   * the partial tiles are reduced through distributed shared memory: CTA r
+//     owns 16/splits of the tile's sixteen 8-row units; after a cluster
+//     barrier (every ring is free) each CTA pushes, with remote stores, the
+//     rows of its FP32 partial that CTA o owns into o's receive slot for
+//     rank r; after a second barrier each CTA sums its units over the slots in
+//     rank order (deterministic) from its own shared memory, adds C and
+//     stores BF16. Remote stores need no round trip; remote loads, which an
+//     owner pulling the partials would issue, are latency-bound.
 //
 // Roles per CTA (320 threads): warp 0 TMA producer, warp 1 TMEM allocator and
-// single-thread tcgen05.mma issuer, warps 2..9 promotion (TMEM lane quadrant
-// w % 4, column half (w - 2) / 4). All waits are bounded (see ptx.cuh); both
-// cluster barriers are reached unconditionally, also after a timeout. With a
-// single split the launch has no cluster and a CTA barrier replaces them.
+// tcgen05.mma issuer (both run their loops as converged warps, lane 0
+// issuing), warps 2..9 promotion (TMEM lane quadrant w % 4, column half
+// (w - 2) / 4). The MMA runs up to NACC - 1 K-blocks ahead of the promotion
+// (NACC accumulator buffers of BNP columns). All waits are bounded (see
+// ptx.cuh); both cluster barriers are reached unconditionally, also after a
+// timeout. With a single split the launch has no cluster and CTA barriers
+// replace them.
 #pragma once
 
 #include <cstdint>
@@ -60,20 +66,25 @@ struct DecodeCfg {
   static constexpr int SLOT_FLOATS = BNP < 32 ? 32 : BNP;
   static constexpr int EC = BNP / 2;            // accumulator columns per promotion thread
   static constexpr int CH = EC < 16 ? EC : 16;  // columns per tcgen05.ld
-  static constexpr int TMEM_COLS = 2 * BNP < 32 ? 32 : 2 * BNP;
+  // accumulator buffers: a CTA owns half of TMEM (two CTAs per SM)
+  static constexpr int NACC = 256 / BNP > 8 ? 8 : 256 / BNP;
+  static constexpr int TMEM_COLS = NACC * BNP;
   static constexpr int OFF_W = 0;
   static constexpr int OFF_X = OFF_W + STAGES * W_BYTES;
   static constexpr int OFF_SCALE = OFF_X + STAGES * X_BYTES;
   static constexpr int OFF_BAR = OFF_SCALE + SS * SLOT_FLOATS * 4;
-  static constexpr int NUM_BARS = 2 * STAGES + 4 + 2 * SS + 1;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * NACC + 2 * SS + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  // partial tile [BNP][RED_PITCH] floats, overlaying the ring; the pitch is
-  // padded from 128 so that the column slices the reduction reads fall into
-  // distinct shared-memory banks for consecutive tokens
-  static constexpr int RED_PITCH = 132;
-  static constexpr int RED_BYTES = BNP * RED_PITCH * 4;
-  static_assert(RED_BYTES <= STAGES * (W_BYTES + X_BYTES), "reduction buffer fits the ring");
+  // receive slots of the split-K reduction, overlaying the ring:
+  // [src rank][owned unit][row in unit (8)][RECV_PITCH] floats, tokens along
+  // the row; the 16 units x 8 rows of a tile fill 128 rows in total. The pitch
+  // is padded by 4 floats so that consecutive rows start in different banks.
+  static constexpr int RECV_PITCH = BNP + 4;
+  static constexpr int RECV_BYTES = 128 * RECV_PITCH * 4;
+  static_assert(RECV_BYTES <= STAGES * (W_BYTES + X_BYTES), "receive slots fit the ring");
+  static_assert((NACC & (NACC - 1)) == 0 && TMEM_COLS >= 32 && (TMEM_COLS & (TMEM_COLS - 1)) == 0,
+                "TMEM allocation is a power of two >= 32 columns");
   static_assert(BNP == 16 || BNP == 32 || BNP == 64 || BNP == 128, "BNP");
   static_assert(OFF_SCALE % 1024 == 0 && (SLOT_FLOATS * 4) % 128 == 0, "TMA smem alignment");
   static_assert(OFF_X % 1024 == 0 && X_BYTES % 1024 == 0, "SW128 tiles are 1024-byte aligned");
@@ -97,15 +108,16 @@ __global__ void __launch_bounds__(320, 2)
   uint8_t* sW = smem + Cfg::OFF_W;
   uint8_t* sX = smem + Cfg::OFF_X;
   float* sScale = reinterpret_cast<float*>(smem + Cfg::OFF_SCALE);
-  float* red = reinterpret_cast<float*>(smem);  // [BNP][RED_PITCH] partial, after the main loop
+  float* recv = reinterpret_cast<float*>(smem);  // receive slots, after the main loop
+  constexpr int NA = Cfg::NACC;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
   uint64_t* tfull = bars + 2 * S;
-  uint64_t* tempty = bars + 2 * S + 2;
-  uint64_t* sfull = bars + 2 * S + 4;
-  uint64_t* sempty = bars + 2 * S + 4 + SS;
-  uint64_t* mma_done = bars + 2 * S + 4 + 2 * SS;
+  uint64_t* tempty = bars + 2 * S + NA;
+  uint64_t* sfull = bars + 2 * S + 2 * NA;
+  uint64_t* sempty = bars + 2 * S + 2 * NA + SS;
+  uint64_t* mma_done = bars + 2 * S + 2 * NA + 2 * SS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
 
@@ -125,7 +137,7 @@ __global__ void __launch_bounds__(320, 2)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NA; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 8);
     }
@@ -159,51 +171,54 @@ __global__ void __launch_bounds__(320, 2)
   const uint32_t h = (warp - 2) >> 2;
 
   if (warp == 0) {
-    // ======================= TMA producer =======================
-    if (lane == 0) {
-      int it = 0;
-      int dropped = -1;
-      for (; it < nkb; ++it) {
-        const int s = it % S;
-        const int ss = it % SS;
-        if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort_flag, tmo, SITE_PRODUCER_EMPTY)) break;
-        if (!mbar_wait(&sempty[ss], ((it / SS) & 1) ^ 1, abort_flag, tmo,
-                       SITE_PRODUCER_SCALE_EMPTY))
-          break;
-        const int kb = kb_begin + it;
-        if (args.drop_arrive && it == 0) {
-          dropped = 0;  // test hook: never arm stage 0
-        } else {
-          mbar_arrive_expect_tx(&full[s], Cfg::W_BYTES + Cfg::X_BYTES);
-          tma_load_2d(sW + s * Cfg::W_BYTES, &tm_w, &full[s], kb * Cfg::BK, n0);
-          tma_load_2d(sX + s * Cfg::X_BYTES, &tm_x, &full[s], kb * Cfg::BK, 0);
-        }
+    // ======================= TMA producer (converged warp, lane 0 issues) ===
+    int it = 0;
+    int dropped = -1;
+    for (; it < nkb; ++it) {
+      const int s = it % S;
+      const int ss = it % SS;
+      bool ok = mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort_flag, tmo, SITE_PRODUCER_EMPTY);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      ok = mbar_wait(&sempty[ss], ((it / SS) & 1) ^ 1, abort_flag, tmo, SITE_PRODUCER_SCALE_EMPTY);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int kb = kb_begin + it;
+      if (args.drop_arrive && it == 0) {
+        dropped = 0;  // test hook: never arm stage 0
+      } else if (lane == 0) {
+        mbar_arrive_expect_tx(&full[s], Cfg::W_BYTES + Cfg::X_BYTES);
+        tma_load_2d(sW + s * Cfg::W_BYTES, &tm_w, &full[s], kb * Cfg::BK, n0);
+        tma_load_2d(sX + s * Cfg::X_BYTES, &tm_x, &full[s], kb * Cfg::BK, 0);
+      }
+      if (lane == 0) {
         mbar_arrive_expect_tx(&sfull[ss], BNP * 4);
         tma_load_2d(sScale + ss * Cfg::SLOT_FLOATS, &tm_sfa, &sfull[ss], 0, kb);
       }
-      // bounded wait for every copy still in flight
-      for (int j = (it > S ? it - S : 0); j < it; ++j) {
-        if (j == dropped) continue;
-        volatile int never = 0;
-        mbar_wait(&full[j % S], (j / S) & 1, &never, tmo, SITE_TEARDOWN_TMA);
-      }
-      for (int j = (it > SS ? it - SS : 0); j < it; ++j) {
-        volatile int never = 0;
-        mbar_wait(&sfull[j % SS], (j / SS) & 1, &never, tmo, SITE_TEARDOWN_TMA);
-      }
+      __syncwarp();
+    }
+    // bounded wait for every copy still in flight
+    for (int j = (it > S ? it - S : 0); j < it; ++j) {
+      if (j == dropped) continue;
+      volatile int never = 0;
+      mbar_wait(&full[j % S], (j / S) & 1, &never, tmo, SITE_TEARDOWN_TMA);
+    }
+    for (int j = (it > SS ? it - SS : 0); j < it; ++j) {
+      volatile int never = 0;
+      mbar_wait(&sfull[j % SS], (j / SS) & 1, &never, tmo, SITE_TEARDOWN_TMA);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ======================= MMA issuer =======================
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(128, BNP, 0, 0);
-      for (int it = 0; it < nkb; ++it) {
-        const uint32_t b = it & 1;
-        if (!mbar_wait(&tempty[b], ((it >> 1) & 1) ^ 1, abort_flag, tmo, SITE_MMA_TMEM_EMPTY)) break;
-        tc_fence_after();
-        const int s = it % S;
-        if (!mbar_wait(&full[s], (it / S) & 1, abort_flag, tmo, SITE_MMA_FULL)) break;
-        tc_fence_after();
+    // ======================= MMA issuer (converged warp, lane 0 issues) =====
+    constexpr uint32_t idesc = idesc_e4m3_f32(128, BNP, 0, 0);
+    for (int it = 0; it < nkb; ++it) {
+      const uint32_t b = static_cast<uint32_t>(it) % NA;
+      bool ok = mbar_wait(&tempty[b], ((it / NA) & 1) ^ 1, abort_flag, tmo, SITE_MMA_TMEM_EMPTY);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int s = it % S;
+      ok = mbar_wait(&full[s], (it / S) & 1, abort_flag, tmo, SITE_MMA_FULL);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      if (lane == 0) {
         const uint32_t w_base = smem_addr(sW + s * Cfg::W_BYTES);
         const uint32_t x_base = smem_addr(sX + s * Cfg::X_BYTES);
 #pragma unroll
@@ -213,10 +228,12 @@ __global__ void __launch_bounds__(320, 2)
         mma_commit(&empty[s]);
         mma_commit(&tfull[b]);
       }
-      mma_commit(mma_done);
-      volatile int never = 0;
-      mbar_wait(mma_done, 0, &never, tmo, SITE_TEARDOWN_MMA);
+      __syncwarp();
     }
+    if (lane == 0) mma_commit(mma_done);
+    __syncwarp();
+    volatile int never = 0;
+    mbar_wait(mma_done, 0, &never, tmo, SITE_TEARDOWN_MMA);
     __syncwarp();
   } else {
     // ======================= promotion (8 warps) =======================
@@ -232,8 +249,8 @@ __global__ void __launch_bounds__(320, 2)
       for (int u = 0; u < 4; ++u) {
         const int it = it0 + u;
         if (it >= nkb) break;
-        const uint32_t b = it & 1;
-        bool ok = mbar_wait(&tfull[b], (it >> 1) & 1, abort_flag, tmo, SITE_EPI_TMEM_FULL);
+        const uint32_t b = static_cast<uint32_t>(it) % NA;
+        bool ok = mbar_wait(&tfull[b], (it / NA) & 1, abort_flag, tmo, SITE_EPI_TMEM_FULL);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) goto promo_done;
         const int ss = it % SS;
@@ -274,57 +291,45 @@ __global__ void __launch_bounds__(320, 2)
   }
 
   // ---------------------------------------------------------- split-K reduction
-  // Every role is done and every copy / MMA has landed, so the ring is free.
+  // Every role is done and every copy / MMA has landed, so this CTA's ring is
+  // free; the first barrier makes that true for every CTA of the cluster.
   tc_fence_before();
-  __syncthreads();
-  if (warp >= 2) {
-    const int n_local = static_cast<int>(q * 32 + lane);
-#pragma unroll
-    for (int j = 0; j < EC; ++j) red[(h * EC + j) * Cfg::RED_PITCH + n_local] = acc[j];
-  }
   pdl_trigger();
   if (splits > 1) cluster_sync_all(); else __syncthreads();
+  const int U = 16 / splits;  // 8-row units per rank (splits divides 16)
+  if (warp >= 2) {
+    // push: this thread holds row n_local of the tile for tokens [h*EC, h*EC+EC)
+    const int n_local = static_cast<int>(q * 32 + lane);
+    const int unit = n_local >> 3;
+    const int owner = unit / U;
+    const int slot_row = ((static_cast<int>(rank) * U + (unit - owner * U)) << 3) + (n_local & 7);
+    float* dst = recv + slot_row * Cfg::RECV_PITCH + h * EC;
+    if (splits == 1) {
+#pragma unroll
+      for (int j = 0; j < EC; j += 4)
+        *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+    } else {
+      const uint32_t remote = dsmem_addr(smem_addr(dst), static_cast<uint32_t>(owner));
+#pragma unroll
+      for (int j = 0; j < EC; j += 4)
+        st_dsmem_f32x4(remote + j * 4, acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+    }
+  }
+  if (splits > 1) cluster_sync_all(); else __syncthreads();
   {
-    // CTA `rank` owns rows [8 lo, 8 hi) of the 128-row tile, lo/hi spreading
-    // the 16 eight-row units over the splits; item = (token m, unit u).
-    const int lo = (static_cast<int>(rank) * 16) / splits;
-    const int hi = ((static_cast<int>(rank) + 1) * 16) / splits;
-    const int units = hi - lo;
-    const int items = BNP * units;
-    const uint32_t red_base = smem_addr(red);
+    // CTA `rank` owns units [rank*U, rank*U + U); item = (unit uu, token m),
+    // token fastest so that a warp reads consecutive floats of a slot row
+    const int items = BNP * U;
     for (int itm = threadIdx.x; itm < items; itm += blockDim.x) {
-      const int m = static_cast<int>(static_cast<uint32_t>(itm) / static_cast<uint32_t>(units));
-      const int u = itm - m * units;
-      const int n = (lo + u) * 8;
-      const int gn = n0 + n;
+      const int uu = itm / BNP;
+      const int m = itm - uu * BNP;
+      const int gn = n0 + ((static_cast<int>(rank) * U + uu) << 3);
       if (m >= args.M || gn >= args.N) continue;
-      const uint32_t off = red_base + static_cast<uint32_t>((m * Cfg::RED_PITCH + n) * 4);
       float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (splits == 1) {
-        const float4 a = *reinterpret_cast<const float4*>(red + m * Cfg::RED_PITCH + n);
-        const float4 b = *reinterpret_cast<const float4*>(red + m * Cfg::RED_PITCH + n + 4);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-      } else {
-        // partials of 4 ranks in flight at a time, summed in rank order
-        for (int r0 = 0; r0 < splits; r0 += 4) {
-          float4 pa[4], pb[4];
+      for (int src = 0; src < splits; ++src) {  // rank order: deterministic
+        const float* p = recv + ((src * U + uu) << 3) * Cfg::RECV_PITCH + m;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (r0 + j < splits) {
-              const uint32_t a = dsmem_addr(off, static_cast<uint32_t>(r0 + j));
-              pa[j] = ld_dsmem_f32x4(a);
-              pb[j] = ld_dsmem_f32x4(a + 16);
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (r0 + j < splits) {
-              v[0] += pa[j].x; v[1] += pa[j].y; v[2] += pa[j].z; v[3] += pa[j].w;
-              v[4] += pb[j].x; v[5] += pb[j].y; v[6] += pb[j].z; v[7] += pb[j].w;
-            }
-          }
-        }
+        for (int r8 = 0; r8 < 8; ++r8) v[r8] += p[r8 * Cfg::RECV_PITCH];
       }
       const long long o = static_cast<long long>(m) * args.N + gn;
       if (args.C) {
@@ -342,7 +347,7 @@ __global__ void __launch_bounds__(320, 2)
       *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.D) + o) = out;
     }
   }
-  if (splits > 1) cluster_sync_all();  // no CTA leaves while others still read its partial
+  // no peer touches this CTA's shared memory after the second barrier
 
   if (warp == 1) {
     tc_fence_after();

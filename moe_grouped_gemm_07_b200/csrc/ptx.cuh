@@ -352,13 +352,13 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t cluster_addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(cluster_addr)
+// Store 16 bytes to shared memory given by its shared::cluster address (local
+// or a peer CTA's). Remote stores need no round trip, unlike remote loads.
+__device__ __forceinline__ void st_dsmem_f32x4(uint32_t cluster_addr, float a, float b, float c,
+                                               float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(a),
+               "f"(b), "f"(c), "f"(d)
                : "memory");
-  return v;
 }
 
 // ---------------------------------------------------------------- descriptors
