@@ -226,6 +226,133 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------- grouped workloads
+def run_grouped(args):
+    """--workload contiguous | masked | kgrouped: the MoE variants at their
+    benchmark sizes (parity cases of the dense sweep's bench line, timed here
+    for the record). One step = quantise the activations on the GPU + the
+    grouped GEMM, inputs resident in HBM and larger than L2 (no flush needed).
+    value = useful TFLOP/s (real rows only); one GPU, rank 0."""
+    import torch
+    import moe_grouped_gemm_07_b200 as dg
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops"]
+    kind = args.workload
+
+    def put(x):
+        return torch.from_numpy(x).to(dev)
+
+    if kind == "contiguous":
+        w = wl.contiguous()
+        A = put(w.A)
+        qb, sb = dg.dg_quantize_fp8(put(w.B), dg.DG_QUANT_BLOCK_128x128)
+        mi = put(w.m_indices)
+        qa = torch.empty(A.shape, dtype=torch.uint8, device=dev)
+        sa = torch.zeros((w.K // 128, (w.Mt + 3) // 4 * 4), dtype=torch.float32, device=dev)
+        D = torch.empty((w.Mt, w.N), dtype=torch.bfloat16, device=dev)
+        flops = 2.0 * w.N * w.K * float(sum(w.rows))
+        algo_bytes = w.Mt * w.K + w.G * w.N * w.K + 2 * w.Mt * w.N
+        bound = "tensor"
+        cfg = {"workload": "m_grouped_contiguous", "G": w.G, "N": w.N, "K": w.K, "Mt": w.Mt,
+               "rows": [int(r) for r in w.rows]}
+
+        def quant():
+            dg.dg_quantize_fp8(A, dg.DG_QUANT_ROW_1x128, codes=qa, scales=sa)
+
+        def gemm():
+            dg.dg_m_grouped_fp8_gemm_nt_contiguous(qa, sa, qb, sb, mi, None, D)
+    elif kind == "masked":
+        NK = wl.MASKED_NK[args.masked_index]
+        w = wl.masked(N=NK[0], K=NK[1], shape=args.masked_index)
+        A = put(w.A)
+        qb, sb = dg.dg_quantize_fp8(put(w.B), dg.DG_QUANT_BLOCK_128x128)
+        mm = put(w.masked_m)
+        qa = torch.empty(A.shape, dtype=torch.uint8, device=dev)
+        sa = torch.zeros((w.G, w.K // 128, (w.max_m + 3) // 4 * 4), dtype=torch.float32, device=dev)
+        D = torch.empty((w.G, w.max_m, w.N), dtype=torch.bfloat16, device=dev)
+        tot = float(np.sum(w.masked_m))
+        flops = 2.0 * w.N * w.K * tot
+        algo_bytes = w.G * w.N * w.K + tot * (w.K + 2 * w.N)
+        bound = "hbm"
+        cfg = {"workload": "m_grouped_masked", "G": w.G, "max_m": w.max_m, "N": w.N, "K": w.K,
+               "sum_masked_m": int(tot)}
+
+        def quant():
+            dg.dg_quantize_fp8(A, dg.DG_QUANT_ROW_1x128, codes=qa, scales=sa)
+
+        def gemm():
+            dg.dg_m_grouped_fp8_gemm_nt_masked(qa, sa, qb, sb, mm, D)
+    else:
+        w = wl.k_grouped()
+        A, B = put(w.A), put(w.B)
+        qa = torch.empty(A.shape, dtype=torch.uint8, device=dev)
+        qb = torch.empty(B.shape, dtype=torch.uint8, device=dev)
+        sa = torch.empty((w.sumK // 128, w.M), dtype=torch.float32, device=dev)
+        sb = torch.empty((w.sumK // 128, w.N), dtype=torch.float32, device=dev)
+        C = put(w.C)
+        D = torch.empty_like(C)
+        flops = 2.0 * w.M * w.N * w.sumK
+        algo_bytes = w.sumK * (w.M + w.N) + 2 * C.numel() * 4
+        bound = "tensor"
+        cfg = {"workload": "k_grouped_tn_contiguous", "G": w.G, "M": w.M, "N": w.N,
+               "ks": [int(k) for k in w.ks]}
+
+        def quant():
+            dg.dg_quantize_fp8(A, dg.DG_QUANT_COL_128x1, codes=qa, scales=sa)
+            dg.dg_quantize_fp8(B, dg.DG_QUANT_COL_128x1, codes=qb, scales=sb)
+
+        def gemm():
+            dg.dg_k_grouped_fp8_gemm_tn_contiguous(qa, sa, qb, sb, w.ks, C, D)
+    torch.cuda.synchronize()
+
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for _ in range(max(args.warmup, 3)):
+        quant()
+        gemm()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    launches0 = dg.dg_get_launch_count()
+    wall0 = time.time()
+    e[0].record()
+    for _ in range(args.steps):
+        quant()
+        gemm()
+    e[1].record()
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    launches = dg.dg_get_launch_count() - launches0
+    clocks = sampler.stop(wall0, wall1)
+    ms_step = e[0].elapsed_time(e[1]) / args.steps
+    # GEMM alone (launch-averaged over the same number of launches)
+    e[0].record()
+    for _ in range(args.steps):
+        gemm()
+    e[1].record()
+    torch.cuda.synchronize()
+    ms_gemm = e[0].elapsed_time(e[1]) / args.steps
+    if bound == "tensor":
+        ach = flops / (ms_gemm * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
+                "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4), "traffic": None}
+    else:
+        ach = algo_bytes / (ms_gemm * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / pk["hbm_gbs"], 4), "traffic": None}
+    line = {"metric": METRIC, "value": round(flops / (ms_step * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": round(ms_step, 4), "gemm_ms": round(ms_gemm, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 x e4m3 -> f32 accumulate", "data": "synthetic (seeded N(0,1))",
+            "config": dict(cfg, l2="inputs larger than L2, no flush"), "roofline": roof,
+            "gpu_launches": int(launches), "clocks": clocks,
+            "algorithmic_bytes_per_launch": int(algo_bytes), "flops_per_step": flops}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -463,11 +590,18 @@ def main():
                     help="M,N,K[;M,N,K...]: time only these shapes (profiling)")
     ap.add_argument("--quick", action="store_true",
                     help="timed device loop only: no e2e leg, CPU baseline or clock sampling")
+    ap.add_argument("--workload", default="dense",
+                    choices=["dense", "contiguous", "masked", "kgrouped"],
+                    help="dense (the bench line) or one MoE variant at its benchmark size")
+    ap.add_argument("--masked-index", type=int, default=0,
+                    help="masked workload: index into the (N, K) pairs")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload != "dense":
+        return run_grouped(args)
     return run_ours(args)
 
 

@@ -331,13 +331,13 @@ dg_status run_pair(const void* A, const float* sfa, int ld_sfa, const void* B, c
 // Largest cluster size (1..16) that the device can co-schedule for this
 // kernel (above 8 only where non-portable cluster sizes are allowed); cached
 // per device and instantiation.
-template <int BNP>
+template <int BNP, int MINB>
 int max_cluster(int dev) {
-  using Cfg = dg::DecodeCfg<BNP>;
+  using Cfg = dg::DecodeCfg<BNP, MINB>;
   static std::once_flag once[kMaxDevices];
   static int best[kMaxDevices];
   std::call_once(once[dev], [&] {
-    auto kern = dg::gemm_decode_kernel<BNP>;
+    auto kern = dg::gemm_decode_kernel<BNP, MINB>;
     best[dev] = 0;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM_BYTES) != cudaSuccess)
@@ -370,29 +370,32 @@ int max_cluster(int dev) {
   return best[dev];
 }
 
-// Split count: double the CTAs per N-tile (up to 8, a cluster size every
-// GPC can co-schedule many times over) while the launch still fits in two
-// CTAs per SM and every CTA keeps at least two K-blocks. Measured: 16-CTA
-// clusters do not all fit at once. The result is a power of two <= 8, so it
-// divides the 16 eight-row units of a tile that the reduction hands out.
-int choose_splits(int n_tiles, int KB, int sms, int cap) {
-  int splits = 1;
-  while (splits * 2 <= (cap < 8 ? cap : 8) &&
-         static_cast<long long>(n_tiles) * splits * 2 <= 2ll * sms && KB / (splits * 2) >= 2)
-    splits *= 2;
-  return splits;
+// Decode plan: CTAs per SM (MINB) and split count. From a sweep of both
+// configurations x 1..8 splits over the decode shapes on B200: more than 4-5
+// splits lose (each CTA keeps too few K-blocks and the reduction grows); with
+// at least one tile per SM a single split on two CTAs per SM is best; M > 64
+// prefers one CTA per SM (all TMEM and registers for the 128-token tile) with
+// at most one CTA per SM in total; M <= 64 prefers two CTAs per SM.
+struct DecodePlan {
+  int minb, splits;
+};
+
+DecodePlan plan_decode(int M, int n_tiles, int KB, int sms, int cap1, int cap2) {
+  auto clampi = [](int v, int lo, int hi) { return std::max(lo, std::min(v, hi)); };
+  if (n_tiles >= sms) return {2, 1};
+  if (M > 64) return {1, clampi(std::min(sms / n_tiles, KB / 2), 1, std::min(5, cap1))};
+  return {2, clampi(std::min(2 * sms / n_tiles, KB / 2), 1, std::min(4, cap2))};
 }
 
-template <int BNP>
+template <int BNP, int MINB>
 dg_status run_decode(const void* A, const float* sfa, const void* B, const float* sfb,
-                     const void* C, void* D, int M, int N, int K, int sms, int dev,
+                     const void* C, void* D, int M, int N, int K, int splits, int sms, int dev,
                      cudaStream_t st) {
-  using Cfg = dg::DecodeCfg<BNP>;
-  const int cap = max_cluster<BNP>(dev);
-  if (cap <= 0) return DG_ERR_CUDA;
+  using Cfg = dg::DecodeCfg<BNP, MINB>;
   const int KB = K / 128;
   const int n_tiles = (N + 127) / 128;
-  const int splits = choose_splits(n_tiles, KB, sms, cap);
+  (void)sms;
+  (void)dev;
   const int ld = (M + 3) / 4 * 4;
   CUtensorMap tw, tx, tsa;
   dg_status s;
@@ -419,10 +422,10 @@ dg_status run_decode(const void* A, const float* sfa, const void* B, const float
   args.drop_arrive = take_drop_flag();
   if (print_configs())
     std::fprintf(stderr,
-                 "[dg] fp8_gemm_nt decode M=%d N=%d K=%d: swap-AB BNP=%d, n_tiles=%d x "
+                 "[dg] fp8_gemm_nt decode M=%d N=%d K=%d: swap-AB BNP=%d (%d CTA/SM), n_tiles=%d x "
                  "split-K %d (cluster), %d CTAs, %d stages\n",
-                 M, N, K, BNP, n_tiles, splits, n_tiles * splits, Cfg::STAGES);
-  cudaError_t e = launch(dg::gemm_decode_kernel<BNP>, dim3(splits, n_tiles, 1), dim3(320),
+                 M, N, K, BNP, MINB, n_tiles, splits, n_tiles * splits, Cfg::STAGES);
+  cudaError_t e = launch(dg::gemm_decode_kernel<BNP, MINB>, dim3(splits, n_tiles, 1), dim3(320),
                          Cfg::SMEM_BYTES, st, splits, tw, tx, tsa, args);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   g_launches.fetch_add(1);
@@ -432,10 +435,42 @@ dg_status run_decode(const void* A, const float* sfa, const void* B, const float
 dg_status dispatch_decode(const void* A, const float* sfa, const void* B, const float* sfb,
                           const void* C, void* D, int M, int N, int K, int sms, int dev,
                           cudaStream_t st) {
-  if (M <= 16) return run_decode<16>(A, sfa, B, sfb, C, D, M, N, K, sms, dev, st);
-  if (M <= 32) return run_decode<32>(A, sfa, B, sfb, C, D, M, N, K, sms, dev, st);
-  if (M <= 64) return run_decode<64>(A, sfa, B, sfb, C, D, M, N, K, sms, dev, st);
-  return run_decode<128>(A, sfa, B, sfb, C, D, M, N, K, sms, dev, st);
+  const int KB = K / 128;
+  const int n_tiles = (N + 127) / 128;
+  const int bnp = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  int cap1 = 0, cap2 = 0;  // co-schedulable cluster sizes of the two configurations
+  switch (bnp) {
+    case 16: cap1 = max_cluster<16, 1>(dev); cap2 = max_cluster<16, 2>(dev); break;
+    case 32: cap1 = max_cluster<32, 1>(dev); cap2 = max_cluster<32, 2>(dev); break;
+    case 64: cap1 = max_cluster<64, 1>(dev); cap2 = max_cluster<64, 2>(dev); break;
+    default: cap1 = max_cluster<128, 1>(dev); cap2 = max_cluster<128, 2>(dev); break;
+  }
+  if (cap1 <= 0 || cap2 <= 0) return DG_ERR_CUDA;
+  DecodePlan p = plan_decode(M, n_tiles, KB, sms, cap1, cap2);
+  // DG_DECODE_MINB=1|2 and DG_DECODE_SPLITS=s force the plan (comparisons;
+  // splits clamped to the cluster limit and to one K-block per split); read
+  // on every call
+  if (const char* e = std::getenv("DG_DECODE_MINB")) {
+    const int f = std::atoi(e);
+    if (f == 1 || f == 2) p.minb = f;
+  }
+  const int cap = p.minb == 1 ? cap1 : cap2;
+  p.splits = std::min(p.splits, std::min(cap, 8));
+  if (const char* e = std::getenv("DG_DECODE_SPLITS")) {
+    const int f = std::atoi(e);
+    if (f >= 1) p.splits = std::max(1, std::min(std::min(f, std::min(cap, 8)), KB));
+  }
+#define DG_RUN_DECODE(BNP_)                                                                   \
+  return p.minb == 1                                                                          \
+             ? run_decode<BNP_, 1>(A, sfa, B, sfb, C, D, M, N, K, p.splits, sms, dev, st) \
+             : run_decode<BNP_, 2>(A, sfa, B, sfb, C, D, M, N, K, p.splits, sms, dev, st)
+  switch (bnp) {
+    case 16: DG_RUN_DECODE(16);
+    case 32: DG_RUN_DECODE(32);
+    case 64: DG_RUN_DECODE(64);
+    default: DG_RUN_DECODE(128);
+  }
+#undef DG_RUN_DECODE
 }
 
 }  // namespace

@@ -13,7 +13,8 @@
 //     share one N-tile and each streams its own slice of K-blocks, so
 //     n_tiles x splits CTAs keep HBM busy even when N/128 is small;
 //   * the partial tiles are reduced through distributed shared memory: CTA r
-//     owns 16/splits of the tile's sixteen 8-row units; after a cluster
+//     owns units [16r/splits, 16(r+1)/splits) of the tile's sixteen 8-row
+//     units (splits <= 8, any count); after a cluster
 //     barrier (every ring is free) each CTA pushes, with remote stores, the
 //     rows of its FP32 partial that CTA o owns into o's receive slot for
 //     rank r; after a second barrier each CTA sums its units over the slots in
@@ -51,13 +52,18 @@ struct DecodeArgs {
   int drop_arrive;
 };
 
-template <int BNP_>
+// MINB = CTAs per SM the configuration is built for: 2 (a CTA gets half of
+// shared memory, registers and TMEM) or 1 (the whole SM: every promotion
+// thread loads all its accumulator columns in one TMEM round trip, and twice
+// the accumulator buffers).
+template <int BNP_, int MINB_>
 struct DecodeCfg {
   static constexpr int BNP = BNP_;              // token columns (MMA N)
+  static constexpr int MINB = MINB_;
   static constexpr int BK = 128;
   static constexpr int W_BYTES = 128 * BK;      // weight tile (MMA A operand)
   static constexpr int X_BYTES = BNP * BK;      // token tile (MMA B operand)
-  static constexpr int RING = 96 * 1024;
+  static constexpr int RING = MINB == 2 ? 96 * 1024 : 192 * 1024;
   static constexpr int STAGES_RAW = RING / (W_BYTES + X_BYTES);
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int SS = 8;                  // sfa slots
@@ -65,9 +71,12 @@ struct DecodeCfg {
   // slot holds at least 32 floats even when BNP = 16
   static constexpr int SLOT_FLOATS = BNP < 32 ? 32 : BNP;
   static constexpr int EC = BNP / 2;            // accumulator columns per promotion thread
-  static constexpr int CH = EC < 16 ? EC : 16;  // columns per tcgen05.ld
-  // accumulator buffers: a CTA owns half of TMEM (two CTAs per SM)
-  static constexpr int NACC = 256 / BNP > 8 ? 8 : 256 / BNP;
+  // columns per tcgen05.ld; with one CTA per SM all EC columns are in flight
+  // before a single wait, with two the loads go one 16-column chunk at a time
+  static constexpr int CH = MINB == 1 ? (EC < 32 ? EC : 32) : (EC < 16 ? EC : 16);
+  static constexpr bool ALL_IN_FLIGHT = MINB == 1;
+  // accumulator buffers in this CTA's share of TMEM
+  static constexpr int NACC = (512 / MINB) / BNP > 8 ? 8 : (512 / MINB) / BNP;
   static constexpr int TMEM_COLS = NACC * BNP;
   static constexpr int OFF_W = 0;
   static constexpr int OFF_X = OFF_W + STAGES * W_BYTES;
@@ -77,27 +86,30 @@ struct DecodeCfg {
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   // receive slots of the split-K reduction, overlaying the ring:
-  // [src rank][owned unit][row in unit (8)][RECV_PITCH] floats, tokens along
-  // the row; the 16 units x 8 rows of a tile fill 128 rows in total. The pitch
-  // is padded by 4 floats so that consecutive rows start in different banks.
+  // [src rank][owned unit (< ceil(16/splits))][row in unit (8)][RECV_PITCH]
+  // floats, tokens along the row; at most 168 rows (splits = 7: 7 x 3 x 8).
+  // The pitch is padded by 4 floats so that consecutive rows start in
+  // different banks.
+  static constexpr int MAX_SPLITS = 8;
   static constexpr int RECV_PITCH = BNP + 4;
-  static constexpr int RECV_BYTES = 128 * RECV_PITCH * 4;
+  static constexpr int RECV_ROWS = 168;
+  static constexpr int RECV_BYTES = RECV_ROWS * RECV_PITCH * 4;
   static_assert(RECV_BYTES <= STAGES * (W_BYTES + X_BYTES), "receive slots fit the ring");
   static_assert((NACC & (NACC - 1)) == 0 && TMEM_COLS >= 32 && (TMEM_COLS & (TMEM_COLS - 1)) == 0,
                 "TMEM allocation is a power of two >= 32 columns");
   static_assert(BNP == 16 || BNP == 32 || BNP == 64 || BNP == 128, "BNP");
   static_assert(OFF_SCALE % 1024 == 0 && (SLOT_FLOATS * 4) % 128 == 0, "TMA smem alignment");
   static_assert(OFF_X % 1024 == 0 && X_BYTES % 1024 == 0, "SW128 tiles are 1024-byte aligned");
-  static_assert(SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
+  static_assert(SMEM_BYTES <= (MINB == 2 ? 113 : 227) * 1024, "MINB CTAs per SM");
 };
 
-template <int BNP>
-__global__ void __launch_bounds__(320, 2)
+template <int BNP, int MINB>
+__global__ void __launch_bounds__(320, MINB)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tm_w,    // B: [N][K] e4m3
                        const __grid_constant__ CUtensorMap tm_x,    // A: [M][K] e4m3
                        const __grid_constant__ CUtensorMap tm_sfa,  // sfa: [KB][ld] f32
                        const __grid_constant__ DecodeArgs args) {
-  using Cfg = DecodeCfg<BNP>;
+  using Cfg = DecodeCfg<BNP, MINB>;
   constexpr int S = Cfg::STAGES;
   constexpr int SS = Cfg::SS;
   constexpr int EC = Cfg::EC;
@@ -261,16 +273,7 @@ __global__ void __launch_bounds__(320, 2)
         const float sb = sbr[u];
         if (it + 4 < nkb) sbr[u] = __ldg(pb + it + 4);
         const float* sa = sScale + ss * Cfg::SLOT_FLOATS + h * EC;
-#pragma unroll
-        for (int c = 0; c < EC / CH; ++c) {
-          uint32_t r[CH];
-          tmem_ld_32x32b<CH>(t_lane + b * BNP + h * EC + c * CH, r);
-          tmem_ld_wait();
-          if (c == EC / CH - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[b]);
-          }
+        auto fma_chunk = [&](int c, const uint32_t (&r)[CH]) {
 #pragma unroll
           for (int i = 0; i < CH; i += 4) {
             const float4 s4 = *reinterpret_cast<const float4*>(sa + c * CH + i);
@@ -281,6 +284,30 @@ __global__ void __launch_bounds__(320, 2)
                  __uint_as_float(r[i + 1]));
             fma2(acc[c * CH + i + 2], acc[c * CH + i + 3], t2, t3, __uint_as_float(r[i + 2]),
                  __uint_as_float(r[i + 3]));
+          }
+        };
+        auto release_tmem = [&]() {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[b]);
+        };
+        if constexpr (Cfg::ALL_IN_FLIGHT) {
+          uint32_t r[EC / CH][CH];
+#pragma unroll
+          for (int c = 0; c < EC / CH; ++c)
+            tmem_ld_32x32b<CH>(t_lane + b * BNP + h * EC + c * CH, r[c]);
+          tmem_ld_wait();
+          release_tmem();
+#pragma unroll
+          for (int c = 0; c < EC / CH; ++c) fma_chunk(c, r[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < EC / CH; ++c) {
+            uint32_t r[CH];
+            tmem_ld_32x32b<CH>(t_lane + b * BNP + h * EC + c * CH, r);
+            tmem_ld_wait();
+            if (c == EC / CH - 1) release_tmem();
+            fma_chunk(c, r);
           }
         }
         __syncwarp();
@@ -296,13 +323,15 @@ __global__ void __launch_bounds__(320, 2)
   tc_fence_before();
   pdl_trigger();
   if (splits > 1) cluster_sync_all(); else __syncthreads();
-  const int U = 16 / splits;  // 8-row units per rank (splits divides 16)
+  // rank o owns units [16o/splits, 16(o+1)/splits); a slot holds UMAX units
+  const int UMAX = (16 + splits - 1) / splits;
   if (warp >= 2) {
     // push: this thread holds row n_local of the tile for tokens [h*EC, h*EC+EC)
     const int n_local = static_cast<int>(q * 32 + lane);
     const int unit = n_local >> 3;
-    const int owner = unit / U;
-    const int slot_row = ((static_cast<int>(rank) * U + (unit - owner * U)) << 3) + (n_local & 7);
+    const int owner = (splits * (unit + 1) + 15) / 16 - 1;  // largest o with 16o/splits <= unit
+    const int owner_lo = (owner * 16) / splits;
+    const int slot_row = ((static_cast<int>(rank) * UMAX + (unit - owner_lo)) << 3) + (n_local & 7);
     float* dst = recv + slot_row * Cfg::RECV_PITCH + h * EC;
     if (splits == 1) {
 #pragma unroll
@@ -317,17 +346,19 @@ __global__ void __launch_bounds__(320, 2)
   }
   if (splits > 1) cluster_sync_all(); else __syncthreads();
   {
-    // CTA `rank` owns units [rank*U, rank*U + U); item = (unit uu, token m),
-    // token fastest so that a warp reads consecutive floats of a slot row
-    const int items = BNP * U;
+    // this CTA owns units [lo, hi); item = (unit uu, token m), token fastest
+    // so that a warp reads consecutive floats of a slot row
+    const int lo = (static_cast<int>(rank) * 16) / splits;
+    const int hi = ((static_cast<int>(rank) + 1) * 16) / splits;
+    const int items = BNP * (hi - lo);
     for (int itm = threadIdx.x; itm < items; itm += blockDim.x) {
       const int uu = itm / BNP;
       const int m = itm - uu * BNP;
-      const int gn = n0 + ((static_cast<int>(rank) * U + uu) << 3);
+      const int gn = n0 + ((lo + uu) << 3);
       if (m >= args.M || gn >= args.N) continue;
       float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       for (int src = 0; src < splits; ++src) {  // rank order: deterministic
-        const float* p = recv + ((src * U + uu) << 3) * Cfg::RECV_PITCH + m;
+        const float* p = recv + ((src * UMAX + uu) << 3) * Cfg::RECV_PITCH + m;
 #pragma unroll
         for (int r8 = 0; r8 < 8; ++r8) v[r8] += p[r8 * Cfg::RECV_PITCH];
       }

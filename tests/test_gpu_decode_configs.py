@@ -1,0 +1,34 @@
+"""Every configuration of the small-M (decode) kernel against the oracle.
+
+The planner picks CTAs per SM (1 or 2) and a split count; DG_DECODE_MINB and
+DG_DECODE_SPLITS force them for every call. Each case re-runs the decode
+parity tests in a child process with one forced plan (split counts that do
+not divide the 16 row-units of a tile included) and checks the config log.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+PLANS = [("1", None), ("2", None), ("1", "7"), ("2", "3"), ("2", "8")]
+
+
+@pytest.mark.parametrize("minb,splits", PLANS)
+def test_decode_kernel_configs_parity(minb, splits):
+    env = dict(os.environ, DG_DECODE_MINB=minb, DG_PRINT_CONFIGS="1")
+    if splits:
+        env["DG_DECODE_SPLITS"] = splits
+    cmd = [sys.executable, "-m", "pytest", "-x", "-q", "-s", "-m", "gpu", "-p", "no:cacheprovider",
+           "tests/test_gpu_gemm.py", "tests/test_gpu_failure.py",
+           "-k", "decode or graph or dropped_arrive"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    out = r.stdout + r.stderr
+    assert r.returncode == 0, out[-4000:]
+    assert f"({minb} CTA/SM)" in out, "forced configuration did not run:\n" + out[-2000:]
+    if splits:
+        assert f"split-K {splits} " in out, "forced split count did not run:\n" + out[-2000:]

@@ -71,6 +71,10 @@ DECODE_CASES = [
     (100, 2112, 3072, True),
     (128, 4096, 1408, False),   # 11 K-blocks: uneven split
     (128, 136, 128, True),      # a single K-block
+    # more tile counts for the split planner (42, 48 and 98 tiles of 128 rows)
+    (48, 5376, 2048, True),
+    (80, 6144, 2048, False),
+    (24, 12544, 768, True),
 ]
 
 
