@@ -151,6 +151,30 @@ dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void* A, const float* sfa, c
                                               float* D, int G, int M, int N, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * K-grouped GEMM with the per-group K sizes in DEVICE memory (a training
+ * backward captured in a CUDA graph, where the sizes are produced on the GPU
+ * and the host cannot read them). Source: README summary, "DenseとGrouped
+ * GEMM" (the K-grouped operation); the device-side sizes are this library's
+ * extension of it.
+ *
+ *   ks_dev      [G] int32 DEVICE array of per-group K sizes, read on the
+ *               device after the previous kernel on the stream completes.
+ *   k_capacity  K rows that A, B (and K/128 rows that sfa, sfb) hold; a
+ *               multiple of 128. The groups occupy rows [0, sum ks) of it.
+ *   Everything else as dg_k_grouped_fp8_gemm_tn_contiguous. Groups with
+ *   K = 0 get D_g = C_g (or 0).
+ * Device-side validation: a size that is negative or not a multiple of 128
+ * counts as 0, and the running sum is clamped to k_capacity; either case
+ * records DG_ERR_INVALID_ARG (site 9) for dg_get_last_device_error(). The
+ * call itself reads nothing on the host, so it can be captured in a graph.
+ * ------------------------------------------------------------------------- */
+dg_status dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks(const void* A, const float* sfa,
+                                                     const void* B, const float* sfb,
+                                                     const int32_t* ks_dev, int k_capacity,
+                                                     const float* C, float* D, int G, int M, int N,
+                                                     void* stream);
+
+/* ---------------------------------------------------------------------------
  * Utilities (README summary, section "ユーティリティと環境変数").
  * ------------------------------------------------------------------------- */
 /* M alignment every contiguous-layout segment must have: 128. */
@@ -171,7 +195,8 @@ int dg_get_pdl(void);
 
 /* Synchronises `stream`, then reads and clears this device's error word.
  * Returns DG_OK, DG_ERR_TIMEOUT (a bounded wait ran out; *site gets the code
- * of the wait that gave up, if site != NULL) or DG_ERR_CUDA. Debug/test use. */
+ * of the wait that gave up, if site != NULL), DG_ERR_INVALID_ARG (device-side
+ * sizes were invalid, site 9) or DG_ERR_CUDA. Debug/test use. */
 dg_status dg_get_last_device_error(void* stream, int* site);
 
 /* Test hook: when nonzero, the next GEMM launch drops one producer arrive so

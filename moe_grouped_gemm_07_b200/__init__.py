@@ -41,7 +41,7 @@ EXPORTED = (
     "dg_k_grouped_fp8_gemm_tn_contiguous", "dg_get_mk_alignment_for_contiguous_layout",
     "dg_get_tma_aligned_size", "dg_set_num_sms", "dg_get_num_sms", "dg_set_wait_timeout_ns",
     "dg_get_last_device_error", "dg_debug_drop_next_arrive", "dg_get_launch_count",
-    "dg_set_pdl", "dg_get_pdl",
+    "dg_set_pdl", "dg_get_pdl", "dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks",
 )
 
 _vp, _i32 = _C.c_void_p, _C.c_int
@@ -55,8 +55,11 @@ _lib.dg_m_grouped_fp8_gemm_nt_masked.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _
                                                  _i32, _vp]
 _lib.dg_k_grouped_fp8_gemm_tn_contiguous.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                                      _i32, _i32, _vp]
+_lib.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _vp,
+                                                            _vp, _i32, _i32, _i32, _vp]
 for _f in ("dg_quantize_fp8", "dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
-           "dg_m_grouped_fp8_gemm_nt_masked", "dg_k_grouped_fp8_gemm_tn_contiguous"):
+           "dg_m_grouped_fp8_gemm_nt_masked", "dg_k_grouped_fp8_gemm_tn_contiguous",
+           "dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks"):
     getattr(_lib, _f).restype = _i32
 _lib.dg_get_mk_alignment_for_contiguous_layout.restype = _i32
 _lib.dg_get_tma_aligned_size.argtypes = [_i32, _i32]
@@ -224,6 +227,27 @@ def dg_k_grouped_fp8_gemm_tn_contiguous(A, sfa, B, sfb, ks, C, D, stream=None):
     _check("dg_k_grouped_fp8_gemm_tn_contiguous",
            _lib.dg_k_grouped_fp8_gemm_tn_contiguous(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), ks_arr,
                                                     _ptr(C), _ptr(D), G, M, N, _stream(stream)))
+    return D
+
+
+def dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks(A, sfa, B, sfb, ks_dev, C, D, stream=None):
+    """As dg_k_grouped_fp8_gemm_tn_contiguous, with the per-group K sizes in a
+    CUDA int32 tensor ks_dev [G] (read on the device); A/B hold k_capacity =
+    A.shape[0] rows."""
+    _cuda_contig(A, sfa, B, sfb, ks_dev, C, D)
+    G = ks_dev.numel()
+    kcap, M = A.shape
+    N = B.shape[1]
+    _need(ks_dev.dtype == torch.int32, "ks_dev must be int32")
+    _need(_is_fp8(A) and _is_fp8(B) and B.shape[0] == kcap, "A/B")
+    _need(D.dtype == torch.float32 and tuple(D.shape) == (G, M, N), "D")
+    _need(C is None or (C.dtype == torch.float32 and tuple(C.shape) == (G, M, N)), "C")
+    _need(sfa.dtype == torch.float32 and sfa.numel() >= (kcap // 128) * M, "sfa")
+    _need(sfb.dtype == torch.float32 and sfb.numel() >= (kcap // 128) * N, "sfb")
+    _check("dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks",
+           _lib.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks(
+               _ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(ks_dev), kcap, _ptr(C), _ptr(D), G, M, N,
+               _stream(stream)))
     return D
 
 

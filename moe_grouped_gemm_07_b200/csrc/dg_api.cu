@@ -90,6 +90,7 @@ dg_status device_sms(int* dev, int* sms) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 unsigned long long timeout_ns() {
   const unsigned long long t = g_timeout_ns.load();
@@ -473,6 +474,80 @@ dg_status dispatch_decode(const void* A, const float* sfa, const void* B, const 
 #undef DG_RUN_DECODE
 }
 
+// K-grouped TN launcher. Sizes come either from the host (`ks`, sumK their
+// total) or from device memory (`ks_dev`, sumK = the K rows the operands
+// hold); the kernel builds the per-group K-block ranges itself in the latter
+// case.
+dg_status run_k_grouped(const void* A, const float* sfa, const void* B, const float* sfb,
+                        const int* ks, const int32_t* ks_dev, long long sumK, const float* C,
+                        float* D, int G, int M, int N, void* stream) {
+  if (M == 0 || N == 0) return DG_OK;
+  if (!D) return DG_ERR_INVALID_ARG;
+  if (!aligned16(D) || (C && !aligned16(C))) return DG_ERR_MISALIGNED;
+  int dev = 0, sms = 0;
+  dg_status s = device_sms(&dev, &sms);
+  if (s != DG_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (sumK == 0) return copy_or_zero<float>(C, D, static_cast<long long>(G) * M * N, sms, st);
+  if (!A || !B || !sfa || !sfb) return DG_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(sfa) || !aligned16(sfb))
+    return DG_ERR_MISALIGNED;
+  const int mb = (M + 127) / 128;
+  const int bn = choose_bn(static_cast<long long>(G) * mb, N, sms);
+  const uint64_t sumKB = static_cast<uint64_t>(sumK / 128);
+  CUtensorMap ta, tb, tsa, tsb;
+  if ((s = make_map_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, M, sumK, M, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  if ((s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, sumK, N, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  if ((s = make_map_2d(&tsa, sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, sumKB, 4ull * M, 128, 1,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
+    return s;
+  if ((s = make_map_2d(&tsb, sfb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, sumKB, 4ull * N, bn, 1,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
+    return s;
+  CUtensorMap td;  // D as [G*M][N] fp32; 16x32 boxes, 64-byte swizzle
+  if ((s = make_map_2d(&td, D, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, static_cast<uint64_t>(G) * M,
+                       4ull * N, 16, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != DG_OK)
+    return s;
+  GemmArgs args;
+  std::memset(&args, 0, sizeof args);
+  args.M = M;
+  args.N = N;
+  args.K = 0;
+  args.G = G;
+  args.d_rows = static_cast<long long>(G) * M;
+  args.num_m_blocks = mb;
+  args.num_n_blocks = (N + bn - 1) / bn;
+  const long long tiles = static_cast<long long>(G) * mb * args.num_n_blocks;
+  args.total_tiles = static_cast<int>(tiles);
+  args.C = C;
+  args.D = D;
+  args.timeout_ns = timeout_ns();
+  args.drop_arrive = take_drop_flag();
+  if (ks) {
+    int acc = 0;
+    for (int g = 0; g < G; ++g) {
+      args.kb_off[g] = acc;
+      acc += ks[g] / 128;
+    }
+    args.kb_off[G] = acc;
+  } else {
+    args.ks_dev = ks_dev;
+    args.kb_cap = static_cast<int>(sumKB);
+  }
+  const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(sms, tiles)));
+  if (print_configs())
+    std::fprintf(stderr,
+                 "[dg] k_grouped_fp8_gemm_tn M=%d N=%d %s=%lld G=%d: BN=%d tiles=%lld grid=%d\n",
+                 M, N, ks ? "sumK" : "K capacity (sizes on device)", sumK, G, bn, tiles, grid);
+  if (bn == 256)
+    return launch_gemm<dg::MODE_KGROUPED, 256>(ta, tb, tsa, tsb, td, args, grid, st, dev);
+  return launch_gemm<dg::MODE_KGROUPED, 128>(ta, tb, tsa, tsb, td, args, grid, st, dev);
+}
+
 }  // namespace
 
 // =============================================================== C ABI
@@ -529,6 +604,7 @@ dg_status dg_get_last_device_error(void* stream, int* site) {
   if (site) *site = static_cast<int>(w[1]);
   if (w[0] == 0) return DG_OK;
   if (w[0] == static_cast<unsigned int>(DG_ERR_TIMEOUT)) return DG_ERR_TIMEOUT;
+  if (w[0] == static_cast<unsigned int>(DG_ERR_INVALID_ARG)) return DG_ERR_INVALID_ARG;
   return DG_ERR_CUDA;
 }
 
@@ -665,65 +741,20 @@ dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void* A, const float* sfa, c
     sumK += ks[g];
   }
   if (sumK > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
-  if (M == 0 || N == 0) return DG_OK;
-  if (!D) return DG_ERR_INVALID_ARG;
-  if (!aligned16(D) || (C && !aligned16(C))) return DG_ERR_MISALIGNED;
-  int dev = 0, sms = 0;
-  dg_status s = device_sms(&dev, &sms);
-  if (s != DG_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (sumK == 0) return copy_or_zero<float>(C, D, static_cast<long long>(G) * M * N, sms, st);
-  if (!A || !B || !sfa || !sfb) return DG_ERR_INVALID_ARG;
-  if (!aligned16(A) || !aligned16(B) || !aligned16(sfa) || !aligned16(sfb))
-    return DG_ERR_MISALIGNED;
-  const int mb = (M + 127) / 128;
-  const int bn = choose_bn(static_cast<long long>(G) * mb, N, sms);
-  const uint64_t sumKB = static_cast<uint64_t>(sumK / 128);
-  CUtensorMap ta, tb, tsa, tsb;
-  if ((s = make_map_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, M, sumK, M, 128, 128,
-                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
-    return s;
-  if ((s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, sumK, N, 128, 128,
-                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
-    return s;
-  if ((s = make_map_2d(&tsa, sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, sumKB, 4ull * M, 128, 1,
-                       CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
-    return s;
-  if ((s = make_map_2d(&tsb, sfb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, sumKB, 4ull * N, bn, 1,
-                       CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
-    return s;
-  CUtensorMap td;  // D as [G*M][N] fp32; 16x32 boxes, 64-byte swizzle
-  if ((s = make_map_2d(&td, D, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, static_cast<uint64_t>(G) * M,
-                       4ull * N, 16, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != DG_OK)
-    return s;
-  GemmArgs args;
-  std::memset(&args, 0, sizeof args);
-  args.M = M;
-  args.N = N;
-  args.K = 0;
-  args.G = G;
-  args.d_rows = static_cast<long long>(G) * M;
-  args.num_m_blocks = mb;
-  args.num_n_blocks = (N + bn - 1) / bn;
-  const long long tiles = static_cast<long long>(G) * mb * args.num_n_blocks;
-  args.total_tiles = static_cast<int>(tiles);
-  args.C = C;
-  args.D = D;
-  args.timeout_ns = timeout_ns();
-  args.drop_arrive = take_drop_flag();
-  int acc = 0;
-  for (int g = 0; g < G; ++g) {
-    args.kb_off[g] = acc;
-    acc += ks[g] / 128;
-  }
-  args.kb_off[G] = acc;
-  const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(sms, tiles)));
-  if (print_configs())
-    std::fprintf(stderr, "[dg] k_grouped_fp8_gemm_tn M=%d N=%d sumK=%lld G=%d: BN=%d tiles=%lld grid=%d\n",
-                 M, N, sumK, G, bn, tiles, grid);
-  if (bn == 256)
-    return launch_gemm<dg::MODE_KGROUPED, 256>(ta, tb, tsa, tsb, td, args, grid, st, dev);
-  return launch_gemm<dg::MODE_KGROUPED, 128>(ta, tb, tsa, tsb, td, args, grid, st, dev);
+  return run_k_grouped(A, sfa, B, sfb, ks, nullptr, sumK, C, D, G, M, N, stream);
+}
+
+dg_status dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks(const void* A, const float* sfa,
+                                                     const void* B, const float* sfb,
+                                                     const int32_t* ks_dev, int k_capacity,
+                                                     const float* C, float* D, int G, int M, int N,
+                                                     void* stream) {
+  if (G < 1 || M < 0 || N < 0 || k_capacity < 0) return DG_ERR_INVALID_ARG;
+  if (G > dg::kMaxKGroups || M % 16 != 0 || N % 16 != 0 || k_capacity % 128 != 0)
+    return DG_ERR_UNSUPPORTED_SHAPE;
+  if (k_capacity > 0 && !ks_dev) return DG_ERR_INVALID_ARG;
+  if (ks_dev && !aligned4(ks_dev)) return DG_ERR_MISALIGNED;
+  return run_k_grouped(A, sfa, B, sfb, nullptr, ks_dev, k_capacity, C, D, G, M, N, stream);
 }
 
 }  // extern "C"

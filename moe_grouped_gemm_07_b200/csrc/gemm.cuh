@@ -58,7 +58,9 @@ struct GemmArgs {
   long long d_rows;  // rows of D viewed as [d_rows][N] (the store tensor map's outer extent)
   unsigned long long timeout_ns;
   int drop_arrive;
-  int kb_off[kMaxKGroups + 1];  // K-grouped: prefix sums of K-blocks per group
+  int kb_off[kMaxKGroups + 1];  // K-grouped, host sizes: prefix sums of K-blocks per group
+  const int32_t* ks_dev;        // K-grouped, device sizes: [G] K per group (else null)
+  int kb_cap;                   // K-grouped, device sizes: K-blocks the operands hold
 };
 
 template <int MODE, int BN_>
@@ -99,7 +101,9 @@ struct GemmCfg {
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NACC + 2 * SCALE_SLOTS + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;       // tmem slot, abort flag
   static constexpr int OFF_PREFIX = OFF_MISC + 16;              // masked: prefix + counts
-  static constexpr int PREFIX_BYTES = MODE == MODE_MASKED ? (2 * kMaxMaskedGroups + 1) * 4 : 0;
+  static constexpr int PREFIX_BYTES = MODE == MODE_MASKED     ? (2 * kMaxMaskedGroups + 1) * 4
+                                      : MODE == MODE_KGROUPED ? (kMaxKGroups + 1) * 4
+                                                              : 0;
   static constexpr int SMEM_BYTES = OFF_PREFIX + PREFIX_BYTES + 1024;  // + alignment slack
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   // TMA destinations: 128-byte aligned; 128B-swizzled tiles 1024-byte aligned
@@ -205,8 +209,8 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int*
     tl.n0 = nb * BN;
     tl.a_row = tl.m0;
     tl.b_row = tl.n0;
-    tl.kb0 = a.kb_off[g];
-    tl.nkb = a.kb_off[g + 1] - a.kb_off[g];
+    tl.kb0 = prefix[g];
+    tl.nkb = prefix[g + 1] - prefix[g];
     tl.rows = min(Cfg::BM, a.M - tl.m0);
     tl.out_row0 = static_cast<long long>(g) * a.M + tl.m0;
   }
@@ -231,6 +235,7 @@ enum : unsigned int {
   SITE_EPI_SCALE_FULL = 6,
   SITE_TEARDOWN_TMA = 7,
   SITE_TEARDOWN_MMA = 8,
+  SITE_K_SIZES = 9,  // device-side K-group sizes were invalid (DG_ERR_INVALID_ARG)
 };
 
 template <int MODE, int BN>
@@ -342,6 +347,46 @@ __global__ void __launch_bounds__(320, 1)
       }
       if (lane == 0) prefix[0] = 0;
     }
+  }
+  if constexpr (MODE == MODE_KGROUPED) {
+    // K-block ranges of the groups in shared memory: from the host's prefix
+    // sums, or built here from per-group K sizes in device memory (written
+    // by an earlier kernel, hence after pdl_wait). A size that is negative
+    // or not a multiple of 128 counts as 0, and the running total is clamped
+    // to the K-blocks the operands hold; either records DG_ERR_INVALID_ARG
+    // with site SITE_K_SIZES in the error word.
+    if (warp == 2) {
+      if (args.ks_dev == nullptr) {
+        for (int g = lane; g <= args.G; g += 32) prefix[g] = args.kb_off[g];
+      } else {
+        int carry = 0;
+        bool bad = false;
+        for (int base = 0; base < args.G; base += 32) {
+          const int g = base + lane;
+          int v = 0;
+          if (g < args.G) {
+            const int k = __ldg(args.ks_dev + g);
+            if (k >= 0 && (k & 127) == 0) v = k >> 7; else bad = true;
+            if (v > args.kb_cap) { v = args.kb_cap; bad = true; }
+          }
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= static_cast<uint32_t>(o)) v += y;
+          }
+          // kb_cap < 2^24, so v < 2^29 and carry + v fits in 32 bits
+          if (g < args.G) {
+            const int p = carry + v;
+            if (p > args.kb_cap) bad = true;
+            prefix[g + 1] = min(p, args.kb_cap);
+          }
+          carry = min(carry + __shfl_sync(0xffffffffu, v, 31), args.kb_cap);
+        }
+        if (lane == 0) prefix[0] = 0;
+        if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(1u, SITE_K_SIZES);
+      }
+    }
+    __syncthreads();
   }
   if constexpr (MODE == MODE_MASKED) {
     __syncthreads();

@@ -86,6 +86,19 @@ def test_host_validation_before_any_cuda_call():
     ks = (ctypes.c_int * 1)(128)
     assert L.dg_k_grouped_fp8_gemm_tn_contiguous(fake, fake, fake, fake, ks, None, fake, 1, 24,
                                                  16, None) == dg.DG_ERR_UNSUPPORTED_SHAPE
+    # device-side K sizes: capacity and group checks happen on the host
+    dk = L.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks
+    assert dk(fake, fake, fake, fake, fake, 100, None, fake, 2, 16, 16, None) == \
+        dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert dk(fake, fake, fake, fake, None, 128, None, fake, 2, 16, 16, None) == \
+        dg.DG_ERR_INVALID_ARG
+    assert dk(fake, fake, fake, fake, fake, 128, None, fake, 0, 16, 16, None) == \
+        dg.DG_ERR_INVALID_ARG
+    assert dk(fake, fake, fake, fake, fake, 128, None, fake, 300, 16, 16, None) == \
+        dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert dk(fake, fake, fake, fake, vp(0x1002), 128, None, fake, 2, 16, 16, None) == \
+        dg.DG_ERR_MISALIGNED
+    assert dk(fake, fake, fake, fake, fake, 128, None, fake, 2, 0, 16, None) == dg.DG_OK
     assert L.dg_quantize_fp8(fake, 0, 1, 128, 100, 0, fake, fake, 128, None) == \
         dg.DG_ERR_UNSUPPORTED_SHAPE
     assert L.dg_quantize_fp8(fake, 0, 1, 100, 128, 2, fake, fake, 0, None) == \

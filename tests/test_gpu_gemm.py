@@ -232,6 +232,84 @@ def test_k_grouped_vs_oracle(G, M, N, ks, with_c):
             assert np.array_equal(D[g].cpu().numpy(), expect)
 
 
+@pytest.mark.parametrize("ks,extra", [([256, 0, 384, 128], 0), ([128, 640], 256), ([0, 0, 128], 128)])
+def test_k_grouped_device_sizes(ks, extra):
+    """Sizes in device memory (capacity may exceed their sum): same result as
+    the host-size call bit for bit, and the oracle's within tolerance."""
+    G, M, N = len(ks), 256, 384
+    w = wl.k_grouped(G=G, M=M, N=N, ks=ks, cfg=89, shape=G + extra)
+    A = np.concatenate([w.A, np.zeros((extra, M), np.float32)])
+    B = np.concatenate([w.B, np.zeros((extra, N), np.float32)])
+    qa, sa = dg.dg_quantize_fp8(to_dev(A), dg.DG_QUANT_COL_128x1)
+    qb, sb = dg.dg_quantize_fp8(to_dev(B), dg.DG_QUANT_COL_128x1)
+    C = to_dev(w.C)
+    D1 = torch.empty((G, M, N), dtype=torch.float32, device=dev())
+    D2 = torch.empty_like(D1)
+    ks_dev = torch.tensor(ks, dtype=torch.int32, device=dev())
+    dg.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks(qa, sa, qb, sb, ks_dev, C, D1)
+    assert dg.dg_get_last_device_error() == (dg.DG_OK, 0)
+    s = sum(ks)
+    dg.dg_k_grouped_fp8_gemm_tn_contiguous(qa[:s], sa[: s // 128], qb[:s], sb[: s // 128], ks, C, D2)
+    assert torch.equal(D1, D2)
+    oqa, osa = oracle.quantize(w.A, oracle.COL_128x1)
+    oqb, osb = oracle.quantize(w.B, oracle.COL_128x1)
+    R = oracle.k_grouped_tn(oqa, osa, oqb, osb, ks, w.C)
+    check_close(D1.cpu().numpy().astype(np.float64), R, "k-grouped, device sizes")
+
+
+def test_k_grouped_device_sizes_invalid_are_reported():
+    """A size that is not a multiple of 128, or a sum beyond the capacity,
+    counts as empty / is clamped and is reported as DG_ERR_INVALID_ARG."""
+    G, M, N = 3, 128, 256
+    w = wl.k_grouped(G=G, M=M, N=N, ks=[128, 256, 128], cfg=90)
+    qa, sa = dg.dg_quantize_fp8(to_dev(w.A), dg.DG_QUANT_COL_128x1)
+    qb, sb = dg.dg_quantize_fp8(to_dev(w.B), dg.DG_QUANT_COL_128x1)
+    C = to_dev(w.C)
+    D = torch.empty((G, M, N), dtype=torch.float32, device=dev())
+    bad = torch.tensor([128, 100, 256], dtype=torch.int32, device=dev())  # 100: not a multiple
+    dg.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks(qa, sa, qb, sb, bad, C, D)
+    st, site = dg.dg_get_last_device_error()
+    assert st == dg.DG_ERR_INVALID_ARG and site == 9
+    # group 1 counted as empty: D_1 = C_1 exactly; groups 0 and 2 use rows [0,128), [128,384)
+    assert torch.equal(D[1], C[1])
+    over = torch.tensor([256, 256, 256], dtype=torch.int32, device=dev())  # sum 768 > 512
+    dg.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks(qa, sa, qb, sb, over, C, D)
+    st, site = dg.dg_get_last_device_error()
+    assert st == dg.DG_ERR_INVALID_ARG and site == 9
+    assert torch.equal(D[2], C[2])  # clamped to the 512 rows: group 2 gets none
+    good = torch.tensor([128, 256, 128], dtype=torch.int32, device=dev())
+    dg.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks(qa, sa, qb, sb, good, C, D)
+    assert dg.dg_get_last_device_error() == (dg.DG_OK, 0)
+
+
+def test_k_grouped_device_sizes_graph_replay():
+    """Captured once, replayed with new sizes written into the same device
+    array: every replay matches a fresh host-size call."""
+    G, M, N, cap = 3, 128, 256, 768
+    w = wl.k_grouped(G=G, M=M, N=N, ks=[256, 256, 256], cfg=91)
+    qa, sa = dg.dg_quantize_fp8(to_dev(w.A), dg.DG_QUANT_COL_128x1)
+    qb, sb = dg.dg_quantize_fp8(to_dev(w.B), dg.DG_QUANT_COL_128x1)
+    D = torch.empty((G, M, N), dtype=torch.float32, device=dev())
+    ks_dev = torch.tensor([256, 256, 256], dtype=torch.int32, device=dev())
+    dg.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks(qa, sa, qb, sb, ks_dev, None, D)  # set-up call
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            dg.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks(qa, sa, qb, sb, ks_dev, None, D)
+    for ks in ([256, 256, 256], [0, 640, 128], [384, 0, 0]):
+        ks_dev.copy_(torch.tensor(ks, dtype=torch.int32))
+        g.replay()
+        torch.cuda.synchronize()
+        ref = torch.empty_like(D)
+        n = sum(ks)
+        dg.dg_k_grouped_fp8_gemm_tn_contiguous(qa[:n], sa[: n // 128], qb[:n], sb[: n // 128], ks,
+                                               None, ref)
+        torch.cuda.synchronize()
+        assert torch.equal(D, ref), ks
+
+
 def test_k_grouped_accumulates_in_place():
     G, M, N, ks = 2, 128, 256, [256, 384]
     w = wl.k_grouped(G=G, M=M, N=N, ks=ks, cfg=87)
