@@ -151,6 +151,38 @@ dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void* A, const float* sfa, c
                                               float* D, int G, int M, int N, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Power-of-two (UE8M0) scales and the tensor core's block-scaled MMA.
+ * Source: README summary, "GEMMインターフェースとレイアウト制約" (UE8M0 scales,
+ * four packed per int32); the hardware path replaces the per-K-block
+ * promotion with tcgen05.mma kind::mxf8f6f4 block scaling, so it relies on
+ * the tensor core's own FP32 accumulation across K-blocks.
+ *
+ * dg_quantize_fp8_ue8m0: as dg_quantize_fp8 (batch 1, modes ROW_1x128 or
+ * BLOCK_128x128, cols % 128 == 0), but every scale is rounded up to a power
+ * of two, s = 2^ceil(log2(max(amax, 1e-4f) / 448)), and code = E4M3_RN(x / s)
+ * (exact division, never saturating).
+ *   scales  optional (NULL allowed): FP32 scales in dg_quantize_fp8's layout
+ *           for that mode (usable by dg_fp8_gemm_nt, the promotion path).
+ *   packed  int32 [ceil(cols/512)][ceil(rows/128)][32][4] (written): byte b of
+ *           word [q][rb][i][j] = biased exponent (log2 s + 127) of row
+ *           128 rb + 32 j + i for K-block 4 q + b. BLOCK mode writes its block
+ *           scale for all 128 rows of the block (rows past `rows` included).
+ *           Bytes of K-blocks past cols/128, and of rows past `rows` in ROW
+ *           mode, are not written.
+ * ------------------------------------------------------------------------- */
+dg_status dg_quantize_fp8_ue8m0(const void* x, int in_dtype, int rows, int cols, int mode,
+                                void* codes, float* scales, int ld_scales, int32_t* packed,
+                                void* stream);
+
+/* Dense NT GEMM on the block-scaled MMA: D = C + A @ B.T with sfa / sfb the
+ * packed UE8M0 scales of A (ROW mode, rows = M) and B (BLOCK mode, rows = N)
+ * from dg_quantize_fp8_ue8m0. A [M][K], B [N][K] E4M3; C [M][N] BF16 or NULL
+ * (may alias D); D [M][N] BF16. K % 128 == 0, N % 8 == 0. */
+dg_status dg_fp8_gemm_nt_ue8m0(const void* A, const int32_t* sfa, const void* B,
+                               const int32_t* sfb, const void* C, void* D, int M, int N, int K,
+                               void* stream);
+
+/* ---------------------------------------------------------------------------
  * K-grouped GEMM with the per-group K sizes in DEVICE memory (a training
  * backward captured in a CUDA graph, where the sizes are produced on the GPU
  * and the host cannot read them). Source: README summary, "DenseとGrouped

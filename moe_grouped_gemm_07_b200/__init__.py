@@ -17,6 +17,7 @@ Functions keep the C names:
 from __future__ import annotations
 
 import ctypes as _C
+import math
 import os as _os
 
 import torch
@@ -42,6 +43,7 @@ EXPORTED = (
     "dg_get_tma_aligned_size", "dg_set_num_sms", "dg_get_num_sms", "dg_set_wait_timeout_ns",
     "dg_get_last_device_error", "dg_debug_drop_next_arrive", "dg_get_launch_count",
     "dg_set_pdl", "dg_get_pdl", "dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks",
+    "dg_quantize_fp8_ue8m0", "dg_fp8_gemm_nt_ue8m0",
 )
 
 _vp, _i32 = _C.c_void_p, _C.c_int
@@ -57,9 +59,12 @@ _lib.dg_k_grouped_fp8_gemm_tn_contiguous.argtypes = [_vp, _vp, _vp, _vp, _vp, _v
                                                      _i32, _i32, _vp]
 _lib.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _vp,
                                                             _vp, _i32, _i32, _i32, _vp]
+_lib.dg_quantize_fp8_ue8m0.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp]
+_lib.dg_fp8_gemm_nt_ue8m0.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]
 for _f in ("dg_quantize_fp8", "dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
            "dg_m_grouped_fp8_gemm_nt_masked", "dg_k_grouped_fp8_gemm_tn_contiguous",
-           "dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks"):
+           "dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks", "dg_quantize_fp8_ue8m0",
+           "dg_fp8_gemm_nt_ue8m0"):
     getattr(_lib, _f).restype = _i32
 _lib.dg_get_mk_alignment_for_contiguous_layout.restype = _i32
 _lib.dg_get_tma_aligned_size.argtypes = [_i32, _i32]
@@ -227,6 +232,60 @@ def dg_k_grouped_fp8_gemm_tn_contiguous(A, sfa, B, sfb, ks, C, D, stream=None):
     _check("dg_k_grouped_fp8_gemm_tn_contiguous",
            _lib.dg_k_grouped_fp8_gemm_tn_contiguous(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), ks_arr,
                                                     _ptr(C), _ptr(D), G, M, N, _stream(stream)))
+    return D
+
+
+def ue8m0_packed_shape(rows: int, cols: int):
+    """Shape of the packed UE8M0 scale tensor (int32) of a [rows, cols] operand."""
+    return ((cols + 511) // 512, (rows + 127) // 128, 32, 4)
+
+
+def dg_quantize_fp8_ue8m0(x, mode, codes=None, scales=None, packed=None, with_scales=True,
+                          stream=None):
+    """x [rows, cols] f32/bf16 CUDA; mode DG_QUANT_ROW_1x128 or DG_QUANT_BLOCK_128x128.
+    Power-of-two scales. Returns (codes, FP32 scales or None, packed UE8M0 int32)."""
+    _cuda_contig(x, codes, scales, packed)
+    _need(x.dim() == 2, "x must be 2-D")
+    rows, cols = x.shape
+    _need(mode in (DG_QUANT_ROW_1x128, DG_QUANT_BLOCK_128x128), "mode")
+    dt = DG_IN_BF16 if x.dtype == torch.bfloat16 else DG_IN_F32
+    _need(x.dtype in (torch.float32, torch.bfloat16), "x dtype")
+    if codes is None:
+        codes = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    ld = 0
+    if with_scales and scales is None:
+        if mode == DG_QUANT_ROW_1x128:
+            scales = torch.zeros((cols // 128, align4(rows)), dtype=torch.float32, device=x.device)
+        else:
+            scales = torch.zeros(((rows + 127) // 128, cols // 128), dtype=torch.float32,
+                                 device=x.device)
+    if scales is not None and mode == DG_QUANT_ROW_1x128:
+        ld = scales.shape[-1]
+    if packed is None:
+        packed = torch.zeros(ue8m0_packed_shape(rows, cols), dtype=torch.int32, device=x.device)
+    _need(packed.dtype == torch.int32 and packed.numel() >= math.prod(ue8m0_packed_shape(rows, cols)),
+          "packed")
+    _check("dg_quantize_fp8_ue8m0",
+           _lib.dg_quantize_fp8_ue8m0(_ptr(x), dt, rows, cols, mode, _ptr(codes), _ptr(scales), ld,
+                                      _ptr(packed), _stream(stream)))
+    return codes, scales, packed
+
+
+def dg_fp8_gemm_nt_ue8m0(A, sfa_packed, B, sfb_packed, C, D, stream=None):
+    """D = C + A @ B.T on the block-scaled MMA with packed UE8M0 scales."""
+    _cuda_contig(A, sfa_packed, B, sfb_packed, C, D)
+    M, K = A.shape
+    N = B.shape[0]
+    _need(_is_fp8(A) and _is_fp8(B) and B.shape[1] == K, "A/B")
+    _need(D.dtype == torch.bfloat16 and tuple(D.shape) == (M, N), "D")
+    _need(C is None or (C.dtype == torch.bfloat16 and tuple(C.shape) == (M, N)), "C")
+    _need(sfa_packed.dtype == torch.int32 and
+          sfa_packed.numel() >= math.prod(ue8m0_packed_shape(M, K)), "sfa_packed")
+    _need(sfb_packed.dtype == torch.int32 and
+          sfb_packed.numel() >= math.prod(ue8m0_packed_shape(N, K)), "sfb_packed")
+    _check("dg_fp8_gemm_nt_ue8m0",
+           _lib.dg_fp8_gemm_nt_ue8m0(_ptr(A), _ptr(sfa_packed), _ptr(B), _ptr(sfb_packed), _ptr(C),
+                                     _ptr(D), M, N, K, _stream(stream)))
     return D
 
 

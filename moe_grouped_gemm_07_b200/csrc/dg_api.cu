@@ -13,6 +13,7 @@
 
 #include "../../include/dg.h"
 #include "gemm.cuh"
+#include "gemm_mx.cuh"
 #include "gemm_decode.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
@@ -548,6 +549,59 @@ dg_status run_k_grouped(const void* A, const float* sfa, const void* B, const fl
   return launch_gemm<dg::MODE_KGROUPED, 128>(ta, tb, tsa, tsb, td, args, grid, st, dev);
 }
 
+// UE8M0 block-scaled dense GEMM launcher (one CTA per SM, persistent).
+dg_status run_mx(const void* A, const int32_t* sfa, const void* B, const int32_t* sfb,
+                 const void* C, void* D, int M, int N, int K, cudaStream_t st) {
+  int dev = 0, sms = 0;
+  dg_status s = device_sms(&dev, &sms);
+  if (s != DG_OK) return s;
+  using Cfg = dg::MxCfg;
+  CUtensorMap ta, tb, td;
+  if ((s = make_map_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  if ((s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, 128, Cfg::BN,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  if ((s = make_map_2d(&td, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, 2ull * N, 32, 32,
+                       CU_TENSOR_MAP_SWIZZLE_64B)) != DG_OK)
+    return s;
+  dg::MxArgs args;
+  std::memset(&args, 0, sizeof args);
+  args.M = M;
+  args.N = N;
+  args.K = K;
+  args.num_m_blocks = (M + 127) / 128;
+  args.num_n_blocks = (N + Cfg::BN - 1) / Cfg::BN;
+  const long long tiles = static_cast<long long>(args.num_m_blocks) * args.num_n_blocks;
+  if (tiles > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
+  args.total_tiles = static_cast<int>(tiles);
+  args.rb_a = (M + 127) / 128;
+  args.rb_b = (N + 127) / 128;
+  args.sfa = sfa;
+  args.sfb = sfb;
+  args.C = C;
+  args.D = D;
+  args.timeout_ns = timeout_ns();
+  args.drop_arrive = take_drop_flag();
+  const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(sms, tiles)));
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t attr_err[kMaxDevices];
+  std::call_once(once[dev], [&] {
+    attr_err[dev] = cudaFuncSetAttribute(dg::gemm_mx_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+  });
+  if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
+  if (print_configs())
+    std::fprintf(stderr, "[dg] fp8_gemm_nt_ue8m0 M=%d N=%d K=%d: 128x256 block-scaled tiles=%lld grid=%d\n",
+                 M, N, K, tiles, grid);
+  cudaError_t e = launch(dg::gemm_mx_kernel, dim3(grid), dim3(320), Cfg::SMEM_BYTES, st, 1, ta, tb,
+                         td, args);
+  if (e != cudaSuccess) return cuda_fail(e, "mx gemm launch");
+  g_launches.fetch_add(1);
+  return DG_OK;
+}
+
 }  // namespace
 
 // =============================================================== C ABI
@@ -634,17 +688,19 @@ dg_status dg_quantize_fp8(const void* x, int in_dtype, int batch, int rows, int 
     const long long strips = static_cast<long long>(batch) * rows * (cols / 128);
     if (strips >= 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
     const int grid = static_cast<int>(std::min<long long>((strips + 31) / 32, 8ll * sms));
+    uint8_t* none = nullptr;
     e = bf ? launch(dg::quant_row_kernel<true>, dim3(grid), dim3(256), 0, st, 1, x, batch, rows,
-                    cols, q, scales, ld_scales)
+                    cols, q, scales, ld_scales, none)
            : launch(dg::quant_row_kernel<false>, dim3(grid), dim3(256), 0, st, 1, x, batch, rows,
-                    cols, q, scales, ld_scales);
+                    cols, q, scales, ld_scales, none);
   } else if (mode == DG_QUANT_BLOCK_128x128) {
     const long long blocks = static_cast<long long>(batch) * ((rows + 127) / 128) * (cols / 128);
     if (blocks > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
+    uint8_t* none = nullptr;
     e = bf ? launch(dg::quant_block_kernel<true>, dim3(static_cast<int>(blocks)), dim3(256), 0, st,
-                    1, x, batch, rows, cols, q, scales)
+                    1, x, batch, rows, cols, q, scales, none)
            : launch(dg::quant_block_kernel<false>, dim3(static_cast<int>(blocks)), dim3(256), 0, st,
-                    1, x, batch, rows, cols, q, scales);
+                    1, x, batch, rows, cols, q, scales, none);
   } else {
     const long long blocks = static_cast<long long>(batch) * (rows / 128) * ((cols + 63) / 64);
     if (blocks > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
@@ -656,6 +712,69 @@ dg_status dg_quantize_fp8(const void* x, int in_dtype, int batch, int rows, int 
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   g_launches.fetch_add(1);
   return DG_OK;
+}
+
+dg_status dg_quantize_fp8_ue8m0(const void* x, int in_dtype, int rows, int cols, int mode,
+                                void* codes, float* scales, int ld_scales, int32_t* packed,
+                                void* stream) {
+  if (rows < 0 || cols < 0) return DG_ERR_INVALID_ARG;
+  if (in_dtype != DG_IN_F32 && in_dtype != DG_IN_BF16) return DG_ERR_INVALID_ARG;
+  if (mode != DG_QUANT_ROW_1x128 && mode != DG_QUANT_BLOCK_128x128) return DG_ERR_INVALID_ARG;
+  if (cols % 128 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  if (mode == DG_QUANT_ROW_1x128 && scales && (ld_scales < rows || ld_scales % 4 != 0))
+    return DG_ERR_INVALID_ARG;
+  if (static_cast<long long>(rows) * cols == 0) return DG_OK;
+  if (!x || !codes || !packed) return DG_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(packed) || (scales && !aligned16(scales)))
+    return DG_ERR_MISALIGNED;
+  int dev = 0, sms = 0;
+  dg_status s = device_sms(&dev, &sms);
+  if (s != DG_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* q = static_cast<uint8_t*>(codes);
+  uint8_t* pk = reinterpret_cast<uint8_t*>(packed);
+  const bool bf = in_dtype == DG_IN_BF16;
+  cudaError_t e;
+  if (mode == DG_QUANT_ROW_1x128) {
+    const long long strips = static_cast<long long>(rows) * (cols / 128);
+    if (strips >= 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
+    const int grid = static_cast<int>(std::min<long long>((strips + 31) / 32, 8ll * sms));
+    e = bf ? launch(dg::quant_row_kernel<true, true>, dim3(grid), dim3(256), 0, st, 1, x, 1, rows,
+                    cols, q, scales, ld_scales, pk)
+           : launch(dg::quant_row_kernel<false, true>, dim3(grid), dim3(256), 0, st, 1, x, 1, rows,
+                    cols, q, scales, ld_scales, pk);
+  } else {
+    const long long blocks = static_cast<long long>((rows + 127) / 128) * (cols / 128);
+    if (blocks > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
+    e = bf ? launch(dg::quant_block_kernel<true, true>, dim3(static_cast<int>(blocks)), dim3(256),
+                    0, st, 1, x, 1, rows, cols, q, scales, pk)
+           : launch(dg::quant_block_kernel<false, true>, dim3(static_cast<int>(blocks)), dim3(256),
+                    0, st, 1, x, 1, rows, cols, q, scales, pk);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  g_launches.fetch_add(1);
+  return DG_OK;
+}
+
+dg_status dg_fp8_gemm_nt_ue8m0(const void* A, const int32_t* sfa, const void* B,
+                               const int32_t* sfb, const void* C, void* D, int M, int N, int K,
+                               void* stream) {
+  if (M < 0 || N < 0 || K < 0) return DG_ERR_INVALID_ARG;
+  if (K % 128 != 0 || N % 8 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return DG_OK;
+  if (!D) return DG_ERR_INVALID_ARG;
+  if (!aligned16(D) || (C && !aligned16(C))) return DG_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (K == 0) {
+    int dev = 0, sms = 0;
+    dg_status s = device_sms(&dev, &sms);
+    if (s != DG_OK) return s;
+    return copy_or_zero<Bf16Raw>(C, D, static_cast<long long>(M) * N, sms, st);
+  }
+  if (!A || !B || !sfa || !sfb) return DG_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(sfa) || !aligned16(sfb))
+    return DG_ERR_MISALIGNED;
+  return run_mx(A, sfa, B, sfb, C, D, M, N, K, st);
 }
 
 dg_status dg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb,

@@ -115,6 +115,17 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Untiled bulk copy global -> shared of `bytes` bytes (both addresses 16-byte
+// aligned, bytes a multiple of 16), completing on `bar` with complete_tx.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gmem_src)), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
 // Shared -> global tensor store (bulk async group of the issuing thread).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* smem_src, int32_t x,
                                              int32_t y) {
@@ -175,6 +186,30 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uin
           d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(zero)
       : "memory");
+}
+
+// Block-scaled MMA (kind::mxf8f6f4, E4M3 x E4M3 -> F32 with UE8M0 scale
+// factors read from TMEM at sfa_tmem / sfb_tmem; one scale per 32 K-elements,
+// the byte inside each 32-bit TMEM cell chosen by the descriptor's scale ids).
+__device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Shared -> TMEM copy of 32 rows x 128 bits, replicated into all four lane
+// quadrants: smem row i (16 bytes) lands in lanes i, 32+i, 64+i, 96+i of the
+// four 32-bit columns starting at taddr. Issued by one thread; asynchronous,
+// ordered before the thread's later tcgen05.mma, tracked by tcgen05.commit.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
+               : "memory");
 }
 
 // Arrive once on `bar` when every tcgen05.mma this thread issued so far is done.
@@ -375,6 +410,30 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t smem_byte_addr, uin
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;
   return d;
+}
+
+// Shared-memory descriptor of a no-swizzle operand: 8-row x 16-byte core
+// matrices stored contiguously (128 bytes each), `sbo_bytes` apart along the
+// rows (layout type 0 in bits [61,64)).
+__device__ __forceinline__ uint64_t smem_desc_noswz(uint32_t smem_byte_addr, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
+// Instruction descriptor for kind::mxf8f6f4 with block scaling: E4M3 x E4M3
+// -> F32, K-major operands, UE8M0 scale factors (bit 23), scale ids (the byte
+// of each 32-bit TMEM scale cell) for B in bits [4,6) and A in [29,31).
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, uint32_t a_sf_id,
+                                                     uint32_t b_sf_id) {
+  return (b_sf_id << 4)                               // B scale id
+         | (0u << 7) | (0u << 10)                     // A, B format: E4M3
+         | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+         | (1u << 23)                                 // scale format: UE8M0
+         | (static_cast<uint32_t>(M >> 4) << 24)      // M / 16
+         | (a_sf_id << 29);                           // A scale id
 }
 
 // Instruction descriptor for kind::f8f6f4, E4M3 x E4M3 -> F32, dense.

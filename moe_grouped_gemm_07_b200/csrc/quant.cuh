@@ -64,6 +64,31 @@ __device__ __forceinline__ float scale_from_amax(float amax) {
   return quotient(fmaxf(amax, 1e-4f), 448.0f, kInv448);
 }
 
+// Power-of-two scale for the UE8M0 variant: s = 2^e with e = ceil(log2 t),
+// t = max(amax, 1e-4f) / 448 (the FP32 mode's quotient, rounded up to the
+// next power of two so that no code saturates). t is normal (>= 2^-22), so e
+// is its exponent, plus one unless its mantissa is zero. Returns e.
+__device__ __forceinline__ int pow2_exponent(float amax) {
+  const uint32_t b = __float_as_uint(scale_from_amax(amax));
+  const int e = static_cast<int>((b >> 23) & 0xFFu) - 127;
+  return (b & 0x7FFFFFu) ? e + 1 : e;
+}
+
+// 2^e as a float, for -126 <= e <= 127.
+__device__ __forceinline__ float exp2_exact(int e) {
+  return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+}
+
+// Byte offset of (row, K-block) in the packed UE8M0 layout
+// [ceil(K/512)][ceil(R/128)][32][4] int32 (byte b of word [q][rb][i][j] is row
+// 128 rb + 32 j + i, K-block 4 q + b).
+__device__ __forceinline__ long long packed_offset(int row, int kb, int rblocks) {
+  const long long word =
+      ((static_cast<long long>(kb >> 2) * rblocks + (row >> 7)) * 32 + (row & 31)) * 4 +
+      ((row >> 5) & 3);
+  return word * 4 + (kb & 3);
+}
+
 // Four E4M3 codes packed little-endian (element 0 in the low byte).
 __device__ __forceinline__ uint32_t encode4(const float (&v)[4], float s, float r) {
   const float y0 = quotient(v[0], s, r), y1 = quotient(v[1], s, r);
@@ -84,11 +109,14 @@ __device__ __forceinline__ float warp_max(float v) {
 // takes 4 consecutive strips per step (2 KB of input in flight per warp); the
 // (row, strip) position of the first one is found with one 32-bit division per
 // step and advanced incrementally. Requires batch * rows * (cols/128) < 2^31.
-template <bool BF16>
+// POW2: power-of-two scales (see pow2_exponent); the UE8M0 bytes also go to
+// `packed` (batch 1) and `scales` may be null.
+template <bool BF16, bool POW2 = false>
 __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__ x, int batch,
                                                         int rows, int cols,
                                                         uint8_t* __restrict__ codes,
-                                                        float* __restrict__ scales, int ld) {
+                                                        float* __restrict__ scales, int ld,
+                                                        uint8_t* __restrict__ packed) {
   constexpr int U = 4;
   pdl_wait();
   pdl_trigger();
@@ -111,14 +139,25 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
       float amax = fmaxf(fmaxf(fabsf(in[u].v[0]), fabsf(in[u].v[1])),
                          fmaxf(fabsf(in[u].v[2]), fabsf(in[u].v[3])));
       amax = warp_max(amax);
-      const float sc = scale_from_amax(amax);
-      const float rc = __frcp_rn(sc);
+      float sc, rc;
+      int e = 0;
+      if constexpr (POW2) {
+        e = pow2_exponent(amax);
+        sc = exp2_exact(e);
+        rc = exp2_exact(-e);  // exact: the quotient below is then x * 2^-e
+      } else {
+        sc = scale_from_amax(amax);
+        rc = __frcp_rn(sc);
+      }
       *reinterpret_cast<uint32_t*>(codes + static_cast<int64_t>(st) * 128 + (lane << 2)) =
           encode4(in[u].v, sc, rc);
       if (lane == 0) {
         const uint32_t b = br / static_cast<uint32_t>(rows);
         const uint32_t r = br - b * static_cast<uint32_t>(rows);
-        scales[(static_cast<int64_t>(b) * kbs + kb) * ld + r] = sc;
+        if (!POW2 || scales) scales[(static_cast<int64_t>(b) * kbs + kb) * ld + r] = sc;
+        if constexpr (POW2)
+          packed[packed_offset(static_cast<int>(r), static_cast<int>(kb), (rows + 127) >> 7)] =
+              static_cast<uint8_t>(e + 127);
       }
       if (++kb == kbs) { kb = 0; ++br; }
     }
@@ -127,11 +166,14 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
 
 // BLOCK_128x128: one 256-thread CTA per 128x128 block; warp w holds rows
 // [16w, 16w+16) of the block, lane l columns [4l, 4l+4).
-template <bool BF16>
+// POW2: power-of-two scales; the block's UE8M0 byte is written for all 128
+// rows of the block into `packed` (batch 1), and `scales` may be null.
+template <bool BF16, bool POW2 = false>
 __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict__ x, int batch,
                                                           int rows, int cols,
                                                           uint8_t* __restrict__ codes,
-                                                          float* __restrict__ scales) {
+                                                          float* __restrict__ scales,
+                                                          uint8_t* __restrict__ packed) {
   __shared__ float red[8];
   pdl_wait();
   pdl_trigger();
@@ -158,8 +200,16 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
   float a = red[0];
 #pragma unroll
   for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
-  const float sc = scale_from_amax(a);
-  const float rc = __frcp_rn(sc);
+  float sc, rc;
+  int e = 0;
+  if constexpr (POW2) {
+    e = pow2_exponent(a);
+    sc = exp2_exact(e);
+    rc = exp2_exact(-e);
+  } else {
+    sc = scale_from_amax(a);
+    rc = __frcp_rn(sc);
+  }
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int r = (nb << 7) + (w << 4) + i;
@@ -167,7 +217,12 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
       *reinterpret_cast<uint32_t*>(codes + (b * rows + r) * cols + (kb << 7) + (lane << 2)) =
           encode4(v[i].v, sc, rc);
   }
-  if (threadIdx.x == 0) scales[(b * nbs + nb) * kbs + kb] = sc;
+  if (threadIdx.x == 0 && (!POW2 || scales)) scales[(b * nbs + nb) * kbs + kb] = sc;
+  if constexpr (POW2) {
+    if (threadIdx.x < 128)
+      packed[packed_offset((nb << 7) + static_cast<int>(threadIdx.x), kb, nbs)] =
+          static_cast<uint8_t>(e + 127);
+  }
 }
 
 // COL_128x1: one 256-thread CTA per (batch, 128-row strip, 64-column slab);

@@ -16,6 +16,7 @@ import numpy as np
 from . import build as _build
 
 ROW_1x128, BLOCK_128x128, COL_128x1 = 0, 1, 2
+ROW_1x128_POW2, BLOCK_128x128_POW2 = 3, 4  # power-of-two (UE8M0) scales
 C_NONE, C_BF16, C_F32 = 0, 1, 2
 
 _lib = None
@@ -95,10 +96,10 @@ def quantize(x: np.ndarray, mode: int, ld_scales: int | None = None, bf16: bool 
     if squeeze:
         x = x[None]
     batch, rows, cols = x.shape
-    if mode == ROW_1x128:
+    if mode in (ROW_1x128, ROW_1x128_POW2):
         ld = ld_scales if ld_scales is not None else sf_rows_ld(rows)
         scales = np.zeros((batch, cols // 128, ld), dtype=np.float32)
-    elif mode == BLOCK_128x128:
+    elif mode in (BLOCK_128x128, BLOCK_128x128_POW2):
         ld = 0
         scales = np.zeros((batch, (rows + 127) // 128, cols // 128), dtype=np.float32)
     elif mode == COL_128x1:

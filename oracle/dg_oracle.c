@@ -79,9 +79,21 @@ static float scale_of(float amax) {
   return a / 448.0f;
 }
 
+/* Power-of-two variant: the smallest power of two >= the FP32 scale above,
+ * i.e. 2^ceil(log2 t). frexpf gives t = m * 2^ex with 0.5 <= m < 1, so t is
+ * itself a power of two exactly when m == 0.5. */
+static float pow2_scale_of(float amax) {
+  float t = scale_of(amax);
+  int ex = 0;
+  float m = frexpf(t, &ex);
+  return ldexpf(1.0f, m == 0.5f ? ex - 1 : ex);
+}
+
 int dgo_quantize(const void* x, int in_is_bf16, int batch, int rows, int cols,
                  int mode, uint8_t* codes, float* scales, int ld_scales) {
   if (batch < 0 || rows < 0 || cols < 0) return -1;
+  int pow2 = mode == DGO_ROW_1x128_POW2 || mode == DGO_BLOCK_128x128_POW2;
+  if (pow2) mode -= DGO_ROW_1x128_POW2;  /* same loops, power-of-two scales */
   if (mode == DGO_ROW_1x128) {
     if (cols % 128 != 0 || ld_scales < rows) return -1;
     int kbs = cols / 128;
@@ -95,7 +107,7 @@ int dgo_quantize(const void* x, int in_is_bf16, int batch, int rows, int cols,
             float v = fabsf(load_x(x, in_is_bf16, base + j));
             if (v > amax) amax = v;
           }
-          float s = scale_of(amax);
+          float s = pow2 ? pow2_scale_of(amax) : scale_of(amax);
           scales[((size_t)b * kbs + kb) * ld_scales + r] = s;
           for (int j = 0; j < 128; ++j) {
             float y = load_x(x, in_is_bf16, base + j) / s;
@@ -120,7 +132,7 @@ int dgo_quantize(const void* x, int in_is_bf16, int batch, int rows, int cols,
               float v = fabsf(load_x(x, in_is_bf16, ((size_t)b * rows + r) * cols + kb * 128 + j));
               if (v > amax) amax = v;
             }
-          float s = scale_of(amax);
+          float s = pow2 ? pow2_scale_of(amax) : scale_of(amax);
           scales[((size_t)b * nbs + nb) * kbs + kb] = s;
           for (int r = r0; r < r1; ++r)
             for (int j = 0; j < 128; ++j) {

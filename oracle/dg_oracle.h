@@ -42,6 +42,12 @@ float dgo_bf16_to_f32(uint16_t bits);
 
 /* Quantisation modes (same numbering as the library ABI, re-declared here). */
 enum { DGO_ROW_1x128 = 0, DGO_BLOCK_128x128 = 1, DGO_COL_128x1 = 2 };
+/* Power-of-two (UE8M0) variants of ROW and BLOCK: the scale is rounded up to
+ * the next power of two, s = 2^ceil(log2(max(amax, 1e-4f) / 448)), so that it
+ * is exactly representable as a UE8M0 byte (the README summary's packed UE8M0
+ * scales, "GEMMインターフェースとレイアウト制約") and no code saturates. Same
+ * scale layouts as ROW / BLOCK. */
+enum { DGO_ROW_1x128_POW2 = 3, DGO_BLOCK_128x128_POW2 = 4 };
 
 /*
  * Quantise x[batch][rows][cols] (float if in_is_bf16 == 0, bf16 bits

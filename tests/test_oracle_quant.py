@@ -150,3 +150,61 @@ def test_batched_layout_equals_per_batch():
     for b in range(3):
         cb, sb = oracle.quantize(x[b], oracle.ROW_1x128)
         assert np.array_equal(c[b], cb) and np.array_equal(s[b], sb)
+
+
+# ------------------------------------------------------------ power-of-two (UE8M0) scales
+def _strip_amax_rows(x):
+    rows, cols = x.shape
+    return np.abs(x).reshape(rows, cols // 128, 128).max(axis=2)
+
+
+def test_pow2_row_scales_are_the_next_power_of_two():
+    """s is a power of two with s/2 < t <= s for t = max(amax, 1e-4)/448 in
+    float32 (closed form, checked with numpy's frexp, independent of the
+    oracle's own rounding step)."""
+    x = synth.normal((70, 512), synth.seed(9, 1, 0)) * F32(3.0)
+    x[5, 128:256] = 0.0                        # floor strip
+    x[6, :128] = 0.0
+    x[6, 7] = 448.0                            # t == 1 exactly -> s == 1
+    x[7, :128] = 0.0
+    x[7, 3] = -449.0                           # t just above 1 -> s == 2
+    codes, s = oracle.quantize(x, oracle.ROW_1x128_POW2)
+    s = s[:, :70].T                            # [rows, kbs]
+    t = np.maximum(_strip_amax_rows(x), F32(1e-4)).astype(F32) / F32(448.0)
+    m, _ = np.frexp(s)
+    assert np.all(m == 0.5)
+    assert np.all(s >= t) and np.all(s / 2 < t)
+    assert s[6, 0] == 1.0 and s[7, 0] == 2.0
+
+
+def test_pow2_codes_equal_torch_cast_of_exact_quotient():
+    """With s a power of two, x / s is exact, and |x / s| <= 448: the codes
+    must equal torch's float8_e4m3fn cast (library routine) of x / s."""
+    x = synth.normal((33, 384), synth.seed(9, 2, 0)) * F32(50.0)
+    codes, s = oracle.quantize(x, oracle.ROW_1x128_POW2)
+    sf = np.repeat(s[:, :33].T, 128, axis=1)   # [rows, cols]
+    y = (x / sf).astype(F32)
+    assert np.all(np.abs(y) <= 448.0)
+    assert np.array_equal(codes, torch_e4m3(y))
+
+
+def test_pow2_block_scales_ragged():
+    rows, cols = 200, 256                      # 2 row blocks, the second has 72 rows
+    x = synth.normal((rows, cols), synth.seed(9, 3, 0))
+    codes, s = oracle.quantize(x, oracle.BLOCK_128x128_POW2)
+    for nb in range(2):
+        for kb in range(2):
+            blk = x[nb * 128:(nb + 1) * 128, kb * 128:(kb + 1) * 128]
+            t = F32(max(np.abs(blk).max(), F32(1e-4))) / F32(448.0)
+            v = s[nb, kb]
+            assert np.frexp(v)[0] == 0.5 and v >= t and v / 2 < t
+            y = (blk / v).astype(F32)
+            assert np.array_equal(codes[nb * 128:(nb + 1) * 128, kb * 128:(kb + 1) * 128],
+                                  torch_e4m3(y))
+
+
+def test_pow2_scales_dequantise_within_bound():
+    x = synth.normal((64, 256), synth.seed(9, 4, 0))
+    codes, s = oracle.quantize(x, oracle.ROW_1x128_POW2)
+    sf = np.repeat(s[:, :64].T, 128, axis=1)
+    assert dequant_err_ok(x, codes, sf)
