@@ -354,6 +354,93 @@ def run_grouped(args):
     return 0
 
 
+# ----------------------------------------------------------------- UE8M0 comparison
+def run_ue8m0(args):
+    """--workload ue8m0: the dense sweep with power-of-two scales, timing the
+    two GEMM paths on the same quantised inputs: explicit promotion
+    (dg_fp8_gemm_nt, FP32 copies of the scales) and the tensor core's
+    block-scaled MMA (dg_fp8_gemm_nt_ue8m0, packed UE8M0). One step = per
+    shape, quantise A (power-of-two 1x128) + the block-scaled GEMM; L2 flushed
+    before every shape as in the main line. One GPU."""
+    import torch
+    import moe_grouped_gemm_07_b200 as dg
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops"]
+    shapes = wl.dense_shapes()
+    if args.shape:
+        shapes = [tuple(int(x) for x in sh.split(",")) for sh in args.shape.split(";") if sh]
+    weights, acts, outs, qbufs = {}, [], [], []
+    for (N, K) in sorted(set((s_[1], s_[2]) for s_ in shapes)):
+        B = torch.from_numpy(synth.normal((N, K), synth.seed(2, nk_index(N, K), 1))).to(dev)
+        weights[(N, K)] = dg.dg_quantize_fp8_ue8m0(B, dg.DG_QUANT_BLOCK_128x128)
+        del B
+    for (M, N, K) in shapes:
+        A = torch.from_numpy(synth.normal((M, K), synth.seed(2, shape_index(M, N, K), 0))).to(dev)
+        acts.append(A)
+        outs.append(torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+        qbufs.append(dg.dg_quantize_fp8_ue8m0(A, dg.DG_QUANT_ROW_1x128))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    n = len(shapes)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+
+    def run(kind, record):
+        for i, (M, N, K) in enumerate(shapes):
+            flush.fill_(i & 0xFF)
+            torch.cuda._sleep(100_000)
+            qa, sa, pa = qbufs[i]
+            qb, sb, pb = weights[(N, K)]
+            if record:
+                ev[i][0].record()
+            if kind == "step":
+                dg.dg_quantize_fp8_ue8m0(acts[i], dg.DG_QUANT_ROW_1x128, codes=qa, scales=sa,
+                                         packed=pa)
+                dg.dg_fp8_gemm_nt_ue8m0(qa, pa, qb, pb, None, outs[i])
+            elif kind == "mx":
+                dg.dg_fp8_gemm_nt_ue8m0(qa, pa, qb, pb, None, outs[i])
+            else:
+                dg.dg_fp8_gemm_nt(qa, sa, qb, sb, None, outs[i])
+            if record:
+                ev[i][1].record()
+
+    res = {}
+    for kind in ("step", "mx", "promotion"):
+        for _ in range(max(args.warmup, 3)):
+            run(kind, False)
+        torch.cuda.synchronize()
+        t = np.zeros(n)
+        for _ in range(args.steps):
+            run(kind, True)
+            torch.cuda.synchronize()
+            for i in range(n):
+                t[i] += ev[i][0].elapsed_time(ev[i][1])
+        res[kind] = t / args.steps
+    flops = [shape_flops(*sh) for sh in shapes]
+    big = max(range(n), key=lambda i: flops[i])
+    per = [{"M": M, "N": N, "K": K, "mx_us": round(res["mx"][i] * 1e3, 2),
+            "promotion_us": round(res["promotion"][i] * 1e3, 2),
+            "mx_tflops": round(flops[i] / (res["mx"][i] * 1e-3) / 1e12, 1),
+            "promotion_tflops": round(flops[i] / (res["promotion"][i] * 1e-3) / 1e12, 1)}
+           for i, (M, N, K) in enumerate(shapes)]
+    ach = flops[big] / (res["mx"][big] * 1e-3) / 1e12
+    line = {"metric": METRIC, "workload": "dense_fp8_gemm_nt_sweep_ue8m0",
+            "value": round(sum(flops) / (res["step"].sum() * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(float(res["step"].sum()), 4), "steps": args.steps,
+            "higher_is_better": True, "dtype": "e4m3 x e4m3 (UE8M0 scales) -> f32 accumulate, bf16 out",
+            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
+                         "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4),
+                         "kernel": f"gemm_mx_kernel:{shapes[big][0]}x{shapes[big][1]}x{shapes[big][2]}"},
+            "promotion_path_same_scales_tflops": round(
+                sum(flops) / (res["promotion"].sum() * 1e-3) / 1e12, 2),
+            "mx_path_gemm_only_tflops": round(sum(flops) / (res["mx"].sum() * 1e-3) / 1e12, 2),
+            "shapes": per}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -592,7 +679,7 @@ def main():
     ap.add_argument("--quick", action="store_true",
                     help="timed device loop only: no e2e leg, CPU baseline or clock sampling")
     ap.add_argument("--workload", default="dense",
-                    choices=["dense", "contiguous", "masked", "kgrouped"],
+                    choices=["dense", "contiguous", "masked", "kgrouped", "ue8m0"],
                     help="dense (the bench line) or one MoE variant at its benchmark size")
     ap.add_argument("--masked-index", type=int, default=0,
                     help="masked workload: index into the (N, K) pairs")
@@ -601,6 +688,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "ue8m0":
+        return run_ue8m0(args)
     if args.workload != "dense":
         return run_grouped(args)
     return run_ours(args)
