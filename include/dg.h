@@ -95,6 +95,30 @@ dg_status dg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const f
                          const void* C, void* D, int M, int N, int K, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Dense GEMM with the other operand layouts (README summary, "GEMMインター
+ * フェースとレイアウト制約": NT is the base layout, NN / TN / TT are offered
+ * besides). Same operation and scale granularity as dg_fp8_gemm_nt; the
+ * letters are named as NT is: A [M][K] = N, A [K][M] = T; B [N][K] = T (as
+ * in D = A @ B.T), B [K][N] = N:
+ *   NN  A [M][K], sfa [K/128][align4(M)];  B [K][N], sfb [K/128][ceil(N/128)]
+ *   TN  A [K][M], sfa [K/128][M];          B [K][N], sfb [K/128][ceil(N/128)]
+ *   TT  A [K][M], sfa [K/128][M];          B [N][K], sfb [ceil(N/128)][K/128]
+ * (the quantiser's COL_128x1 mode on A [K][M] and BLOCK_128x128 mode on
+ * B [K][N] produce exactly these scale layouts). C / D [M][N] BF16 as NT.
+ * K % 128 == 0, N % 8 == 0; M % 16 == 0 when A is [K][M]; N % 16 == 0 when
+ * B is [K][N]. The small-M (decode) strategy is NT-only: these run the
+ * persistent kernel for every M.
+ * A dense weight gradient (dW = dY^T X, both operands K-outer, FP32 output,
+ * accumulation onto C) is dg_k_grouped_fp8_gemm_tn_contiguous with G = 1.
+ * ------------------------------------------------------------------------- */
+dg_status dg_fp8_gemm_nn(const void* A, const float* sfa, const void* B, const float* sfb,
+                         const void* C, void* D, int M, int N, int K, void* stream);
+dg_status dg_fp8_gemm_tn(const void* A, const float* sfa, const void* B, const float* sfb,
+                         const void* C, void* D, int M, int N, int K, void* stream);
+dg_status dg_fp8_gemm_tt(const void* A, const float* sfa, const void* B, const float* sfb,
+                         const void* C, void* D, int M, int N, int K, void* stream);
+
+/* ---------------------------------------------------------------------------
  * M-grouped GEMM, contiguous layout (MoE prefill / training forward).
  * Source: README summary, section "DenseとGrouped GEMM": experts share N and K;
  * each expert's tokens are concatenated along M, each segment aligned to the

@@ -43,7 +43,8 @@ EXPORTED = (
     "dg_get_tma_aligned_size", "dg_set_num_sms", "dg_get_num_sms", "dg_set_wait_timeout_ns",
     "dg_get_last_device_error", "dg_debug_drop_next_arrive", "dg_get_launch_count",
     "dg_set_pdl", "dg_get_pdl", "dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks",
-    "dg_quantize_fp8_ue8m0", "dg_fp8_gemm_nt_ue8m0",
+    "dg_quantize_fp8_ue8m0", "dg_fp8_gemm_nt_ue8m0", "dg_fp8_gemm_nn", "dg_fp8_gemm_tn",
+    "dg_fp8_gemm_tt",
 )
 
 _vp, _i32 = _C.c_void_p, _C.c_int
@@ -61,6 +62,9 @@ _lib.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks.argtypes = [_vp, _vp, _vp, _vp, 
                                                             _vp, _i32, _i32, _i32, _vp]
 _lib.dg_quantize_fp8_ue8m0.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp]
 _lib.dg_fp8_gemm_nt_ue8m0.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]
+for _f in ("dg_fp8_gemm_nn", "dg_fp8_gemm_tn", "dg_fp8_gemm_tt"):
+    getattr(_lib, _f).argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]
+    getattr(_lib, _f).restype = _i32
 for _f in ("dg_quantize_fp8", "dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
            "dg_m_grouped_fp8_gemm_nt_masked", "dg_k_grouped_fp8_gemm_tn_contiguous",
            "dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks", "dg_quantize_fp8_ue8m0",
@@ -233,6 +237,37 @@ def dg_k_grouped_fp8_gemm_tn_contiguous(A, sfa, B, sfb, ks, C, D, stream=None):
            _lib.dg_k_grouped_fp8_gemm_tn_contiguous(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), ks_arr,
                                                     _ptr(C), _ptr(D), G, M, N, _stream(stream)))
     return D
+
+
+def _dense_layout(name, a_mn, b_mn, A, sfa, B, sfb, C, D, stream):
+    _cuda_contig(A, sfa, B, sfb, C, D)
+    _need(_is_fp8(A) and _is_fp8(B), "A/B must be E4M3 bytes")
+    K, M = A.shape if a_mn else A.shape[::-1]
+    N = B.shape[1] if b_mn else B.shape[0]
+    _need((B.shape[0] if b_mn else B.shape[1]) == K, "A/B K mismatch")
+    _need(D.dtype == torch.bfloat16 and tuple(D.shape) == (M, N), "D must be bf16 [M, N]")
+    _need(C is None or (C.dtype == torch.bfloat16 and tuple(C.shape) == (M, N)), "C")
+    _need(sfa.dtype == torch.float32 and sfa.numel() >= (K // 128) * (M if a_mn else align4(M)),
+          "sfa")
+    _need(sfb.dtype == torch.float32 and sfb.numel() >= (K // 128) * ((N + 127) // 128), "sfb")
+    _check(name, getattr(_lib, name)(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(C), _ptr(D),
+                                     M, N, K, _stream(stream)))
+    return D
+
+
+def dg_fp8_gemm_nn(A, sfa, B, sfb, C, D, stream=None):
+    """A [M, K], sfa [K/128, align4(M)]; B [K, N], sfb [K/128, ceil(N/128)]."""
+    return _dense_layout("dg_fp8_gemm_nn", False, True, A, sfa, B, sfb, C, D, stream)
+
+
+def dg_fp8_gemm_tn(A, sfa, B, sfb, C, D, stream=None):
+    """A [K, M], sfa [K/128, M]; B [K, N], sfb [K/128, ceil(N/128)]."""
+    return _dense_layout("dg_fp8_gemm_tn", True, True, A, sfa, B, sfb, C, D, stream)
+
+
+def dg_fp8_gemm_tt(A, sfa, B, sfb, C, D, stream=None):
+    """A [K, M], sfa [K/128, M]; B [N, K], sfb [ceil(N/128), K/128]."""
+    return _dense_layout("dg_fp8_gemm_tt", True, False, A, sfa, B, sfb, C, D, stream)
 
 
 def ue8m0_packed_shape(rows: int, cols: int):

@@ -260,6 +260,95 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
   return launch_gemm<MODE, 128>(ta, tb, dummy, dummy, td, args, grid, st, dev);
 }
 
+// Dense GEMM with A and/or B stored MN-major (NN, TN, TT); 128 x 256 tiles.
+template <int MODE>
+dg_status run_layout(const void* A, const float* sfa, int ld_sfa, const void* B, const float* sfb,
+                     const void* C, void* D, int M, int N, int K, cudaStream_t st,
+                     const char* name) {
+  using Cfg = dg::GemmCfg<MODE, 256>;
+  int dev = 0, sms = 0;
+  dg_status s = device_sms(&dev, &sms);
+  if (s != DG_OK) return s;
+  CUtensorMap ta, tb, td, dummy;
+  std::memset(&dummy, 0, sizeof dummy);
+  if (Cfg::A_MN)  // A stored [K][M]: 128 x 128 boxes, x along M
+    s = make_map_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, M, K, M, 128, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    s = make_map_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != DG_OK) return s;
+  if (Cfg::B_MN)  // B stored [K][N]: two 128 x 128 boxes per tile, x along N
+    s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, N, 128, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, 128, 256,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != DG_OK) return s;
+  s = make_map_2d(&td, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, 2ull * N, 32, 32,
+                  CU_TENSOR_MAP_SWIZZLE_64B);
+  if (s != DG_OK) return s;
+  GemmArgs args;
+  std::memset(&args, 0, sizeof args);
+  args.M = M;
+  args.N = N;
+  args.K = K;
+  args.G = 1;
+  args.d_rows = M;
+  args.num_m_blocks = (M + 127) / 128;
+  args.num_n_blocks = (N + 255) / 256;
+  const long long tiles = static_cast<long long>(args.num_m_blocks) * args.num_n_blocks;
+  if (tiles > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
+  args.total_tiles = static_cast<int>(tiles);
+  args.sfa = sfa;
+  args.ld_sfa = ld_sfa;
+  args.sfb = sfb;
+  args.C = C;
+  args.D = D;
+  args.timeout_ns = timeout_ns();
+  args.drop_arrive = take_drop_flag();
+  const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(sms, tiles)));
+  if (print_configs())
+    std::fprintf(stderr, "[dg] %s M=%d N=%d K=%d: BM=128 BN=256 tiles=%lld grid=%d\n", name, M, N,
+                 K, tiles, grid);
+  return launch_gemm<MODE, 256>(ta, tb, dummy, dummy, td, args, grid, st, dev);
+}
+
+// Shared argument checks of the dense entry points. a_mn / b_mn: the operand
+// is stored MN-major, so its rows of M (N) bytes must be 16-byte multiples.
+dg_status check_dense(const void* A, const void* sfa, const void* B, const void* sfb, const void* C,
+                      void* D, int M, int N, int K, bool a_mn, bool b_mn) {
+  if (M < 0 || N < 0 || K < 0) return DG_ERR_INVALID_ARG;
+  if (K % 128 != 0 || N % 8 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  if ((a_mn && M % 16 != 0) || (b_mn && N % 16 != 0)) return DG_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return DG_OK;
+  if (!D) return DG_ERR_INVALID_ARG;
+  if (!aligned16(D) || (C && !aligned16(C))) return DG_ERR_MISALIGNED;
+  if (K == 0) return DG_OK;
+  if (!A || !B || !sfa || !sfb) return DG_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(sfa) || !aligned16(sfb))
+    return DG_ERR_MISALIGNED;
+  return DG_OK;
+}
+
+template <int MODE>
+dg_status dense_layout_entry(const void* A, const float* sfa, const void* B, const float* sfb,
+                             const void* C, void* D, int M, int N, int K, void* stream,
+                             const char* name) {
+  using Cfg = dg::GemmCfg<MODE, 256>;
+  dg_status s = check_dense(A, sfa, B, sfb, C, D, M, N, K, Cfg::A_MN, Cfg::B_MN);
+  if (s != DG_OK || M == 0 || N == 0) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (K == 0) {
+    int dev = 0, sms = 0;
+    if ((s = device_sms(&dev, &sms)) != DG_OK) return s;
+    return copy_or_zero<Bf16Raw>(C, D, static_cast<long long>(M) * N, sms, st);
+  }
+  // sfa: [K/128][align4(M)] for A stored [M][K], [K/128][M] for A stored [K][M]
+  const int ld = Cfg::A_MN ? M : (M + 3) / 4 * 4;
+  return run_layout<MODE>(A, sfa, ld, B, sfb, C, D, M, N, K, st, name);
+}
+
 // ---------------------------------------------------------------- CTA pairs
 // Dense GEMM with M > 128 on CTA pairs (256 x BN tiles, cta_group::2 MMAs;
 // each CTA loads half of the B tile). Opt-in with DG_PAIR=1: measured on B200
@@ -805,6 +894,21 @@ dg_status dg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const f
   if (use_pairs()) return run_pair(A, sfa, ld, B, sfb, C, D, M, N, K, st);
   return run_nt<dg::MODE_DENSE>(A, sfa, ld, B, sfb, nullptr, nullptr, C, D, M, M, N, K, 1, mb, mb,
                                 st, "fp8_gemm_nt");
+}
+
+dg_status dg_fp8_gemm_nn(const void* A, const float* sfa, const void* B, const float* sfb,
+                         const void* C, void* D, int M, int N, int K, void* stream) {
+  return dense_layout_entry<dg::MODE_NN>(A, sfa, B, sfb, C, D, M, N, K, stream, "fp8_gemm_nn");
+}
+
+dg_status dg_fp8_gemm_tn(const void* A, const float* sfa, const void* B, const float* sfb,
+                         const void* C, void* D, int M, int N, int K, void* stream) {
+  return dense_layout_entry<dg::MODE_TN>(A, sfa, B, sfb, C, D, M, N, K, stream, "fp8_gemm_tn");
+}
+
+dg_status dg_fp8_gemm_tt(const void* A, const float* sfa, const void* B, const float* sfb,
+                         const void* C, void* D, int M, int N, int K, void* stream) {
+  return dense_layout_entry<dg::MODE_TT>(A, sfa, B, sfb, C, D, M, N, K, stream, "fp8_gemm_tt");
 }
 
 dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void* A, const float* sfa, const void* B,

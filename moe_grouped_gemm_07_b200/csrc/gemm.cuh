@@ -36,8 +36,13 @@ namespace dg {
 // 256 x BN tile with tcgen05 cta_group::2 MMAs (each CTA holds 128 rows of A,
 // half of the B tile and the accumulator of its 128 rows): the same operand
 // traffic per SM as a 128 x 2BN single-CTA tile with half the accumulator.
+// MODE_NN / MODE_TN / MODE_TT are the dense GEMM with the other operand
+// layouts, named as NT is: the first letter for A ([M][K] = N, [K][M] = T),
+// the second for B ([N][K] = T, as in D = A @ B.T; [K][N] = N). NN takes B as
+// [K][N], TN takes A as [K][M] and B as [K][N], TT takes A as [K][M].
 enum GemmMode : int {
-  MODE_DENSE = 0, MODE_CONTIG = 1, MODE_MASKED = 2, MODE_KGROUPED = 3, MODE_PAIR = 4
+  MODE_DENSE = 0, MODE_CONTIG = 1, MODE_MASKED = 2, MODE_KGROUPED = 3, MODE_PAIR = 4,
+  MODE_NN = 5, MODE_TN = 6, MODE_TT = 7
 };
 
 constexpr int kMaxKGroups = 256;
@@ -82,6 +87,9 @@ struct GemmCfg {
 
   static constexpr int GROUP_M = 16;       // tile rasterisation group (L2 reuse)
   static constexpr bool KG = MODE == MODE_KGROUPED;
+  // operands stored MN-major (K-outer) in global and shared memory
+  static constexpr bool A_MN = KG || MODE == MODE_TN || MODE == MODE_TT;
+  static constexpr bool B_MN = KG || MODE == MODE_NN || MODE == MODE_TN;
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
@@ -151,7 +159,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int*
     tl.b_row = tl.n0 + rank * (BN / 2);
     tl.rows = min(Cfg::BM, a.M - tl.m0);  // may be <= 0 for the second CTA
     tl.out_row0 = tl.m0;
-  } else if constexpr (MODE == MODE_DENSE || MODE == MODE_CONTIG) {
+  } else if constexpr (MODE == MODE_DENSE || MODE == MODE_CONTIG || MODE >= MODE_NN) {
     const int group_tiles = Cfg::GROUP_M * a.num_n_blocks;
     const int grp = t / group_tiles;
     const int first_m = grp * Cfg::GROUP_M;
@@ -163,7 +171,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int*
     tl.n0 = nb * BN;
     tl.a_row = tl.m0;
     tl.out_row0 = tl.m0;
-    if constexpr (MODE == MODE_DENSE) {
+    if constexpr (MODE != MODE_CONTIG) {
       tl.g = 0;
       tl.b_row = tl.n0;
       tl.rows = min(Cfg::BM, a.M - tl.m0);
@@ -429,14 +437,17 @@ __global__ void __launch_bounds__(320, 1)
             } else {
               mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES);
               const int kk = (tl.kb0 + kb) * Cfg::BK;
-              if constexpr (Cfg::KG) {
+              // MN-major operands: 128-element-wide boxes of BK K-rows (x = MN)
+              if constexpr (Cfg::A_MN)
                 tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], tl.a_row, kk);
+              else
+                tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], kk, tl.a_row);
+              if constexpr (Cfg::B_MN) {
 #pragma unroll
                 for (int h = 0; h < BN / 128; ++h)
                   tma_load_2d(sB + s * Cfg::B_BYTES + h * 128 * Cfg::BK, &tm_b, &full[s],
                               tl.b_row + h * 128, kk);
               } else {
-                tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], kk, tl.a_row);
                 tma_load_2d(sB + s * Cfg::B_BYTES, &tm_b, &full[s], kk, tl.b_row);
               }
             }
@@ -482,7 +493,7 @@ __global__ void __launch_bounds__(320, 1)
     // same work in a converged warp does not.
     if (leader) {
       constexpr uint32_t idesc =
-          idesc_e4m3_f32(PAIR ? 2 * Cfg::BM : Cfg::BM, BN, Cfg::KG ? 1 : 0, Cfg::KG ? 1 : 0);
+          idesc_e4m3_f32(PAIR ? 2 * Cfg::BM : Cfg::BM, BN, Cfg::A_MN ? 1 : 0, Cfg::B_MN ? 1 : 0);
       uint32_t s = 0, full_ph = 0, b = 0, tmem_ph = 0;
       for (int t = cta_first; t < total_tiles; t += cta_step) {
         const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped, rank);
@@ -500,16 +511,14 @@ __global__ void __launch_bounds__(320, 1)
             const uint32_t d_tmem = tmem_base + b * BN;
 #pragma unroll
             for (int k = 0; k < Cfg::BK / 32; ++k) {
-              uint64_t da, db;
-              if constexpr (Cfg::KG) {
-                // MN-major: 32 K-rows of 128 bytes per MMA; MN atoms 16 KB apart.
-                da = smem_desc_sw128(a_base + k * 32 * 128, 128 * Cfg::BK, 1024);
-                db = smem_desc_sw128(b_base + k * 32 * 128, 128 * Cfg::BK, 1024);
-              } else {
-                // K-major: 32 bytes of K per MMA inside the 128-byte swizzle row.
-                da = smem_desc_sw128(a_base + k * 32, 16, 1024);
-                db = smem_desc_sw128(b_base + k * 32, 16, 1024);
-              }
+              // MN-major: 32 K-rows of 128 bytes per MMA; MN atoms 16 KB apart.
+              // K-major: 32 bytes of K per MMA inside the 128-byte swizzle row.
+              const uint64_t da = Cfg::A_MN
+                                      ? smem_desc_sw128(a_base + k * 32 * 128, 128 * Cfg::BK, 1024)
+                                      : smem_desc_sw128(a_base + k * 32, 16, 1024);
+              const uint64_t db = Cfg::B_MN
+                                      ? smem_desc_sw128(b_base + k * 32 * 128, 128 * Cfg::BK, 1024)
+                                      : smem_desc_sw128(b_base + k * 32, 16, 1024);
               if constexpr (PAIR)
                 mma_f8f6f4_pair(d_tmem, da, db, idesc, k > 0 ? 1u : 0u);
               else
@@ -574,7 +583,9 @@ __global__ void __launch_bounds__(320, 1)
           pa = args.sfa + m_local;
         const int col_first = tl.n0 + static_cast<int>(h) * EC;
         half_in = col_first < args.N;
-        pb = args.sfb + (static_cast<long long>(tl.g) * nbN + col_first / 128) * KBn;
+        // sfb is [G][ceil(N/128)][K/128], or [K/128][ceil(N/128)] for B stored [K][N]
+        pb = Cfg::B_MN ? args.sfb + col_first / 128
+                       : args.sfb + (static_cast<long long>(tl.g) * nbN + col_first / 128) * KBn;
       }
       // NT scales stream through this warp's shared-memory ring by cp.async,
       // SRING K-blocks ahead: lane l copies sfa for its row, lane 0 also the
@@ -586,7 +597,8 @@ __global__ void __launch_bounds__(320, 1)
         if (kb < tl.nkb) {
           float* slot = ring + (kb % SR) * 33;
           if (row_in) cp_async_4(slot + lane, pa + static_cast<long long>(kb) * args.ld_sfa);
-          if (lane == 0 && half_in) cp_async_4(slot + 32, pb + kb);
+          if (lane == 0 && half_in)
+            cp_async_4(slot + 32, pb + (Cfg::B_MN ? static_cast<long long>(kb) * nbN : kb));
         }
         cp_async_commit();
       };
