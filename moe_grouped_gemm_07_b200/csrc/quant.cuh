@@ -104,11 +104,40 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// 16 consecutive inputs starting at element i (i a multiple of 16).
+template <bool BF16>
+__device__ __forceinline__ void load16(const void* x, int64_t i, float (&v)[16]) {
+  if constexpr (BF16) {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + i);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4 u = __ldg(p + h);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[h * 8 + 2 * k] = __uint_as_float(w[k] << 16);
+        v[h * 8 + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+      }
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + i);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float4 f = __ldg(p + h);
+      v[4 * h] = f.x;
+      v[4 * h + 1] = f.y;
+      v[4 * h + 2] = f.z;
+      v[4 * h + 3] = f.w;
+    }
+  }
+}
+
 // ROW_1x128: strips enumerated (batch, row, strip) with the strip index
-// fastest, so strip s covers elements [128 s, 128 s + 128) of x. Each warp
-// takes 4 consecutive strips per step (2 KB of input in flight per warp); the
-// (row, strip) position of the first one is found with one 32-bit division per
-// step and advanced incrementally. Requires batch * rows * (cols/128) < 2^31.
+// fastest, so strip s covers elements [128 s, 128 s + 128) of x. Eight lanes
+// share a strip, each holding 16 consecutive values (the strip's amax takes 3
+// shuffles, its 128 codes go out as 8 x 16-byte stores); a warp covers 4
+// strips per round and keeps 2 rounds (8 strips, 4 KB of FP32 input) in
+// flight. Requires batch * rows * (cols/128) < 2^31.
 // POW2: power-of-two scales (see pow2_exponent); the UE8M0 bytes also go to
 // `packed` (batch 1) and `scales` may be null.
 template <bool BF16, bool POW2 = false>
@@ -117,28 +146,37 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
                                                         uint8_t* __restrict__ codes,
                                                         float* __restrict__ scales, int ld,
                                                         uint8_t* __restrict__ packed) {
-  constexpr int U = 4;
+  constexpr int U = 2;  // rounds of 4 strips in flight per warp
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
+  const int g = lane >> 3;   // strip of this lane within a round
+  const int li = lane & 7;   // 16-value slice of the strip
   const uint32_t kbs = static_cast<uint32_t>(cols) >> 7;
   const uint32_t nstrips = static_cast<uint32_t>(batch) * static_cast<uint32_t>(rows) * kbs;
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
   const uint32_t warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  for (uint32_t s0 = warp0 * U; s0 < nstrips; s0 += nwarps * U) {
-    In4 in[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-      if (s0 + u < nstrips) in[u] = load4<BF16>(x, (static_cast<int64_t>(s0) + u) * 128 + (lane << 2));
-    uint32_t br = s0 / kbs;            // batch * rows + row of strip s0
-    uint32_t kb = s0 - br * kbs;
+  for (uint32_t s0 = warp0 * (4 * U); s0 < nstrips; s0 += nwarps * (4 * U)) {
+    float v[U][16];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const uint32_t st = s0 + u;
-      if (st >= nstrips) break;
-      float amax = fmaxf(fmaxf(fabsf(in[u].v[0]), fabsf(in[u].v[1])),
-                         fmaxf(fabsf(in[u].v[2]), fabsf(in[u].v[3])));
-      amax = warp_max(amax);
+      const uint32_t st = s0 + 4 * u + g;
+      if (st < nstrips) {
+        load16<BF16>(x, static_cast<int64_t>(st) * 128 + li * 16, v[u]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[u][k] = 0.0f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t st = s0 + 4 * u + g;
+      float amax = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(v[u][k]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
       float sc, rc;
       int e = 0;
       if constexpr (POW2) {
@@ -149,17 +187,24 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
         sc = scale_from_amax(amax);
         rc = __frcp_rn(sc);
       }
-      *reinterpret_cast<uint32_t*>(codes + static_cast<int64_t>(st) * 128 + (lane << 2)) =
-          encode4(in[u].v, sc, rc);
-      if (lane == 0) {
-        const uint32_t b = br / static_cast<uint32_t>(rows);
-        const uint32_t r = br - b * static_cast<uint32_t>(rows);
-        if (!POW2 || scales) scales[(static_cast<int64_t>(b) * kbs + kb) * ld + r] = sc;
-        if constexpr (POW2)
-          packed[packed_offset(static_cast<int>(r), static_cast<int>(kb), (rows + 127) >> 7)] =
-              static_cast<uint8_t>(e + 127);
+      if (st < nstrips) {
+        uint4 o;
+        o.x = encode4(*reinterpret_cast<const float(*)[4]>(&v[u][0]), sc, rc);
+        o.y = encode4(*reinterpret_cast<const float(*)[4]>(&v[u][4]), sc, rc);
+        o.z = encode4(*reinterpret_cast<const float(*)[4]>(&v[u][8]), sc, rc);
+        o.w = encode4(*reinterpret_cast<const float(*)[4]>(&v[u][12]), sc, rc);
+        *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(st) * 128 + li * 16) = o;
+        if (li == 0) {
+          const uint32_t br = st / kbs;  // batch * rows + row
+          const uint32_t kb = st - br * kbs;
+          const uint32_t b = br / static_cast<uint32_t>(rows);
+          const uint32_t r = br - b * static_cast<uint32_t>(rows);
+          if (!POW2 || scales) scales[(static_cast<int64_t>(b) * kbs + kb) * ld + r] = sc;
+          if constexpr (POW2)
+            packed[packed_offset(static_cast<int>(r), static_cast<int>(kb), (rows + 127) >> 7)] =
+                static_cast<uint8_t>(e + 127);
+        }
       }
-      if (++kb == kbs) { kb = 0; ++br; }
     }
   }
 }
