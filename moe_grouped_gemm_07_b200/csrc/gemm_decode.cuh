@@ -174,6 +174,12 @@ __global__ void __launch_bounds__(320, MINB)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The first weight tiles of this CTA go to L2 while the previous kernel on
+  // the stream (typically the activation quantiser) finishes: their DRAM
+  // latency leaves the critical path. Only a prefetch happens before the wait.
+  if (warp == 0 && lane == 0) {
+    for (int j = 0; j < S && j < nkb; ++j) tma_prefetch_l2(&tm_w, (kb_begin + j) * Cfg::BK, n0);
+  }
   pdl_wait();  // inputs may come from the previous launch on the stream
 
   float acc[EC];

@@ -126,6 +126,16 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, 
       : "memory");
 }
 
+// Fetch a tile into L2 only (no shared memory, no barrier, no data consumed
+// by the kernel): safe before griddepcontrol.wait, since L2 is where a
+// predecessor's writes land and later loads read from.
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* m, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 // Shared -> global tensor store (bulk async group of the issuing thread).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* smem_src, int32_t x,
                                              int32_t y) {
