@@ -207,6 +207,63 @@ struct Bf16Raw {
 };
 
 // Shared NT launcher for dense / contiguous / masked.
+// Split-K tail of a dense launch (MODE_SPLITK): DG_TAIL_SPLIT=0 turns it off.
+bool tail_split_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("DG_TAIL_SPLIT");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// With R = tiles % grid tiles left for a partial last wave, split each over k
+// CTAs (k a power of two, at most 8, R * k <= grid, at least 4 K-blocks per
+// part). The second launch, its prologue and the cluster exchange cost about
+// as much as 40 K-blocks of a tile (measured on B200: splits that save fewer
+// ran slower), so a split must save at least that: KB - KB / k >= 40.
+// Returns k (1 = no split).
+int tail_split_for(long long tiles, int grid, int KB) {
+  if (tiles <= grid) return 1;
+  const long long R = tiles % grid;
+  if (R == 0) return 1;
+  int k = 1;
+  while (k < 8 && R * (2 * k) <= grid && KB / (2 * k) >= 4) k *= 2;
+  return KB - KB / k >= 40 ? k : 1;
+}
+
+// How many k-CTA clusters of the split-K kernel the device runs at once
+// (cached per device and k; 0 on error).
+int splitk_clusters(int dev, int k) {
+  using Cfg = dg::GemmCfg<dg::MODE_SPLITK, 256>;
+  static std::mutex mu;
+  static int cache[kMaxDevices][9];
+  static bool done[kMaxDevices][9];
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev][k]) {
+    done[dev][k] = true;
+    cache[dev][k] = 0;
+    auto kern = dg::gemm_fp8_kernel<dg::MODE_SPLITK, 256>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(k, 1, 1);
+      cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+      cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = k;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess) cache[dev][k] = n;
+    }
+    cudaGetLastError();
+  }
+  return cache[dev][k];
+}
+
 template <int MODE>
 dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, const float* sfb,
                  const int32_t* m_indices, const int32_t* masked_m, const void* C, void* D,
@@ -253,9 +310,31 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
   args.timeout_ns = timeout_ns();
   args.drop_arrive = take_drop_flag();
   const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(sms, tiles)));
+  // Dense: a partial last wave of R tiles runs as a second launch that
+  // splits each tile along K over a cluster of k CTAs (MODE_SPLITK); the
+  // first launch takes the full waves. Both are ordered on the stream.
+  int split = 1;
+  const long long R = tiles > grid ? tiles % grid : 0;
+  if (MODE == dg::MODE_DENSE && bn == 256 && tail_split_enabled()) {
+    split = tail_split_for(tiles, grid, K / 128);
+    if (split > 1 && splitk_clusters(dev, split) < R) split = 1;  // not all at once
+  }
   if (print_configs())
-    std::fprintf(stderr, "[dg] %s M=%d N=%d K=%d G=%d: BM=128 BN=%d tiles=%lld grid=%d\n", name,
-                 M_logical, N, K, G, bn, tiles, grid);
+    std::fprintf(stderr,
+                 "[dg] %s M=%d N=%d K=%d G=%d: BM=128 BN=%d tiles=%lld grid=%d tail split %dx%lld\n",
+                 name, M_logical, N, K, G, bn, tiles, grid, split, split > 1 ? R : 0ll);
+  if (split > 1) {
+    GemmArgs tail = args;
+    args.total_tiles = static_cast<int>(tiles - R);
+    dg_status s2 = launch_gemm<MODE, 256>(ta, tb, dummy, dummy, td, args, grid, st, dev);
+    if (s2 != DG_OK) return s2;
+    tail.total_tiles = static_cast<int>(R);
+    tail.split_tile0 = static_cast<int>(tiles - R);
+    tail.split = split;
+    tail.drop_arrive = 0;
+    return launch_gemm<dg::MODE_SPLITK, 256>(ta, tb, dummy, dummy, td, tail,
+                                             static_cast<int>(R) * split, st, dev, split);
+  }
   if (bn == 256) return launch_gemm<MODE, 256>(ta, tb, dummy, dummy, td, args, grid, st, dev);
   return launch_gemm<MODE, 128>(ta, tb, dummy, dummy, td, args, grid, st, dev);
 }

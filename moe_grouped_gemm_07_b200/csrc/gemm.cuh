@@ -42,7 +42,11 @@ namespace dg {
 // [K][N], TN takes A as [K][M] and B as [K][N], TT takes A as [K][M].
 enum GemmMode : int {
   MODE_DENSE = 0, MODE_CONTIG = 1, MODE_MASKED = 2, MODE_KGROUPED = 3, MODE_PAIR = 4,
-  MODE_NN = 5, MODE_TN = 6, MODE_TT = 7
+  MODE_NN = 5, MODE_TN = 6, MODE_TT = 7,
+  // the dense launch's partial last wave, as its own launch: each leftover
+  // tile is split along K over a cluster of `split` CTAs, whose FP32
+  // partials are summed through distributed shared memory
+  MODE_SPLITK = 8
 };
 
 constexpr int kMaxKGroups = 256;
@@ -66,6 +70,7 @@ struct GemmArgs {
   int kb_off[kMaxKGroups + 1];  // K-grouped, host sizes: prefix sums of K-blocks per group
   const int32_t* ks_dev;        // K-grouped, device sizes: [G] K per group (else null)
   int kb_cap;                   // K-grouped, device sizes: K-blocks the operands hold
+  int split_tile0, split;       // MODE_SPLITK: first tail tile, CTAs per tile
 };
 
 template <int MODE, int BN_>
@@ -159,7 +164,8 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int*
     tl.b_row = tl.n0 + rank * (BN / 2);
     tl.rows = min(Cfg::BM, a.M - tl.m0);  // may be <= 0 for the second CTA
     tl.out_row0 = tl.m0;
-  } else if constexpr (MODE == MODE_DENSE || MODE == MODE_CONTIG || MODE >= MODE_NN) {
+  } else if constexpr (MODE == MODE_DENSE || MODE == MODE_CONTIG ||
+                       (MODE >= MODE_NN && MODE <= MODE_TT)) {
     const int group_tiles = Cfg::GROUP_M * a.num_n_blocks;
     const int grp = t / group_tiles;
     const int first_m = grp * Cfg::GROUP_M;
@@ -182,6 +188,25 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int*
       tl.b_row = g * a.N + tl.n0;
       tl.rows = Cfg::BM;
     }
+  } else if constexpr (MODE == MODE_SPLITK) {
+    // tile split_tile0 + t of the dense rasterisation; CTA `rank` of the
+    // cluster takes K-blocks [rank * KB / split, (rank + 1) * KB / split)
+    const int tt = a.split_tile0 + t;
+    const int group_tiles = Cfg::GROUP_M * a.num_n_blocks;
+    const int grp = tt / group_tiles;
+    const int first_m = grp * Cfg::GROUP_M;
+    const int gm = min(a.num_m_blocks - first_m, Cfg::GROUP_M);
+    const int local = tt - grp * group_tiles;
+    tl.g = 0;
+    tl.m0 = (first_m + local % gm) * Cfg::BM;
+    tl.n0 = (local / gm) * BN;
+    tl.a_row = tl.m0;
+    tl.b_row = tl.n0;
+    tl.out_row0 = tl.m0;
+    tl.rows = min(Cfg::BM, a.M - tl.m0);
+    const int KB = a.K / Cfg::BK;
+    tl.kb0 = (rank * KB) / a.split;
+    tl.nkb = ((rank + 1) * KB) / a.split - tl.kb0;
   } else if constexpr (MODE == MODE_MASKED) {
     // largest g with prefix[g] <= t
     int lo = 0, hi = a.G - 1;
@@ -283,10 +308,16 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t lane = lane_id();
   const uint64_t tmo = args.timeout_ns;
   constexpr bool PAIR = Cfg::PAIR;
-  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = leader of the pair
-  const bool leader = rank == 0;
-  const int cta_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
-  const int cta_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  constexpr bool SPLITK = MODE == MODE_SPLITK;
+  // pair: 0 = leader of the pair; split-K tail: the part of the K range
+  const uint32_t rank = (PAIR || SPLITK) ? cluster_ctarank() : 0u;
+  const bool leader = !PAIR || rank == 0;
+  const int cta_step = PAIR     ? static_cast<int>(gridDim.x >> 1)
+                       : SPLITK ? static_cast<int>(gridDim.x) / args.split
+                                : static_cast<int>(gridDim.x);
+  const int cta_first = PAIR     ? static_cast<int>(blockIdx.x >> 1)
+                        : SPLITK ? static_cast<int>(blockIdx.x) / args.split
+                                 : static_cast<int>(blockIdx.x);
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
@@ -484,6 +515,10 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
+    if constexpr (SPLITK) {  // the promotion warps' two cluster barriers
+      cluster_sync_all();
+      cluster_sync_all();
+    }
   } else if (warp == 1) {
     // ======================= MMA issuer ======================================
     // The whole warp runs the loop and waits; lane 0 issues the MMAs and
@@ -551,6 +586,10 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
+    if constexpr (SPLITK) {  // the promotion warps' two cluster barriers
+      cluster_sync_all();
+      cluster_sync_all();
+    }
   } else {
     // ======================= promotion + epilogue (8 warps) =================
     const uint32_t q = warp & 3;              // TMEM lane quadrant
@@ -558,6 +597,7 @@ __global__ void __launch_bounds__(320, 1)
     const int r_in_tile = static_cast<int>(q * 32 + lane);
     const uint32_t t_lane = tmem_base + ((q * 32) << 16);
     uint32_t acc_it = 0, sit = 0;
+    bool cluster_synced = false;  // split-K tail: both cluster barriers passed
     const int KBn = args.K / Cfg::BK;  // NT: K-blocks per row of sfb
     const int nbN = (args.N + 127) / 128;
     for (int t = cta_first; t < total_tiles; t += cta_step) {
@@ -586,6 +626,10 @@ __global__ void __launch_bounds__(320, 1)
         // sfb is [G][ceil(N/128)][K/128], or [K/128][ceil(N/128)] for B stored [K][N]
         pb = Cfg::B_MN ? args.sfb + col_first / 128
                        : args.sfb + (static_cast<long long>(tl.g) * nbN + col_first / 128) * KBn;
+        if constexpr (SPLITK) {  // this part starts at K-block kb0
+          pa += static_cast<long long>(tl.kb0) * args.ld_sfa;
+          pb += tl.kb0;
+        }
       }
       // NT scales stream through this warp's shared-memory ring by cp.async,
       // SRING K-blocks ahead: lane l copies sfa for its row, lane 0 also the
@@ -695,6 +739,50 @@ __global__ void __launch_bounds__(320, 1)
         ++acc_it;
       }
       if constexpr (!Cfg::KG) cp_async_wait<0>();
+
+      // ------------------------------------------------ split-K tail
+      if constexpr (SPLITK) {
+        // 1. every CTA of the cluster has finished its K range, so every
+        //    ring is free; 2. push the rows each part owns, [own r, own r +
+        //    own), into that part's ring as [src rank][own rows][256 cols];
+        // 3. after the second barrier, sum the owned rows over the parts in
+        //    rank order (deterministic), add C, store BF16.
+        cluster_sync_all();
+        const int sp = args.split, own = 128 / sp;
+        const int owner = r_in_tile / own;
+        const uint32_t slot = smem_addr(smem) +
+            static_cast<uint32_t>(((static_cast<int>(rank) * own + (r_in_tile - owner * own)) * 256 +
+                                   static_cast<int>(h) * EC) * 4);
+        const uint32_t remote = dsmem_addr(slot, static_cast<uint32_t>(owner));
+#pragma unroll
+        for (int j = 0; j < EC; j += 4)
+          st_dsmem_f32x4(remote + j * 4, acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+        cluster_sync_all();
+        cluster_synced = true;
+        const float* recv = reinterpret_cast<const float*>(smem);
+        const int tid = static_cast<int>(warp - 2) * 32 + static_cast<int>(lane);
+        for (int idx = tid; idx < own * (BN / 4); idx += 256) {
+          const int row = idx / (BN / 4), col = (idx % (BN / 4)) * 4;
+          const int trow = static_cast<int>(rank) * own + row;
+          const int gcol = tl.n0 + col;
+          if (trow >= tl.rows || gcol >= args.N) continue;
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int src = 0; src < sp; ++src) {
+            const float4 p = *reinterpret_cast<const float4*>(recv + (src * own + row) * 256 + col);
+            v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
+          }
+          const long long o = (tl.out_row0 + trow) * args.N + gcol;  // N % 8 == 0
+          if (args.C) {
+            const uint2 c2 =
+                *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(args.C) + o);
+            v.x += bf16_lo(c2.x); v.y += bf16_hi(c2.x);
+            v.z += bf16_lo(c2.y); v.w += bf16_hi(c2.y);
+          }
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(args.D) + o) =
+              make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+        }
+        continue;
+      }
 
       // ------------------------------------------------ tile epilogue
       // A warp whose 32 rows may all be written (or lie past the end of D,
@@ -808,6 +896,13 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   epi_done:
+    if constexpr (SPLITK) {  // reach both cluster barriers on every path
+      if (!cluster_synced) {
+        cluster_sync_all();
+        cluster_synced = true;
+        cluster_sync_all();
+      }
+    }
     cp_async_wait<0>();  // no shared-memory copy may land after the CTA exits
     if (lane == 0) bulk_wait0();  // every TMA store of this warp has completed
     __syncwarp();
