@@ -43,6 +43,15 @@ def lib():
         L.dgo_m_grouped_masked.restype = i32
         L.dgo_k_grouped_tn.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32]
         L.dgo_k_grouped_tn.restype = i32
+        L.dgo_e2m1_decode.argtypes = [C.c_uint8]
+        L.dgo_e2m1_decode.restype = f64
+        L.dgo_e2m1_encode.argtypes = [C.c_float]
+        L.dgo_e2m1_encode.restype = C.c_uint8
+        L.dgo_quantize_fp4.argtypes = [vp, i32, i32, i32, vp, vp]
+        L.dgo_quantize_fp4.restype = i32
+        L.dgo_gemm_fp8_fp4_nt.argtypes = [vp, vp, i32, vp, vp, vp, i32, vp, i32, i32, i32, vp,
+                                          i32]
+        L.dgo_gemm_fp8_fp4_nt.restype = i32
         L.dgo_calc_diff.argtypes = [vp, vp, C.c_size_t]
         L.dgo_calc_diff.restype = f64
         L.dgo_num_threads.argtypes = []
@@ -184,6 +193,44 @@ def k_grouped_tn(A, sfa, B, sfb, ks, C=None, rows=None):
                                 _p(r), nr)
     if rc != 0:
         raise ValueError("oracle k_grouped_tn: invalid arguments")
+    return R
+
+
+def e2m1_decode(code: int) -> float:
+    return lib().dgo_e2m1_decode(int(code) & 0xF)
+
+
+def e2m1_encode(y: float) -> int:
+    return int(lib().dgo_e2m1_encode(float(y)))
+
+
+def quantize_fp4(x: np.ndarray, bf16: bool = False):
+    """x: float32 [rows, cols] (or uint16 bf16 bits with bf16=True), cols % 32 == 0.
+    Returns (codes uint8 [rows, cols/2], element 2j in the low nibble of byte j;
+    scales float32 [rows, cols/32], powers of two)."""
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    codes = np.zeros((rows, cols // 2), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 32), dtype=np.float32)
+    if lib().dgo_quantize_fp4(_p(x), int(bf16), rows, cols, _p(codes), _p(scales)) != 0:
+        raise ValueError("oracle quantize_fp4: invalid arguments")
+    return codes, scales
+
+
+def gemm_fp8_fp4_nt(A, sfa, B, sfb, C=None, rows=None):
+    """FP8 x FP4 NT. A uint8 [M,K] E4M3, sfa float32 [K/128, ld]; B uint8
+    [N,K/2] packed E2M1, sfb float32 [N, K/32]; C as gemm_nt.
+    Returns float64 [len(rows) or M, N]."""
+    M, K = A.shape
+    N = B.shape[0]
+    assert B.shape[1] * 2 == K and sfb.shape == (N, K // 32)
+    r, nr = _rows(rows)
+    nr = M if r is None else nr
+    R = np.empty((nr, N), dtype=np.float64)
+    rc = lib().dgo_gemm_fp8_fp4_nt(_p(A), _p(sfa), sfa.shape[-1], _p(B), _p(sfb), _p(C),
+                                   _c_kind(C), _p(R), M, N, K, _p(r), nr)
+    if rc != 0:
+        raise ValueError("oracle gemm_fp8_fp4_nt: invalid arguments")
     return R
 
 

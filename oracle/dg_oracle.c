@@ -213,6 +213,99 @@ int dgo_gemm_nt(const uint8_t* A, const float* sfa, int ld_sfa,
   return 0;
 }
 
+/* ---- E2M1 (FP4), OCP MX v1.0 section 5.3.3 --------------------------------- */
+
+double dgo_e2m1_decode(uint8_t code) {
+  int s = (code >> 3) & 1;
+  int e = (code >> 1) & 3;
+  int m = code & 1;
+  double v = e == 0 ? 0.5 * m                     /* subnormal: m/2 * 2^(1-1) */
+                    : ldexp(1.0 + 0.5 * m, e - 1); /* normal, bias 1 */
+  return s ? -v : v;
+}
+
+uint8_t dgo_e2m1_encode(float y) {
+  uint8_t sign = signbit(y) ? 0x8 : 0x0;
+  double a = fabs((double)y);
+  if (a > 6.0) return (uint8_t)(sign | 0x7);      /* satfinite */
+  /* brute force: nearest of the 8 non-negative codes */
+  int best = 0;
+  double best_err = INFINITY;
+  for (int c = 0; c <= 7; ++c) {
+    double err = fabs(a - dgo_e2m1_decode((uint8_t)c));
+    if (err < best_err) { best = c; best_err = err; }
+    else if (err == best_err && (c & 1) == 0 && (best & 1) == 1) best = c;  /* tie: even code */
+  }
+  return (uint8_t)(sign | best);
+}
+
+/* s = 2^ceil(log2 t), t = max(amax, 1e-4f) / 6 (IEEE single division). */
+static float fp4_scale_of(float amax) {
+  float a = amax > 1e-4f ? amax : 1e-4f;
+  float t = a / 6.0f;
+  int ex = 0;
+  float m = frexpf(t, &ex);
+  return ldexpf(1.0f, m == 0.5f ? ex - 1 : ex);
+}
+
+int dgo_quantize_fp4(const void* x, int in_is_bf16, int rows, int cols,
+                     uint8_t* codes, float* scales) {
+  if (rows < 0 || cols < 0 || cols % 32 != 0) return -1;
+  int strips = cols / 32;
+  #pragma omp parallel for schedule(static)
+  for (int r = 0; r < rows; ++r) {
+    for (int c = 0; c < strips; ++c) {
+      size_t base = (size_t)r * cols + (size_t)c * 32;
+      float amax = 0.0f;
+      for (int j = 0; j < 32; ++j) {
+        float v = fabsf(load_x(x, in_is_bf16, base + j));
+        if (v > amax) amax = v;
+      }
+      float s = fp4_scale_of(amax);
+      scales[(size_t)r * strips + c] = s;
+      for (int j = 0; j < 32; j += 2) {
+        uint8_t lo = dgo_e2m1_encode(load_x(x, in_is_bf16, base + j) / s);
+        uint8_t hi = dgo_e2m1_encode(load_x(x, in_is_bf16, base + j + 1) / s);
+        codes[(base + j) / 2] = (uint8_t)(lo | (hi << 4));
+      }
+    }
+  }
+  return 0;
+}
+
+int dgo_gemm_fp8_fp4_nt(const uint8_t* A, const float* sfa, int ld_sfa,
+                        const uint8_t* B, const float* sfb,
+                        const void* C, int c_kind, double* R,
+                        int M, int N, int K, const int* rows, int n_rows) {
+  if (K % 128 != 0 || ld_sfa < M) return -1;
+  if (rows == NULL && n_rows != M) return -1;
+  int KB = K / 128, strips = K / 32;
+  #pragma omp parallel for schedule(dynamic, 1)
+  for (int i = 0; i < n_rows; ++i) {
+    int m = rows ? rows[i] : i;
+    const uint8_t* a = A + (size_t)m * K;
+    for (int n = 0; n < N; ++n) {
+      const uint8_t* b = B + (size_t)n * (K / 2);
+      double total = 0.0;
+      for (int kb = 0; kb < KB; ++kb) {
+        double blk = 0.0;
+        for (int c = 0; c < 4; ++c) {
+          int strip = 4 * kb + c;
+          double dot = 0.0;
+          for (int k = 32 * strip; k < 32 * strip + 32; ++k) {
+            uint8_t nib = (k & 1) ? (uint8_t)(b[k / 2] >> 4) : (uint8_t)(b[k / 2] & 0xF);
+            dot += g_tab[a[k]] * dgo_e2m1_decode(nib);
+          }
+          blk += (double)sfb[(size_t)n * strips + strip] * dot;
+        }
+        total += (double)sfa[(size_t)kb * ld_sfa + m] * blk;
+      }
+      R[(size_t)i * N + n] = load_c(C, c_kind, (size_t)m * N + n) + total;
+    }
+  }
+  return 0;
+}
+
 int dgo_m_grouped_contiguous(const uint8_t* A, const float* sfa, int ld_sfa,
                              const uint8_t* B, const float* sfb,
                              const int32_t* m_indices, const void* C, int c_kind,

@@ -64,6 +64,46 @@ enum { DGO_ROW_1x128_POW2 = 3, DGO_BLOCK_128x128_POW2 = 4 };
 int dgo_quantize(const void* x, int in_is_bf16, int batch, int rows, int cols,
                  int mode, uint8_t* codes, float* scales, int ld_scales);
 
+/* ---- FP8 x FP4 (mixed precision) -------------------------------------------
+ * Sources: README summary (ja.news.hada.io topic 19459), section on the
+ * 2026-04 update (FP8xFP4 GEMM) and section "GEMMインターフェースとレイアウト
+ * 制約" (SM100 scaling factors are packed UE8M0); "DeepGEMM技术解析" (mlqm.cn),
+ * section 5.2 (FP8xFP4 -> BF16). The pages fix neither the FP4 encoding nor
+ * its scale granularity; this oracle takes FP4 = E2M1 as defined by the OCP
+ * Microscaling Formats (MX) Specification v1.0, section 5.3.3 (1 sign bit,
+ * 2 exponent bits with bias 1, 1 mantissa bit, no Inf/NaN, max 6), with one
+ * power-of-two scale per 32 consecutive K elements of a row (the MX block
+ * size of that specification). */
+
+/* E2M1 code (low 4 bits used) -> value. */
+double dgo_e2m1_decode(uint8_t code);
+
+/* Nearest E2M1 value to y, ties to the even code, |y| > 6 saturates to +-6.
+ * Sign bit copied from y. */
+uint8_t dgo_e2m1_encode(float y);
+
+/*
+ * FP4 quantiser: x[rows][cols] (float, or bf16 bits if in_is_bf16) with
+ * cols % 32 == 0 -> codes[rows][cols/2] (element 2j in the low nibble of byte
+ * j, element 2j+1 in the high nibble) and scales[rows][cols/32], one per
+ * (row, 32-column strip): s = 2^ceil(log2 t) with t = max(amax, 1e-4f) / 6.0f
+ * (IEEE float division), code = E2M1(x / s). Returns 0 or -1.
+ */
+int dgo_quantize_fp4(const void* x, int in_is_bf16, int rows, int cols,
+                     uint8_t* codes, float* scales);
+
+/*
+ * FP8 x FP4 NT: R[i][n] = C[m][n] + sum_kb sfa[kb][m] *
+ *                 sum_{c < 4} sfb[n][4 kb + c] * sum_{k in strip 4 kb + c}
+ *                 dec8(A[m][k]) * dec4(B[n][k]),  m = rows[i]
+ * A [M][K] E4M3, sfa [K/128][ld_sfa]; B [N][K/2] packed E2M1 (layout of
+ * dgo_quantize_fp4), sfb [N][K/32]; C, R, rows as dgo_gemm_nt. K % 128 == 0.
+ */
+int dgo_gemm_fp8_fp4_nt(const uint8_t* A, const float* sfa, int ld_sfa,
+                        const uint8_t* B, const float* sfb,
+                        const void* C, int c_kind, double* R,
+                        int M, int N, int K, const int* rows, int n_rows);
+
 /* C operand kinds for the GEMMs below. */
 enum { DGO_C_NONE = 0, DGO_C_BF16 = 1, DGO_C_F32 = 2 };
 
