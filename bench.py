@@ -441,6 +441,97 @@ def run_ue8m0(args):
     return 0
 
 
+def run_fp8fp4(args):
+    """--workload fp8fp4: the dense sweep with E2M1 (FP4) weights, one
+    power-of-two scale per 1x32 K-strip, against E4M3 activations with
+    power-of-two 1x128 scales, on the block-scaled MMA. One step = per shape,
+    quantise A + the FP8 x FP4 GEMM; the FP8 x FP8 block-scaled GEMM on the
+    same activations is timed beside it. L2 flushed before every shape. One GPU."""
+    import torch
+    import moe_grouped_gemm_07_b200 as dg
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops"]
+    shapes = wl.dense_shapes()
+    if args.shape:
+        shapes = [tuple(int(x) for x in sh.split(",")) for sh in args.shape.split(";") if sh]
+    w4, w8, acts, outs, qbufs = {}, {}, [], [], []
+    for (N, K) in sorted(set((s_[1], s_[2]) for s_ in shapes)):
+        B = torch.from_numpy(synth.normal((N, K), synth.seed(2, nk_index(N, K), 1))).to(dev)
+        w4[(N, K)] = dg.dg_quantize_fp4_e2m1(B, with_scales=False)
+        w8[(N, K)] = dg.dg_quantize_fp8_ue8m0(B, dg.DG_QUANT_BLOCK_128x128, with_scales=False)
+        del B
+    for (M, N, K) in shapes:
+        A = torch.from_numpy(synth.normal((M, K), synth.seed(2, shape_index(M, N, K), 0))).to(dev)
+        acts.append(A)
+        outs.append(torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+        qbufs.append(dg.dg_quantize_fp8_ue8m0(A, dg.DG_QUANT_ROW_1x128, with_scales=False))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    n = len(shapes)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+
+    def run(kind, record):
+        for i, (M, N, K) in enumerate(shapes):
+            flush.fill_(i & 0xFF)
+            torch.cuda._sleep(100_000)
+            qa, _, pa = qbufs[i]
+            if record:
+                ev[i][0].record()
+            if kind == "step":
+                dg.dg_quantize_fp8_ue8m0(acts[i], dg.DG_QUANT_ROW_1x128, codes=qa, packed=pa,
+                                         with_scales=False)
+            if kind in ("step", "fp4"):
+                qb, _, pb = w4[(N, K)]
+                dg.dg_fp8_fp4_gemm_nt(qa, pa, qb, pb, None, outs[i])
+            else:
+                qb, _, pb = w8[(N, K)]
+                dg.dg_fp8_gemm_nt_ue8m0(qa, pa, qb, pb, None, outs[i])
+            if record:
+                ev[i][1].record()
+
+    res = {}
+    for kind in ("step", "fp4", "fp8"):
+        for _ in range(max(args.warmup, 3)):
+            run(kind, False)
+        torch.cuda.synchronize()
+        t = np.zeros(n)
+        for _ in range(args.steps):
+            run(kind, True)
+            torch.cuda.synchronize()
+            for i in range(n):
+                t[i] += ev[i][0].elapsed_time(ev[i][1])
+        res[kind] = t / args.steps
+    flops = [shape_flops(*sh) for sh in shapes]
+    # algorithmic bytes with FP4 weights: A + B/2 + scales (A 1 per 128, B 1 per 32) + D
+    nbytes = [M * K + N * K // 2 + M * (K // 128) + N * (K // 32) + 2 * M * N
+              for (M, N, K) in shapes]
+    big = max(range(n), key=lambda i: flops[i])
+    per = [{"M": M, "N": N, "K": K, "fp4_us": round(res["fp4"][i] * 1e3, 2),
+            "fp8_mx_us": round(res["fp8"][i] * 1e3, 2),
+            "fp4_tflops": round(flops[i] / (res["fp4"][i] * 1e-3) / 1e12, 1),
+            "fp4_gbs": round(nbytes[i] / (res["fp4"][i] * 1e-3) / 1e9, 1),
+            "fp8_mx_tflops": round(flops[i] / (res["fp8"][i] * 1e-3) / 1e12, 1)}
+           for i, (M, N, K) in enumerate(shapes)]
+    ach = flops[big] / (res["fp4"][big] * 1e-3) / 1e12
+    line = {"metric": METRIC, "workload": "dense_fp8_fp4_gemm_nt_sweep",
+            "value": round(sum(flops) / (res["step"].sum() * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(float(res["step"].sum()), 4), "steps": args.steps,
+            "higher_is_better": True,
+            "dtype": "e4m3 x e2m1 (UE8M0 scales, 1x128 / 1x32) -> f32 accumulate, bf16 out",
+            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
+                         "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4),
+                         "kernel": f"gemm_mx_kernel<FP4B>:{shapes[big][0]}x{shapes[big][1]}x{shapes[big][2]}",
+                         "peak_note": "FP8 x FP4 on kind::mxf8f6f4 runs at the FP8 rate"},
+            "fp4_gemm_only_tflops": round(sum(flops) / (res["fp4"].sum() * 1e-3) / 1e12, 2),
+            "fp8_mx_gemm_only_tflops": round(sum(flops) / (res["fp8"].sum() * 1e-3) / 1e12, 2),
+            "shapes": per}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -679,7 +770,7 @@ def main():
     ap.add_argument("--quick", action="store_true",
                     help="timed device loop only: no e2e leg, CPU baseline or clock sampling")
     ap.add_argument("--workload", default="dense",
-                    choices=["dense", "contiguous", "masked", "kgrouped", "ue8m0"],
+                    choices=["dense", "contiguous", "masked", "kgrouped", "ue8m0", "fp8fp4"],
                     help="dense (the bench line) or one MoE variant at its benchmark size")
     ap.add_argument("--masked-index", type=int, default=0,
                     help="masked workload: index into the (N, K) pairs")
@@ -688,6 +779,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "fp8fp4":
+        return run_fp8fp4(args)
     if args.workload == "ue8m0":
         return run_ue8m0(args)
     if args.workload != "dense":

@@ -207,6 +207,48 @@ dg_status dg_fp8_gemm_nt_ue8m0(const void* A, const int32_t* sfa, const void* B,
                                void* stream);
 
 /* ---------------------------------------------------------------------------
+ * FP8 x FP4 (mixed precision): E4M3 activations times E2M1 weights.
+ * Sources: README summary (ja.news.hada.io topic 19459), the 2026-04 update
+ * (FP8xFP4 GEMM on SM100) and "GEMMインターフェースとレイアウト制約" (SM100
+ * scaling factors are packed UE8M0); "DeepGEMM技术解析" (mlqm.cn), section
+ * 5.2 (FP8xFP4 -> BF16). The pages fix neither the 4-bit format nor its scale
+ * granularity; this library takes E2M1 of the OCP Microscaling Formats
+ * specification v1.0 (section 5.3.3: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6)
+ * with one power-of-two scale per 32 consecutive K elements of a row, the
+ * block size of that specification and the 1X scale vector of the tensor
+ * core's block-scaled MMA.
+ *
+ * dg_quantize_fp4_e2m1: x [rows][cols] (in_dtype F32 or BF16), cols % 128 == 0.
+ *   s = 2^ceil(log2(max(amax, 1e-4f) / 6)) per (row, 32-column strip),
+ *   code = E2M1_RN(x / s) (exact division, ties to the even code).
+ *   codes   uint8 [rows][cols/2] (written): element 2j in the low nibble of
+ *           byte j, element 2j+1 in the high nibble. 16-byte aligned.
+ *   scales  optional (NULL allowed): FP32 scales [rows][cols/32].
+ *   packed  int32 [cols/128][ceil(rows/128)][32][4] (written): byte b of word
+ *           [kb][rb][i][j] = biased exponent (log2 s + 127) of row
+ *           128 rb + 32 j + i for strip 4 kb + b -- the UE8M0 layout of
+ *           dg_quantize_fp8_ue8m0 with 32-wide strips in place of K-blocks.
+ *           Bytes of rows past `rows` are not written.
+ *   Inputs must be finite. Allocates nothing; asynchronous on `stream`.
+ *
+ * dg_fp8_fp4_gemm_nt: D = C + A @ B.T on the block-scaled MMA,
+ *   D[m][n] = C[m][n] + sum_kb sa(m, kb) * sum_{c<4} sb(n, 4 kb + c) *
+ *             sum_{k in strip 4 kb + c} A[m][k] * B[n][k]
+ *   A   [M][K] E4M3, sfa its packed UE8M0 scales from dg_quantize_fp8_ue8m0
+ *       in ROW_1x128 mode (rows = M);
+ *   B   [N][K/2] packed E2M1 and sfb its packed scales, both from
+ *       dg_quantize_fp4_e2m1 (rows = N); B 32-byte aligned;
+ *   C   [M][N] BF16 or NULL (may alias D); D [M][N] BF16.
+ *   K % 128 == 0, N % 8 == 0. Accumulation is the tensor core's FP32 across
+ *   all K (no per-K-block promotion). Errors as dg_fp8_gemm_nt_ue8m0.
+ * ------------------------------------------------------------------------- */
+dg_status dg_quantize_fp4_e2m1(const void* x, int in_dtype, int rows, int cols, void* codes,
+                               float* scales, int32_t* packed, void* stream);
+dg_status dg_fp8_fp4_gemm_nt(const void* A, const int32_t* sfa, const void* B,
+                             const int32_t* sfb, const void* C, void* D, int M, int N, int K,
+                             void* stream);
+
+/* ---------------------------------------------------------------------------
  * K-grouped GEMM with the per-group K sizes in DEVICE memory (a training
  * backward captured in a CUDA graph, where the sizes are produced on the GPU
  * and the host cannot read them). Source: README summary, "DenseとGrouped

@@ -44,7 +44,7 @@ EXPORTED = (
     "dg_get_last_device_error", "dg_debug_drop_next_arrive", "dg_get_launch_count",
     "dg_set_pdl", "dg_get_pdl", "dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks",
     "dg_quantize_fp8_ue8m0", "dg_fp8_gemm_nt_ue8m0", "dg_fp8_gemm_nn", "dg_fp8_gemm_tn",
-    "dg_fp8_gemm_tt",
+    "dg_fp8_gemm_tt", "dg_quantize_fp4_e2m1", "dg_fp8_fp4_gemm_nt",
 )
 
 _vp, _i32 = _C.c_void_p, _C.c_int
@@ -62,6 +62,8 @@ _lib.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks.argtypes = [_vp, _vp, _vp, _vp, 
                                                             _vp, _i32, _i32, _i32, _vp]
 _lib.dg_quantize_fp8_ue8m0.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp]
 _lib.dg_fp8_gemm_nt_ue8m0.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]
+_lib.dg_quantize_fp4_e2m1.argtypes = [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp]
+_lib.dg_fp8_fp4_gemm_nt.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]
 for _f in ("dg_fp8_gemm_nn", "dg_fp8_gemm_tn", "dg_fp8_gemm_tt"):
     getattr(_lib, _f).argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]
     getattr(_lib, _f).restype = _i32
@@ -321,6 +323,56 @@ def dg_fp8_gemm_nt_ue8m0(A, sfa_packed, B, sfb_packed, C, D, stream=None):
     _check("dg_fp8_gemm_nt_ue8m0",
            _lib.dg_fp8_gemm_nt_ue8m0(_ptr(A), _ptr(sfa_packed), _ptr(B), _ptr(sfb_packed), _ptr(C),
                                      _ptr(D), M, N, K, _stream(stream)))
+    return D
+
+
+def fp4_packed_shape(rows: int, cols: int):
+    """Shape of the packed UE8M0 scale tensor (int32) of a [rows, cols] FP4
+    operand: one byte per (row, 32-column strip), four strips per word."""
+    return ((cols + 127) // 128, (rows + 127) // 128, 32, 4)
+
+
+def dg_quantize_fp4_e2m1(x, codes=None, scales=None, packed=None, with_scales=True, stream=None):
+    """x [rows, cols] f32/bf16 CUDA, cols % 128 == 0. Returns (codes uint8
+    [rows, cols/2] packed E2M1, FP32 scales [rows, cols/32] or None, packed
+    UE8M0 int32 [cols/128, ceil(rows/128), 32, 4])."""
+    _cuda_contig(x, codes, scales, packed)
+    _need(x.dim() == 2, "x must be 2-D")
+    rows, cols = x.shape
+    _need(x.dtype in (torch.float32, torch.bfloat16), "x dtype")
+    dt = DG_IN_BF16 if x.dtype == torch.bfloat16 else DG_IN_F32
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    _need(codes.dtype == torch.uint8 and codes.numel() >= rows * (cols // 2), "codes")
+    if with_scales and scales is None:
+        scales = torch.zeros((rows, cols // 32), dtype=torch.float32, device=x.device)
+    if packed is None:
+        packed = torch.zeros(fp4_packed_shape(rows, cols), dtype=torch.int32, device=x.device)
+    _need(packed.dtype == torch.int32 and packed.numel() >= math.prod(fp4_packed_shape(rows, cols)),
+          "packed")
+    _check("dg_quantize_fp4_e2m1",
+           _lib.dg_quantize_fp4_e2m1(_ptr(x), dt, rows, cols, _ptr(codes), _ptr(scales),
+                                     _ptr(packed), _stream(stream)))
+    return codes, scales, packed
+
+
+def dg_fp8_fp4_gemm_nt(A, sfa_packed, B, sfb_packed, C, D, stream=None):
+    """D = C + A @ B.T, A E4M3 [M, K] with packed UE8M0 1x128 scales (from
+    dg_quantize_fp8_ue8m0, ROW mode), B packed E2M1 uint8 [N, K/2] with packed
+    1x32 scales (from dg_quantize_fp4_e2m1)."""
+    _cuda_contig(A, sfa_packed, B, sfb_packed, C, D)
+    M, K = A.shape
+    N = B.shape[0]
+    _need(_is_fp8(A) and B.dtype == torch.uint8 and B.shape[1] * 2 == K, "A/B")
+    _need(D.dtype == torch.bfloat16 and tuple(D.shape) == (M, N), "D")
+    _need(C is None or (C.dtype == torch.bfloat16 and tuple(C.shape) == (M, N)), "C")
+    _need(sfa_packed.dtype == torch.int32 and
+          sfa_packed.numel() >= math.prod(ue8m0_packed_shape(M, K)), "sfa_packed")
+    _need(sfb_packed.dtype == torch.int32 and
+          sfb_packed.numel() >= math.prod(fp4_packed_shape(N, K)), "sfb_packed")
+    _check("dg_fp8_fp4_gemm_nt",
+           _lib.dg_fp8_fp4_gemm_nt(_ptr(A), _ptr(sfa_packed), _ptr(B), _ptr(sfb_packed), _ptr(C),
+                                   _ptr(D), M, N, K, _stream(stream)))
     return D
 
 

@@ -718,19 +718,26 @@ dg_status run_k_grouped(const void* A, const float* sfa, const void* B, const fl
 }
 
 // UE8M0 block-scaled dense GEMM launcher (one CTA per SM, persistent).
+// FP4B: B is packed E2M1 [N][K/2], loaded by the 4-bit TMA type that spreads
+// each 8 packed bytes over a 16-byte shared-memory cell.
+template <bool FP4B>
 dg_status run_mx(const void* A, const int32_t* sfa, const void* B, const int32_t* sfb,
                  const void* C, void* D, int M, int N, int K, cudaStream_t st) {
   int dev = 0, sms = 0;
   dg_status s = device_sms(&dev, &sms);
   if (s != DG_OK) return s;
-  using Cfg = dg::MxCfg;
+  using Cfg = dg::MxCfgT<FP4B>;
   CUtensorMap ta, tb, td;
   if ((s = make_map_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 128,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
     return s;
-  if ((s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, 128, Cfg::BN,
-                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
-    return s;
+  if (FP4B)
+    s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, K, N, K / 2, 128, Cfg::BN,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, 128, Cfg::BN,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != DG_OK) return s;
   if ((s = make_map_2d(&td, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, 2ull * N, 32, 32,
                        CU_TENSOR_MAP_SWIZZLE_64B)) != DG_OK)
     return s;
@@ -756,15 +763,15 @@ dg_status run_mx(const void* A, const int32_t* sfa, const void* B, const int32_t
   static std::once_flag once[kMaxDevices];
   static cudaError_t attr_err[kMaxDevices];
   std::call_once(once[dev], [&] {
-    attr_err[dev] = cudaFuncSetAttribute(dg::gemm_mx_kernel,
+    attr_err[dev] = cudaFuncSetAttribute(dg::gemm_mx_kernel<FP4B>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
   });
   if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
   if (print_configs())
-    std::fprintf(stderr, "[dg] fp8_gemm_nt_ue8m0 M=%d N=%d K=%d: 128x256 block-scaled tiles=%lld grid=%d\n",
-                 M, N, K, tiles, grid);
-  cudaError_t e = launch(dg::gemm_mx_kernel, dim3(grid), dim3(320), Cfg::SMEM_BYTES, st, 1, ta, tb,
-                         td, args);
+    std::fprintf(stderr, "[dg] %s M=%d N=%d K=%d: 128x256 block-scaled tiles=%lld grid=%d\n",
+                 FP4B ? "fp8_fp4_gemm_nt" : "fp8_gemm_nt_ue8m0", M, N, K, tiles, grid);
+  cudaError_t e = launch(dg::gemm_mx_kernel<FP4B>, dim3(grid), dim3(320), Cfg::SMEM_BYTES, st, 1,
+                         ta, tb, td, args);
   if (e != cudaSuccess) return cuda_fail(e, "mx gemm launch");
   g_launches.fetch_add(1);
   return DG_OK;
@@ -942,7 +949,58 @@ dg_status dg_fp8_gemm_nt_ue8m0(const void* A, const int32_t* sfa, const void* B,
   if (!A || !B || !sfa || !sfb) return DG_ERR_INVALID_ARG;
   if (!aligned16(A) || !aligned16(B) || !aligned16(sfa) || !aligned16(sfb))
     return DG_ERR_MISALIGNED;
-  return run_mx(A, sfa, B, sfb, C, D, M, N, K, st);
+  return run_mx<false>(A, sfa, B, sfb, C, D, M, N, K, st);
+}
+
+dg_status dg_quantize_fp4_e2m1(const void* x, int in_dtype, int rows, int cols, void* codes,
+                               float* scales, int32_t* packed, void* stream) {
+  if (rows < 0 || cols < 0) return DG_ERR_INVALID_ARG;
+  if (in_dtype != DG_IN_F32 && in_dtype != DG_IN_BF16) return DG_ERR_INVALID_ARG;
+  if (cols % 128 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(rows) * cols == 0) return DG_OK;
+  if (!x || !codes || !packed) return DG_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(packed) || (scales && !aligned16(scales)))
+    return DG_ERR_MISALIGNED;
+  const long long strips = static_cast<long long>(rows) * (cols / 128);
+  if (strips >= 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
+  int dev = 0, sms = 0;
+  dg_status s = device_sms(&dev, &sms);
+  if (s != DG_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* q = static_cast<uint8_t*>(codes);
+  uint8_t* pk = reinterpret_cast<uint8_t*>(packed);
+  const int grid = static_cast<int>(std::min<long long>((strips + 63) / 64, 8ll * sms));
+  cudaError_t e =
+      in_dtype == DG_IN_BF16
+          ? launch(dg::quant_fp4_kernel<true>, dim3(grid), dim3(256), 0, st, 1, x, rows, cols, q,
+                   scales, pk)
+          : launch(dg::quant_fp4_kernel<false>, dim3(grid), dim3(256), 0, st, 1, x, rows, cols, q,
+                   scales, pk);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  g_launches.fetch_add(1);
+  return DG_OK;
+}
+
+dg_status dg_fp8_fp4_gemm_nt(const void* A, const int32_t* sfa, const void* B,
+                             const int32_t* sfb, const void* C, void* D, int M, int N, int K,
+                             void* stream) {
+  if (M < 0 || N < 0 || K < 0) return DG_ERR_INVALID_ARG;
+  if (K % 128 != 0 || N % 8 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return DG_OK;
+  if (!D) return DG_ERR_INVALID_ARG;
+  if (!aligned16(D) || (C && !aligned16(C))) return DG_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (K == 0) {
+    int dev = 0, sms = 0;
+    dg_status s = device_sms(&dev, &sms);
+    if (s != DG_OK) return s;
+    return copy_or_zero<Bf16Raw>(C, D, static_cast<long long>(M) * N, sms, st);
+  }
+  if (!A || !B || !sfa || !sfb) return DG_ERR_INVALID_ARG;
+  if (!aligned16(A) || reinterpret_cast<uintptr_t>(B) % 32 != 0 || !aligned16(sfa) ||
+      !aligned16(sfb))
+    return DG_ERR_MISALIGNED;
+  return run_mx<true>(A, sfa, B, sfb, C, D, M, N, K, st);
 }
 
 dg_status dg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb,

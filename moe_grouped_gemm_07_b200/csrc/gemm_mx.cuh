@@ -56,16 +56,26 @@ struct MxArgs {
   int drop_arrive;
 };
 
-struct MxCfg {
+// FP4B: B is E2M1 (FP8 x FP4). Its tile occupies the same shared memory as
+// an E4M3 tile -- the 4-bit TMA load leaves every 8 bytes of packed codes in
+// a 16-byte cell, the layout kind::mxf8f6f4 reads 4-bit operands in -- but
+// only the packed bytes are transferred, and its scales come per 32-wide
+// K-strip: one 512-byte unit per (K-block, 128 rows), byte b = strip b.
+template <bool FP4B>
+struct MxCfgT {
   static constexpr int BM = 128, BN = 256, BK = 128;
   static constexpr int STAGES = 4;
   static constexpr int A_BYTES = BM * BK, B_BYTES = BN * BK;
-  static constexpr int SF_STAGES = 4;
-  static constexpr int SFA_BYTES = 512, SFB_BYTES = 1024;
+  static constexpr int B_TX = FP4B ? B_BYTES / 2 : B_BYTES;  // bytes the B load delivers
+  static constexpr int SF_STAGES = FP4B ? 3 : 4;
+  // per group of 4 K-blocks: A one unit; B two units (rows 0..127, 128..255),
+  // per K-block when FP4B
+  static constexpr int SFA_BYTES = 512, SFB_BYTES = FP4B ? 4 * 1024 : 1024;
   static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;
   static constexpr int TM_SF = 256;        // first TMEM column of the scale slots
   static constexpr int SF_SLOTS = 4;       // TMEM scale slots (one group of 4 K-blocks each)
-  static constexpr int SF_SLOT_COLS = 16;  // columns per slot: A 0..3, B 4..11
+  // columns per slot: A 0..3, B 4..11 (FP4B: K-block j of the group 4+8j..11+8j)
+  static constexpr int SF_SLOT_COLS = FP4B ? 48 : 16;
   static constexpr int TMEM_COLS = 512;
   static constexpr int GROUP_M = 16;
   static constexpr int OFF_A = 0;
@@ -81,6 +91,7 @@ struct MxCfg {
   static_assert(OFF_B % 1024 == 0 && OFF_SF % 128 == 0 && OFF_STAGE % 1024 == 0, "alignment");
   static_assert(TM_SF + SF_SLOTS * SF_SLOT_COLS <= TMEM_COLS, "TMEM budget");
 };
+using MxCfg = MxCfgT<false>;
 
 template <int BN>
 __device__ __forceinline__ void mx_tile(int t, const MxArgs& a, int& m0, int& n0) {
@@ -93,10 +104,11 @@ __device__ __forceinline__ void mx_tile(int t, const MxArgs& a, int& m0, int& n0
   n0 = (local / gm) * BN;
 }
 
+template <bool FP4B>
 __global__ void __launch_bounds__(320, 1)
     gemm_mx_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ MxArgs args) {
-  using Cfg = MxCfg;
+  using Cfg = MxCfgT<FP4B>;
   constexpr int S = Cfg::STAGES;
   constexpr int SFS = Cfg::SF_STAGES;
   constexpr int BN = Cfg::BN;
@@ -171,14 +183,25 @@ __global__ void __launch_bounds__(320, 1)
           if (lane == 0) {
             const int q = kb >> 2;
             const int rba = m0 >> 7, rbb = n0 >> 7;
-            const uint32_t bbytes = rbb + 1 < args.rb_b ? Cfg::SFB_BYTES : Cfg::SFB_BYTES / 2;
+            const uint32_t bbytes = rbb + 1 < args.rb_b ? 1024u : 512u;  // B units of this tile
             uint8_t* dst = sSF + gs * Cfg::SF_BYTES;
-            mbar_arrive_expect_tx(&sf_full[gs], Cfg::SFA_BYTES + bbytes);
-            bulk_load(dst, args.sfa + (static_cast<long long>(q) * args.rb_a + rba) * 128,
-                      Cfg::SFA_BYTES, &sf_full[gs]);
-            bulk_load(dst + Cfg::SFA_BYTES,
-                      args.sfb + (static_cast<long long>(q) * args.rb_b + rbb) * 128, bbytes,
-                      &sf_full[gs]);
+            if constexpr (FP4B) {
+              const int nk = min(4, nkb - kb);  // K-blocks in this group
+              mbar_arrive_expect_tx(&sf_full[gs], Cfg::SFA_BYTES + nk * bbytes);
+              bulk_load(dst, args.sfa + (static_cast<long long>(q) * args.rb_a + rba) * 128,
+                        Cfg::SFA_BYTES, &sf_full[gs]);
+              for (int j = 0; j < nk; ++j)
+                bulk_load(dst + Cfg::SFA_BYTES + j * 1024,
+                          args.sfb + (static_cast<long long>(kb + j) * args.rb_b + rbb) * 128,
+                          bbytes, &sf_full[gs]);
+            } else {
+              mbar_arrive_expect_tx(&sf_full[gs], Cfg::SFA_BYTES + bbytes);
+              bulk_load(dst, args.sfa + (static_cast<long long>(q) * args.rb_a + rba) * 128,
+                        Cfg::SFA_BYTES, &sf_full[gs]);
+              bulk_load(dst + Cfg::SFA_BYTES,
+                        args.sfb + (static_cast<long long>(q) * args.rb_b + rbb) * 128, bbytes,
+                        &sf_full[gs]);
+            }
           }
           ++git;
         }
@@ -188,7 +211,7 @@ __global__ void __launch_bounds__(320, 1)
         if (args.drop_arrive && it == 0) {
           dropped = 0;  // test hook: never arm stage 0
         } else if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES);
+          mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_TX);
           tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], kb * Cfg::BK, m0);
           tma_load_2d(sB + s * Cfg::B_BYTES, &tm_b, &full[s], kb * Cfg::BK, n0);
         }
@@ -232,8 +255,17 @@ __global__ void __launch_bounds__(320, 1)
             const uint32_t src = smem_addr(sSF + gs * Cfg::SF_BYTES);
             const uint32_t dst = tmem_base + Cfg::TM_SF + slot * Cfg::SF_SLOT_COLS;
             tmem_cp_32x128b_x4(dst, smem_desc_noswz(src, 128));                  // A rows 0..127
-            tmem_cp_32x128b_x4(dst + 4, smem_desc_noswz(src + 512, 128));        // B rows 0..127
-            tmem_cp_32x128b_x4(dst + 8, smem_desc_noswz(src + 1024, 128));       // B rows 128..255
+            if constexpr (FP4B) {
+              const int nk = min(4, nkb - kb);
+              for (int j = 0; j < nk; ++j) {  // B, K-block kb + j
+                const uint32_t sj = src + Cfg::SFA_BYTES + j * 1024;
+                tmem_cp_32x128b_x4(dst + 4 + 8 * j, smem_desc_noswz(sj, 128));        // rows 0..127
+                tmem_cp_32x128b_x4(dst + 8 + 8 * j, smem_desc_noswz(sj + 512, 128));  // 128..255
+              }
+            } else {
+              tmem_cp_32x128b_x4(dst + 4, smem_desc_noswz(src + 512, 128));     // B rows 0..127
+              tmem_cp_32x128b_x4(dst + 8, smem_desc_noswz(src + 1024, 128));    // B rows 128..255
+            }
             mma_commit(&sf_empty[gs]);  // the scale stage is free once the copies are done
           }
           __syncwarp();
@@ -247,13 +279,25 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t a_base = smem_addr(sA + s * Cfg::A_BYTES);
           const uint32_t b_base = smem_addr(sB + s * Cfg::B_BYTES);
           const uint32_t sid = static_cast<uint32_t>(kb & 3);
-          const uint32_t idesc = idesc_mx_e4m3(Cfg::BM, BN, sid, sid);
           const uint32_t sfa_t = tmem_base + Cfg::TM_SF + slot * Cfg::SF_SLOT_COLS;
+          if constexpr (FP4B) {
+            // A: byte kb % 4 (one scale per K-block); B: the K-block's own
+            // unit, byte k = the 32-wide strip this MMA covers
+            const uint32_t sfb_t = sfa_t + 4 + 8 * sid;
 #pragma unroll
-          for (int k = 0; k < Cfg::BK / 32; ++k)
-            mma_mxf8f6f4(tmem_base, smem_desc_sw128(a_base + k * 32, 16, 1024),
-                         smem_desc_sw128(b_base + k * 32, 16, 1024), idesc, sfa_t, sfa_t + 4,
-                         (kb > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < Cfg::BK / 32; ++k)
+              mma_mxf8f6f4(tmem_base, smem_desc_sw128(a_base + k * 32, 16, 1024),
+                           smem_desc_sw128(b_base + k * 32, 16, 1024),
+                           idesc_mx_e4m3_e2m1(Cfg::BM, BN, sid, static_cast<uint32_t>(k)), sfa_t,
+                           sfb_t, (kb > 0 || k > 0) ? 1u : 0u);
+          } else {
+            const uint32_t idesc = idesc_mx_e4m3(Cfg::BM, BN, sid, sid);
+#pragma unroll
+            for (int k = 0; k < Cfg::BK / 32; ++k)
+              mma_mxf8f6f4(tmem_base, smem_desc_sw128(a_base + k * 32, 16, 1024),
+                           smem_desc_sw128(b_base + k * 32, 16, 1024), idesc, sfa_t, sfa_t + 4,
+                           (kb > 0 || k > 0) ? 1u : 0u);
+          }
           mma_commit(&empty[s]);
           if ((kb & 3) == 3 || kb == nkb - 1) mma_commit(&slot_done[slot]);
           if (kb == nkb - 1) mma_commit(tfull);

@@ -461,6 +461,13 @@ __host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, uint32_t a_sf
          | (a_sf_id << 29);                           // A scale id
 }
 
+// Same with B in E2M1 (format code 5 at bits 10..12; 4-bit operands are
+// K-major only).
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3_e2m1(int M, int N, uint32_t a_sf_id,
+                                                          uint32_t b_sf_id) {
+  return idesc_mx_e4m3(M, N, a_sf_id, b_sf_id) | (5u << 10);
+}
+
 // Instruction descriptor for kind::f8f6f4, E4M3 x E4M3 -> F32, dense.
 // a_mn_major / b_mn_major select MN-major (transposed) smem operands.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn_major,

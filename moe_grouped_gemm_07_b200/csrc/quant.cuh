@@ -330,4 +330,93 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const void* __restrict__
   }
 }
 
+// ---------------------------------------------------------------- FP4 (E2M1)
+// E2M1 (OCP Microscaling Formats v1.0, section 5.3.3): 1 sign bit, 2 exponent
+// bits (bias 1), 1 mantissa bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6. Round
+// to nearest, ties to the even code: the thresholds are the midpoints of
+// neighbouring magnitudes, strict where the lower neighbour has the even code
+// and inclusive where the upper one has; |y| > 6 gives the largest code.
+__device__ __forceinline__ uint32_t e2m1_code(float y) {
+  const float a = fabsf(y);
+  const uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
+                     (a >= 3.5f) + (a > 5.0f);
+  return c | ((__float_as_uint(y) >> 28) & 8u);
+}
+
+// Exponent e of the FP4 scale 2^e = 2^ceil(log2 t), t = max(amax, 1e-4f) / 6
+// rounded exactly as the IEEE division (quotient(); t >= 1.6e-5 is normal).
+__device__ __forceinline__ int fp4_exponent(float amax) {
+  constexpr float kInv6 = 1.0f / 6.0f;  // correctly rounded at compile time
+  const uint32_t b = __float_as_uint(quotient(fmaxf(amax, 1e-4f), 6.0f, kInv6));
+  const int e = static_cast<int>((b >> 23) & 0xFFu) - 127;
+  return (b & 0x7FFFFFu) ? e + 1 : e;
+}
+
+// FP4 quantiser: x [rows][cols] (cols % 128 == 0) -> codes [rows][cols/2]
+// (element 2j in the low nibble of byte j), one power-of-two scale per
+// (row, 32-column strip): FP32 copies in scales [rows][cols/32] (optional) and
+// UE8M0 bytes in `packed` at packed_offset(row, strip), i.e. the block-scaled
+// MMA's layout with 32-wide strips in place of K-blocks. Lanes as in
+// quant_row_kernel: 8 lanes per 128-column strip, 16 values each, so a lane
+// pair holds one 32-wide strip; U rounds of 4 strips in flight per warp.
+template <bool BF16>
+__global__ void __launch_bounds__(256) quant_fp4_kernel(const void* __restrict__ x, int rows,
+                                                        int cols, uint8_t* __restrict__ codes,
+                                                        float* __restrict__ scales,
+                                                        uint8_t* __restrict__ packed) {
+  constexpr int U = 2;
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 3;
+  const int li = lane & 7;
+  const uint32_t kbs = static_cast<uint32_t>(cols) >> 7;
+  const uint32_t nstrips = static_cast<uint32_t>(rows) * kbs;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  const uint32_t warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int rblocks = (rows + 127) >> 7;
+  for (uint32_t s0 = warp0 * (4 * U); s0 < nstrips; s0 += nwarps * (4 * U)) {
+    float v[U][16];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t st = s0 + 4 * u + g;
+      if (st < nstrips) {
+        load16<BF16>(x, static_cast<int64_t>(st) * 128 + li * 16, v[u]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[u][k] = 0.0f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t st = s0 + 4 * u + g;
+      float amax = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(v[u][k]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      const int e = fp4_exponent(amax);
+      const float rc = exp2_exact(-e);  // x * 2^-e is the exact quotient x / s
+      if (st < nstrips) {
+        uint32_t w[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t acc = 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc |= e2m1_code(v[u][h * 8 + j] * rc) << (4 * j);
+          w[h] = acc;
+        }
+        *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(st) * 64 + li * 8) =
+            make_uint2(w[0], w[1]);
+        if ((li & 1) == 0) {
+          const uint32_t r = st / kbs;
+          const uint32_t kb = st - r * kbs;
+          const int strip = static_cast<int>(kb) * 4 + (li >> 1);
+          if (scales) scales[static_cast<int64_t>(st) * 4 + (li >> 1)] = exp2_exact(e);
+          packed[packed_offset(static_cast<int>(r), strip, rblocks)] = static_cast<uint8_t>(e + 127);
+        }
+      }
+    }
+  }
+}
+
 }  // namespace dg

@@ -224,6 +224,13 @@ double dgo_e2m1_decode(uint8_t code) {
   return s ? -v : v;
 }
 
+/* 16-entry decode table, filled once when the library is loaded. */
+static double g_tab4[16];
+
+__attribute__((constructor)) static void build_table4_at_load(void) {
+  for (int c = 0; c < 16; ++c) g_tab4[c] = dgo_e2m1_decode((uint8_t)c);
+}
+
 uint8_t dgo_e2m1_encode(float y) {
   uint8_t sign = signbit(y) ? 0x8 : 0x0;
   double a = fabs((double)y);
@@ -294,7 +301,7 @@ int dgo_gemm_fp8_fp4_nt(const uint8_t* A, const float* sfa, int ld_sfa,
           double dot = 0.0;
           for (int k = 32 * strip; k < 32 * strip + 32; ++k) {
             uint8_t nib = (k & 1) ? (uint8_t)(b[k / 2] >> 4) : (uint8_t)(b[k / 2] & 0xF);
-            dot += g_tab[a[k]] * dgo_e2m1_decode(nib);
+            dot += g_tab[a[k]] * g_tab4[nib];
           }
           blk += (double)sfb[(size_t)n * strips + strip] * dot;
         }

@@ -107,3 +107,22 @@ def test_host_validation_before_any_cuda_call():
         dg.DG_ERR_INVALID_ARG
     assert L.dg_quantize_fp8(fake, 0, 1, 128, 128, 0, fake, fake, 126, None) == \
         dg.DG_ERR_INVALID_ARG
+
+
+def test_fp4_entry_validation_before_any_cuda_call():
+    import moe_grouped_gemm_07_b200 as dg
+    L, vp = dg._lib, ctypes.c_void_p
+    fake = vp(0x1000)
+    q = L.dg_quantize_fp4_e2m1
+    assert q(fake, 0, 8, 100, fake, None, fake, None) == dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert q(fake, 7, 8, 128, fake, None, fake, None) == dg.DG_ERR_INVALID_ARG
+    assert q(fake, 0, -1, 128, fake, None, fake, None) == dg.DG_ERR_INVALID_ARG
+    assert q(None, 0, 0, 128, None, None, None, None) == dg.DG_OK
+    assert q(fake, 0, 8, 128, vp(0x1008), None, fake, None) == dg.DG_ERR_MISALIGNED
+    g = L.dg_fp8_fp4_gemm_nt
+    assert g(fake, fake, fake, fake, None, fake, 8, 8, 100, None) == dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert g(fake, fake, fake, fake, None, fake, 8, 12, 128, None) == dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert g(fake, fake, fake, fake, None, fake, -1, 8, 128, None) == dg.DG_ERR_INVALID_ARG
+    assert g(None, None, None, None, None, None, 0, 8, 128, None) == dg.DG_OK
+    # the packed E2M1 operand must be 32-byte aligned (4-bit TMA loads)
+    assert g(fake, fake, vp(0x1010), fake, None, fake, 8, 8, 128, None) == dg.DG_ERR_MISALIGNED
