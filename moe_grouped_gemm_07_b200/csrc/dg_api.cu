@@ -14,6 +14,7 @@
 #include "../../include/dg.h"
 #include "gemm.cuh"
 #include "gemm_mx.cuh"
+#include "gemm_mx_decode.cuh"
 #include "gemm_decode.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
@@ -501,41 +502,52 @@ dg_status run_pair(const void* A, const float* sfa, int ld_sfa, const void* B, c
 // Largest cluster size (1..16) that the device can co-schedule for this
 // kernel (above 8 only where non-portable cluster sizes are allowed); cached
 // per device and instantiation.
+// Largest cluster size (<= 16, or 8 without non-portable sizes) of which
+// enough co-resident clusters fit to fill most of the GPU; 0 on failure.
+int probe_max_cluster(const void* kern, int smem) {
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return 0;
+  const bool nonportable =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+  cudaGetLastError();
+  for (int c = nonportable ? 16 : 8; c >= 1; --c) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(c, 1, 1);
+    cfg.blockDim = dim3(320, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = c;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n * c >= 64) return c;
+    cudaGetLastError();
+  }
+  return 0;
+}
+
 template <int BNP, int MINB>
 int max_cluster(int dev) {
-  using Cfg = dg::DecodeCfg<BNP, MINB>;
   static std::once_flag once[kMaxDevices];
   static int best[kMaxDevices];
   std::call_once(once[dev], [&] {
-    auto kern = dg::gemm_decode_kernel<BNP, MINB>;
-    best[dev] = 0;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::SMEM_BYTES) != cudaSuccess)
-      return;
-    const bool nonportable =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-        cudaSuccess;
-    cudaGetLastError();
-    for (int c = nonportable ? 16 : 8; c >= 1; --c) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(c, 1, 1);
-      cfg.blockDim = dim3(320, 1, 1);
-      cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = c;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      // enough co-resident clusters of this size to fill most of the GPU
-      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n * c >= 64) {
-        best[dev] = c;
-        return;
-      }
-      cudaGetLastError();
-    }
+    best[dev] = probe_max_cluster(reinterpret_cast<const void*>(dg::gemm_decode_kernel<BNP, MINB>),
+                                  dg::DecodeCfg<BNP, MINB>::SMEM_BYTES);
+  });
+  return best[dev];
+}
+
+template <int BNP, int MINB, bool W4>
+int max_cluster_mx(int dev) {
+  static std::once_flag once[kMaxDevices];
+  static int best[kMaxDevices];
+  std::call_once(once[dev], [&] {
+    best[dev] = probe_max_cluster(
+        reinterpret_cast<const void*>(dg::gemm_mx_decode_kernel<BNP, MINB, W4>),
+        dg::MxDecodeCfg<BNP, MINB, W4>::SMEM_BYTES);
   });
   return best[dev];
 }
@@ -641,6 +653,95 @@ dg_status dispatch_decode(const void* A, const float* sfa, const void* B, const 
     default: DG_RUN_DECODE(128);
   }
 #undef DG_RUN_DECODE
+}
+
+// Block-scaled small-M launcher (swap-AB, cluster split-K; W4: E2M1 weights).
+template <int BNP, int MINB, bool W4>
+dg_status run_mx_decode(const void* X, const int32_t* sfx, const void* W, const int32_t* sfw,
+                        const void* C, void* D, int M, int N, int K, int splits, cudaStream_t st) {
+  using Cfg = dg::MxDecodeCfg<BNP, MINB, W4>;
+  const int n_tiles = (N + 127) / 128;
+  CUtensorMap tw, tx;
+  dg_status s;
+  if (W4)
+    s = make_map_2d(&tw, W, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, K, N, K / 2, 128, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    s = make_map_2d(&tw, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, 128, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != DG_OK) return s;
+  if ((s = make_map_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, BNP,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  dg::MxDecodeArgs args;
+  std::memset(&args, 0, sizeof args);
+  args.M = M;
+  args.N = N;
+  args.K = K;
+  args.KB = K / 128;
+  args.splits = splits;
+  args.rb_w = n_tiles;
+  args.sfx = sfx;
+  args.sfw = sfw;
+  args.C = C;
+  args.D = D;
+  args.timeout_ns = timeout_ns();
+  args.drop_arrive = take_drop_flag();
+  if (print_configs())
+    std::fprintf(stderr,
+                 "[dg] %s decode M=%d N=%d K=%d: block-scaled swap-AB BNP=%d (%d CTA/SM), "
+                 "n_tiles=%d x split-K %d (cluster), %d stages\n",
+                 W4 ? "fp8_fp4_gemm_nt" : "fp8_gemm_nt_ue8m0", M, N, K, BNP, MINB, n_tiles, splits,
+                 Cfg::STAGES);
+  cudaError_t e = launch(dg::gemm_mx_decode_kernel<BNP, MINB, W4>, dim3(splits, n_tiles, 1),
+                         dim3(320), Cfg::SMEM_BYTES, st, splits, tw, tx, args);
+  if (e != cudaSuccess) return cuda_fail(e, "block-scaled decode launch");
+  g_launches.fetch_add(1);
+  return DG_OK;
+}
+
+// M <= 128 on the block-scaled path: the decode plan of the promotion path
+// (CTAs per SM, split count), DG_DECODE_MINB / DG_DECODE_SPLITS honoured.
+template <bool W4>
+dg_status dispatch_mx_decode(const void* X, const int32_t* sfx, const void* W,
+                             const int32_t* sfw, const void* C, void* D, int M, int N, int K,
+                             cudaStream_t st) {
+  int dev = 0, sms = 0;
+  dg_status s = device_sms(&dev, &sms);
+  if (s != DG_OK) return s;
+  const int KB = K / 128;
+  const int n_tiles = (N + 127) / 128;
+  const int bnp = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  int cap1 = 0, cap2 = 0;
+  switch (bnp) {
+    case 16: cap1 = max_cluster_mx<16, 1, W4>(dev); cap2 = max_cluster_mx<16, 2, W4>(dev); break;
+    case 32: cap1 = max_cluster_mx<32, 1, W4>(dev); cap2 = max_cluster_mx<32, 2, W4>(dev); break;
+    case 64: cap1 = max_cluster_mx<64, 1, W4>(dev); cap2 = max_cluster_mx<64, 2, W4>(dev); break;
+    default: cap1 = max_cluster_mx<128, 1, W4>(dev); cap2 = max_cluster_mx<128, 2, W4>(dev); break;
+  }
+  if (cap1 <= 0 || cap2 <= 0) return DG_ERR_CUDA;
+  DecodePlan p = plan_decode(M, n_tiles, KB, sms, cap1, cap2);
+  if (const char* e = std::getenv("DG_DECODE_MINB")) {
+    const int f = std::atoi(e);
+    if (f == 1 || f == 2) p.minb = f;
+  }
+  const int cap = p.minb == 1 ? cap1 : cap2;
+  p.splits = std::min(p.splits, std::min(cap, 8));
+  if (const char* e = std::getenv("DG_DECODE_SPLITS")) {
+    const int f = std::atoi(e);
+    if (f >= 1) p.splits = std::max(1, std::min(std::min(f, std::min(cap, 8)), KB));
+  }
+#define DG_RUN_MX_DECODE(BNP_)                                                                  \
+  return p.minb == 1                                                                            \
+             ? run_mx_decode<BNP_, 1, W4>(X, sfx, W, sfw, C, D, M, N, K, p.splits, st)       \
+             : run_mx_decode<BNP_, 2, W4>(X, sfx, W, sfw, C, D, M, N, K, p.splits, st)
+  switch (bnp) {
+    case 16: DG_RUN_MX_DECODE(16);
+    case 32: DG_RUN_MX_DECODE(32);
+    case 64: DG_RUN_MX_DECODE(64);
+    default: DG_RUN_MX_DECODE(128);
+  }
+#undef DG_RUN_MX_DECODE
 }
 
 // K-grouped TN launcher. Sizes come either from the host (`ks`, sumK their
@@ -949,6 +1050,7 @@ dg_status dg_fp8_gemm_nt_ue8m0(const void* A, const int32_t* sfa, const void* B,
   if (!A || !B || !sfa || !sfb) return DG_ERR_INVALID_ARG;
   if (!aligned16(A) || !aligned16(B) || !aligned16(sfa) || !aligned16(sfb))
     return DG_ERR_MISALIGNED;
+  if (M <= 128) return dispatch_mx_decode<false>(A, sfa, B, sfb, C, D, M, N, K, st);
   return run_mx<false>(A, sfa, B, sfb, C, D, M, N, K, st);
 }
 
@@ -1000,6 +1102,7 @@ dg_status dg_fp8_fp4_gemm_nt(const void* A, const int32_t* sfa, const void* B,
   if (!aligned16(A) || reinterpret_cast<uintptr_t>(B) % 32 != 0 || !aligned16(sfa) ||
       !aligned16(sfb))
     return DG_ERR_MISALIGNED;
+  if (M <= 128) return dispatch_mx_decode<true>(A, sfa, B, sfb, C, D, M, N, K, st);
   return run_mx<true>(A, sfa, B, sfb, C, D, M, N, K, st);
 }
 

@@ -103,6 +103,81 @@ struct DecodeCfg {
   static_assert(SMEM_BYTES <= (MINB == 2 ? 113 : 227) * 1024, "MINB CTAs per SM");
 };
 
+// Split-K reduction of a cluster's partial 128 x BNP tiles (swap-AB decode
+// kernels): CTA `rank` of `splits` owns the 8-row units [16 rank / splits,
+// 16 (rank + 1) / splits) of the tile. After a cluster barrier (every ring is
+// free) each of warps 2..9 -- thread (q, h, lane) holding tile row
+// 32 q + lane, tokens [h EC, h EC + EC) in acc -- pushes its row into the
+// owner's receive slot for this rank with remote stores; after a second
+// barrier each CTA sums its units over the slots in rank order
+// (deterministic), adds C and stores BF16 rows of D (tokens m < M, weight rows
+// n < N). With one split the barriers are CTA barriers and the slots local.
+// `recv` is this CTA's shared memory (the ring, free by then).
+template <int BNP, int EC, int RECV_PITCH>
+__device__ __forceinline__ void splitk_reduce_store(const float (&acc)[EC], float* recv,
+                                                    uint32_t rank, int splits, uint32_t warp,
+                                                    uint32_t lane, int n0, int M, int N,
+                                                    const void* C, void* D) {
+  const uint32_t q = warp & 3;
+  const uint32_t h = (warp - 2) >> 2;
+  if (splits > 1) cluster_sync_all(); else __syncthreads();
+  // rank o owns units [16o/splits, 16(o+1)/splits); a slot holds UMAX units
+  const int UMAX = (16 + splits - 1) / splits;
+  if (warp >= 2) {
+    // push: this thread holds row n_local of the tile for tokens [h*EC, h*EC+EC)
+    const int n_local = static_cast<int>(q * 32 + lane);
+    const int unit = n_local >> 3;
+    const int owner = (splits * (unit + 1) + 15) / 16 - 1;  // largest o with 16o/splits <= unit
+    const int owner_lo = (owner * 16) / splits;
+    const int slot_row = ((static_cast<int>(rank) * UMAX + (unit - owner_lo)) << 3) + (n_local & 7);
+    float* dst = recv + slot_row * RECV_PITCH + h * EC;
+    if (splits == 1) {
+#pragma unroll
+      for (int j = 0; j < EC; j += 4)
+        *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+    } else {
+      const uint32_t remote = dsmem_addr(smem_addr(dst), static_cast<uint32_t>(owner));
+#pragma unroll
+      for (int j = 0; j < EC; j += 4)
+        st_dsmem_f32x4(remote + j * 4, acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+    }
+  }
+  if (splits > 1) cluster_sync_all(); else __syncthreads();
+  {
+    // this CTA owns units [lo, hi); item = (unit uu, token m), token fastest
+    // so that a warp reads consecutive floats of a slot row
+    const int lo = (static_cast<int>(rank) * 16) / splits;
+    const int hi = ((static_cast<int>(rank) + 1) * 16) / splits;
+    const int items = BNP * (hi - lo);
+    for (int itm = threadIdx.x; itm < items; itm += blockDim.x) {
+      const int uu = itm / BNP;
+      const int m = itm - uu * BNP;
+      const int gn = n0 + ((lo + uu) << 3);
+      if (m >= M || gn >= N) continue;
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int src = 0; src < splits; ++src) {  // rank order: deterministic
+        const float* p = recv + ((src * UMAX + uu) << 3) * RECV_PITCH + m;
+#pragma unroll
+        for (int r8 = 0; r8 < 8; ++r8) v[r8] += p[r8 * RECV_PITCH];
+      }
+      const long long o = static_cast<long long>(m) * N + gn;
+      if (C) {
+        const uint4 c4 = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(C) + o);
+        v[0] += bf16_lo(c4.x); v[1] += bf16_hi(c4.x);
+        v[2] += bf16_lo(c4.y); v[3] += bf16_hi(c4.y);
+        v[4] += bf16_lo(c4.z); v[5] += bf16_hi(c4.z);
+        v[6] += bf16_lo(c4.w); v[7] += bf16_hi(c4.w);
+      }
+      uint4 out;
+      out.x = pack_bf16x2(v[0], v[1]);
+      out.y = pack_bf16x2(v[2], v[3]);
+      out.z = pack_bf16x2(v[4], v[5]);
+      out.w = pack_bf16x2(v[6], v[7]);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(D) + o) = out;
+    }
+  }
+}
+
 template <int BNP, int MINB>
 __global__ void __launch_bounds__(320, MINB)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tm_w,    // B: [N][K] e4m3
@@ -325,65 +400,11 @@ __global__ void __launch_bounds__(320, MINB)
 
   // ---------------------------------------------------------- split-K reduction
   // Every role is done and every copy / MMA has landed, so this CTA's ring is
-  // free; the first barrier makes that true for every CTA of the cluster.
+  // free; the first barrier (inside) makes that true for every CTA of the cluster.
   tc_fence_before();
   pdl_trigger();
-  if (splits > 1) cluster_sync_all(); else __syncthreads();
-  // rank o owns units [16o/splits, 16(o+1)/splits); a slot holds UMAX units
-  const int UMAX = (16 + splits - 1) / splits;
-  if (warp >= 2) {
-    // push: this thread holds row n_local of the tile for tokens [h*EC, h*EC+EC)
-    const int n_local = static_cast<int>(q * 32 + lane);
-    const int unit = n_local >> 3;
-    const int owner = (splits * (unit + 1) + 15) / 16 - 1;  // largest o with 16o/splits <= unit
-    const int owner_lo = (owner * 16) / splits;
-    const int slot_row = ((static_cast<int>(rank) * UMAX + (unit - owner_lo)) << 3) + (n_local & 7);
-    float* dst = recv + slot_row * Cfg::RECV_PITCH + h * EC;
-    if (splits == 1) {
-#pragma unroll
-      for (int j = 0; j < EC; j += 4)
-        *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-    } else {
-      const uint32_t remote = dsmem_addr(smem_addr(dst), static_cast<uint32_t>(owner));
-#pragma unroll
-      for (int j = 0; j < EC; j += 4)
-        st_dsmem_f32x4(remote + j * 4, acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-    }
-  }
-  if (splits > 1) cluster_sync_all(); else __syncthreads();
-  {
-    // this CTA owns units [lo, hi); item = (unit uu, token m), token fastest
-    // so that a warp reads consecutive floats of a slot row
-    const int lo = (static_cast<int>(rank) * 16) / splits;
-    const int hi = ((static_cast<int>(rank) + 1) * 16) / splits;
-    const int items = BNP * (hi - lo);
-    for (int itm = threadIdx.x; itm < items; itm += blockDim.x) {
-      const int uu = itm / BNP;
-      const int m = itm - uu * BNP;
-      const int gn = n0 + ((lo + uu) << 3);
-      if (m >= args.M || gn >= args.N) continue;
-      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int src = 0; src < splits; ++src) {  // rank order: deterministic
-        const float* p = recv + ((src * UMAX + uu) << 3) * Cfg::RECV_PITCH + m;
-#pragma unroll
-        for (int r8 = 0; r8 < 8; ++r8) v[r8] += p[r8 * Cfg::RECV_PITCH];
-      }
-      const long long o = static_cast<long long>(m) * args.N + gn;
-      if (args.C) {
-        const uint4 c4 = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(args.C) + o);
-        v[0] += bf16_lo(c4.x); v[1] += bf16_hi(c4.x);
-        v[2] += bf16_lo(c4.y); v[3] += bf16_hi(c4.y);
-        v[4] += bf16_lo(c4.z); v[5] += bf16_hi(c4.z);
-        v[6] += bf16_lo(c4.w); v[7] += bf16_hi(c4.w);
-      }
-      uint4 out;
-      out.x = pack_bf16x2(v[0], v[1]);
-      out.y = pack_bf16x2(v[2], v[3]);
-      out.z = pack_bf16x2(v[4], v[5]);
-      out.w = pack_bf16x2(v[6], v[7]);
-      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.D) + o) = out;
-    }
-  }
+  splitk_reduce_store<BNP, EC, Cfg::RECV_PITCH>(acc, recv, rank, splits, warp, lane, n0, args.M,
+                                                args.N, args.C, args.D);
   // no peer touches this CTA's shared memory after the second barrier
 
   if (warp == 1) {

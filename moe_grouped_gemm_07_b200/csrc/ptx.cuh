@@ -468,6 +468,14 @@ __host__ __device__ constexpr uint32_t idesc_mx_e4m3_e2m1(int M, int N, uint32_t
   return idesc_mx_e4m3(M, N, a_sf_id, b_sf_id) | (5u << 10);
 }
 
+// Block-scaled kind::mxf8f6f4 descriptor with explicit operand formats
+// (0 = E4M3, 5 = E2M1) at bits 7..9 (A) and 10..12 (B).
+__host__ __device__ constexpr uint32_t idesc_mx_f8f6f4(int M, int N, uint32_t a_sf_id,
+                                                       uint32_t b_sf_id, uint32_t a_fmt,
+                                                       uint32_t b_fmt) {
+  return idesc_mx_e4m3(M, N, a_sf_id, b_sf_id) | (a_fmt << 7) | (b_fmt << 10);
+}
+
 // Instruction descriptor for kind::f8f6f4, E4M3 x E4M3 -> F32, dense.
 // a_mn_major / b_mn_major select MN-major (transposed) smem operands.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn_major,

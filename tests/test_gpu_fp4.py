@@ -138,3 +138,76 @@ def test_fp8_fp4_dropped_arrive_times_out_and_recovers():
         check_close(as_f64(D), oracle.gemm_fp8_fp4_nt(oqa, osa, oqb, osb), "after recovery")
     finally:
         dg.dg_set_wait_timeout_ns(0)
+
+
+# --------------------------------------------------------------- M <= 128
+# The block-scaled decode kernel (swap-AB, cluster split-K): token widths
+# 16..128, split counts from the plan, ragged N, C.
+DECODE_CASES = [
+    (1, 256, 4096, False),
+    (16, 2112, 1024, True),
+    (30, 384, 640, False),
+    (64, 264, 512, True),     # ragged last weight tile
+    (100, 1032, 2048, True),
+    (128, 7168, 2048, False),
+    (128, 19200, 256, False),  # at least one weight tile per SM: one split
+]
+
+
+@pytest.mark.parametrize("M,N,K,with_c", DECODE_CASES)
+def test_fp8_fp4_decode_vs_oracle(M, N, K, with_c):
+    w = wl.dense(M, N, K, cfg=98, shape=M + N + K, with_c=with_c)
+    (qa, pa, qb, pb), (oqa, osa, oqb, osb) = quantise_both(w)
+    Cb = synth.to_bf16_bits(w.C) if with_c else None
+    R = oracle.gemm_fp8_fp4_nt(oqa, osa, oqb, osb, Cb)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
+    dg.dg_fp8_fp4_gemm_nt(qa, pa, qb, pb, bf16_dev(Cb) if with_c else None, D)
+    check_close(as_f64(D), R, f"fp8 x fp4 decode {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("minb,splits", [(1, 1), (2, 1), (1, 3), (2, 5), (1, 8), (2, 8)])
+def test_fp8_fp4_decode_plans(monkeypatch, minb, splits):
+    """Forced plans (CTAs per SM, split count) give the same result, bit for
+    bit across repeats, and meet the bar."""
+    monkeypatch.setenv("DG_DECODE_MINB", str(minb))
+    monkeypatch.setenv("DG_DECODE_SPLITS", str(splits))
+    M, N, K = 48, 640, 2048
+    w = wl.dense(M, N, K, cfg=99, shape=minb * 10 + splits, with_c=True)
+    (qa, pa, qb, pb), (oqa, osa, oqb, osb) = quantise_both(w)
+    Cb = synth.to_bf16_bits(w.C)
+    outs = []
+    for _ in range(2):
+        D = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
+        dg.dg_fp8_fp4_gemm_nt(qa, pa, qb, pb, bf16_dev(Cb), D)
+        outs.append(D)
+    assert torch.equal(outs[0], outs[1])
+    check_close(as_f64(outs[0]), oracle.gemm_fp8_fp4_nt(oqa, osa, oqb, osb, Cb),
+                f"plan minb={minb} splits={splits}")
+
+
+def test_fp8_fp4_decode_full_size():
+    """64 x 7168 x 16384, every row against the oracle."""
+    M, N, K = 64, 7168, 16384
+    w = wl.dense(M, N, K, cfg=100, shape=0)
+    (qa, pa, qb, pb), (oqa, osa, oqb, osb) = quantise_both(w)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
+    dg.dg_fp8_fp4_gemm_nt(qa, pa, qb, pb, None, D)
+    check_close(as_f64(D), oracle.gemm_fp8_fp4_nt(oqa, osa, oqb, osb), "decode full size")
+
+
+def test_fp8_fp4_decode_dropped_arrive_times_out_and_recovers():
+    dg.dg_set_wait_timeout_ns(50_000_000)
+    try:
+        M, N, K = 32, 512, 1024
+        w = wl.dense(M, N, K, cfg=101, shape=3)
+        (qa, pa, qb, pb), (oqa, osa, oqb, osb) = quantise_both(w)
+        D = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
+        dg.dg_debug_drop_next_arrive(True)
+        dg.dg_fp8_fp4_gemm_nt(qa, pa, qb, pb, None, D)
+        st, site = dg.dg_get_last_device_error()
+        assert st == dg.DG_ERR_TIMEOUT and site > 0
+        dg.dg_fp8_fp4_gemm_nt(qa, pa, qb, pb, None, D)
+        assert dg.dg_get_last_device_error() == (dg.DG_OK, 0)
+        check_close(as_f64(D), oracle.gemm_fp8_fp4_nt(oqa, osa, oqb, osb), "after recovery")
+    finally:
+        dg.dg_set_wait_timeout_ns(0)

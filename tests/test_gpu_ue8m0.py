@@ -149,3 +149,37 @@ def test_ue8m0_dropped_arrive_times_out_and_recovers():
         check_close(as_f64(D), oracle.gemm_nt(oqa, osa, oqb, osb), "after recovery")
     finally:
         dg.dg_set_wait_timeout_ns(0)
+
+
+# --------------------------------------------------------------- M <= 128
+# dg_fp8_gemm_nt_ue8m0 routes M <= 128 to the block-scaled decode kernel
+# (swap-AB, cluster split-K).
+@pytest.mark.parametrize("M,N,K,with_c", [(1, 256, 4096, False), (30, 384, 640, True),
+                                          (64, 264, 1536, True), (128, 7168, 2048, False)])
+def test_ue8m0_decode_vs_oracle(M, N, K, with_c):
+    w = wl.dense(M, N, K, cfg=102, shape=M + N + K, with_c=with_c)
+    Cb = synth.to_bf16_bits(w.C) if with_c else None
+    qa, _, pa = dg.dg_quantize_fp8_ue8m0(to_dev(w.A), dg.DG_QUANT_ROW_1x128, with_scales=False)
+    qb, _, pb = dg.dg_quantize_fp8_ue8m0(to_dev(w.B), dg.DG_QUANT_BLOCK_128x128,
+                                         with_scales=False)
+    oqa, osa = oracle.quantize(w.A, oracle.ROW_1x128_POW2)
+    oqb, osb = oracle.quantize(w.B, oracle.BLOCK_128x128_POW2)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
+    dg.dg_fp8_gemm_nt_ue8m0(qa, pa, qb, pb, bf16_dev(Cb) if with_c else None, D)
+    check_close(as_f64(D), oracle.gemm_nt(oqa, osa, oqb, osb, Cb), f"ue8m0 decode {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("minb,splits", [(1, 2), (2, 4), (1, 7)])
+def test_ue8m0_decode_plans(monkeypatch, minb, splits):
+    monkeypatch.setenv("DG_DECODE_MINB", str(minb))
+    monkeypatch.setenv("DG_DECODE_SPLITS", str(splits))
+    M, N, K = 100, 512, 3072
+    w = wl.dense(M, N, K, cfg=103, shape=minb * 10 + splits)
+    qa, _, pa = dg.dg_quantize_fp8_ue8m0(to_dev(w.A), dg.DG_QUANT_ROW_1x128, with_scales=False)
+    qb, _, pb = dg.dg_quantize_fp8_ue8m0(to_dev(w.B), dg.DG_QUANT_BLOCK_128x128,
+                                         with_scales=False)
+    oqa, osa = oracle.quantize(w.A, oracle.ROW_1x128_POW2)
+    oqb, osb = oracle.quantize(w.B, oracle.BLOCK_128x128_POW2)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
+    dg.dg_fp8_gemm_nt_ue8m0(qa, pa, qb, pb, None, D)
+    check_close(as_f64(D), oracle.gemm_nt(oqa, osa, oqb, osb), f"plan {minb}/{splits}")
