@@ -721,6 +721,14 @@ dg_status dispatch_mx_decode(const void* X, const int32_t* sfx, const void* W,
   }
   if (cap1 <= 0 || cap2 <= 0) return DG_ERR_CUDA;
   DecodePlan p = plan_decode(M, n_tiles, KB, sms, cap1, cap2);
+  if (W4 && n_tiles < sms) {
+    // E2M1 weights (from a sweep of both configurations x 1..8 splits over
+    // the decode shapes): two CTAs per SM at every M, and a split keeps at
+    // least 8 K-blocks -- half the weight bytes per K-block leave a split with
+    // fewer K-blocks too little to stream.
+    p.minb = 2;
+    p.splits = std::max(1, std::min(std::min(2 * sms / n_tiles, KB / 8), std::min(4, cap2)));
+  }
   if (const char* e = std::getenv("DG_DECODE_MINB")) {
     const int f = std::atoi(e);
     if (f == 1 || f == 2) p.minb = f;
