@@ -149,11 +149,17 @@ dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void* A, const float* sfa, c
  *   masked_m [G] int32 device array, read on the device; values are clamped
  *            to [0, max_m].
  *   D        [G][max_m][N] BF16; rows m >= masked_m[g] are left untouched.
+ *   expected_m  host-side hint, the typical number of valid rows per group
+ *            (same section: the call takes an expected M because the counts
+ *            are only known on the device). It only steers the tile-width
+ *            choice; results do not depend on it. <= 0 means unknown (plan for
+ *            max_m); values above max_m count as max_m.
  * G <= 1024.
  * ------------------------------------------------------------------------- */
 dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* A, const float* sfa, const void* B,
                                           const float* sfb, const int32_t* masked_m, void* D,
-                                          int G, int max_m, int N, int K, void* stream);
+                                          int G, int max_m, int expected_m, int N, int K,
+                                          void* stream);
 
 /* ---------------------------------------------------------------------------
  * K-grouped GEMM, TN, contiguous along K (MoE weight gradient).

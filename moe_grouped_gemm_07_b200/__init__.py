@@ -55,7 +55,7 @@ _lib.dg_fp8_gemm_nt.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, 
 _lib.dg_m_grouped_fp8_gemm_nt_contiguous.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                                      _i32, _i32, _i32, _vp]
 _lib.dg_m_grouped_fp8_gemm_nt_masked.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
-                                                 _i32, _vp]
+                                                 _i32, _i32, _vp]
 _lib.dg_k_grouped_fp8_gemm_tn_contiguous.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                                      _i32, _i32, _vp]
 _lib.dg_k_grouped_fp8_gemm_tn_contiguous_dev_ks.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _vp,
@@ -202,9 +202,11 @@ def dg_m_grouped_fp8_gemm_nt_contiguous(A, sfa, B, sfb, m_indices, C, D, stream=
     return D
 
 
-def dg_m_grouped_fp8_gemm_nt_masked(A, sfa, B, sfb, masked_m, D, stream=None):
+def dg_m_grouped_fp8_gemm_nt_masked(A, sfa, B, sfb, masked_m, D, expected_m=None, stream=None):
     """A [G,max_m,K], sfa [G, K/128, align4(max_m)], B [G,N,K],
-    sfb [G, ceil(N/128), K/128], masked_m [G] int32, D [G,max_m,N] bf16."""
+    sfb [G, ceil(N/128), K/128], masked_m [G] int32, D [G,max_m,N] bf16.
+    expected_m: optional host hint of the typical valid rows per group (plans
+    the tile width only; None = plan for max_m)."""
     _cuda_contig(A, sfa, B, sfb, masked_m, D)
     G, max_m, K = A.shape
     G2, N, K2 = B.shape
@@ -216,8 +218,8 @@ def dg_m_grouped_fp8_gemm_nt_masked(A, sfa, B, sfb, masked_m, D, stream=None):
           "sfb")
     _check("dg_m_grouped_fp8_gemm_nt_masked",
            _lib.dg_m_grouped_fp8_gemm_nt_masked(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb),
-                                                _ptr(masked_m), _ptr(D), G, max_m, N, K,
-                                                _stream(stream)))
+                                                _ptr(masked_m), _ptr(D), G, max_m,
+                                                int(expected_m or 0), N, K, _stream(stream)))
     return D
 
 

@@ -269,11 +269,14 @@ template <int MODE>
 dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, const float* sfb,
                  const int32_t* m_indices, const int32_t* masked_m, const void* C, void* D,
                  int rows_total, int M_logical, int N, int K, int G, long long m_blocks_bound,
-                 long long tiles_if_known, cudaStream_t st, const char* name) {
+                 long long tiles_if_known, cudaStream_t st, const char* name,
+                 long long m_blocks_plan = -1) {
   int dev = 0, sms = 0;
   dg_status s = device_sms(&dev, &sms);
   if (s != DG_OK) return s;
-  const int bn = choose_bn(m_blocks_bound, N, sms);
+  // the tile width is planned for the expected number of 128-row blocks
+  // (masked: the caller's expected_m hint), the launch for the bound
+  const int bn = choose_bn(m_blocks_plan > 0 ? m_blocks_plan : m_blocks_bound, N, sms);
   CUtensorMap ta, tb, dummy;
   std::memset(&dummy, 0, sizeof dummy);
   s = make_map_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, rows_total, K, 128, 128,
@@ -1181,7 +1184,8 @@ dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void* A, const float* sfa, c
 
 dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* A, const float* sfa, const void* B,
                                           const float* sfb, const int32_t* masked_m, void* D,
-                                          int G, int max_m, int N, int K, void* stream) {
+                                          int G, int max_m, int expected_m, int N, int K,
+                                          void* stream) {
   if (G < 1 || max_m < 0 || N < 0 || K < 0) return DG_ERR_INVALID_ARG;
   if (G > dg::kMaxMaskedGroups || K % 128 != 0 || N % 8 != 0 || K == 0)
     return DG_ERR_UNSUPPORTED_SHAPE;
@@ -1195,9 +1199,11 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* A, const float* sfa, const
     return DG_ERR_UNSUPPORTED_SHAPE;
   const int ld = (max_m + 3) / 4 * 4;
   const long long mb_bound = static_cast<long long>(G) * ((max_m + 127) / 128);
+  const int em = expected_m <= 0 ? max_m : std::min(expected_m, max_m);
+  const long long mb_plan = static_cast<long long>(G) * ((em + 127) / 128);
   return run_nt<dg::MODE_MASKED>(A, sfa, ld, B, sfb, nullptr, masked_m, nullptr, D, G * max_m,
                                  max_m, N, K, G, mb_bound, -1, static_cast<cudaStream_t>(stream),
-                                 "m_grouped_fp8_gemm_nt_masked");
+                                 "m_grouped_fp8_gemm_nt_masked", mb_plan);
 }
 
 dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void* A, const float* sfa, const void* B,

@@ -10,16 +10,18 @@
 // applied: acc += sfa * sfb * P_kb.
 //
 // CTA = 320 threads, one CTA per SM, persistent over output tiles:
-//   warp 0      TMA producer: A/B tiles (128B-swizzled) into an S-stage ring
-//               (plus, for K-grouped, the per-K-block scale vectors); the
-//               warp runs the loop, lane 0 issues.
+//   warp 0      TMA producer: A/B tiles (128B-swizzled) into an S-stage ring,
+//               and the per-K-block scales into a ring of their own (the
+//               tile's 128 sfa values by bulk copy; for K-grouped, the sfa
+//               and sfb vectors by TMA); the warp runs the loop, lane 0 issues.
 //   warp 1      TMEM allocator + tcgen05.mma issuer (lane 0 of the converged
 //               warp): for each
 //               K-block, 4 x (M=128, N=BN, K=32) MMAs into one of 512/BN TMEM
 //               accumulator buffers (all 512 columns), reset per K-block.
 //   warps 2..9  promotion / epilogue: warp w reads TMEM lane quadrant (w % 4)
-//               and column half ((w - 2) / 4); acc += s * P in registers;
-//               at tile end adds C, converts and stores D.
+//               and column half ((w - 2) / 4); acc += s * P in registers
+//               (NT: s = sfa from the scale ring x sfb read one K-block
+//               ahead); at tile end adds C, converts and stores D.
 // The MMA runs up to 512/BN - 1 K-blocks ahead of the promotion (2 buffers at
 // BN=256, 4 at BN=128); the producer runs up to S K-blocks ahead.
 #pragma once
@@ -99,13 +101,12 @@ struct GemmCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_SCALE = OFF_B + STAGES * B_BYTES;
-  // NT modes: per promotion warp, a ring of SRING K-blocks of scales (32 sfa
-  // values for the warp's rows + 1 sfb value for its column half), filled by
-  // cp.async SRING K-blocks ahead
-  static constexpr int SRING = 8;
-  static constexpr int SRING_FLOATS = 8 * SRING * 33;
+  // NT modes: a ring of SCALE_SLOTS K-blocks of sfa for the tile's BM rows,
+  // filled by the producer's bulk copies (the sfb value of a column half is
+  // one float per K-block, read by the promotion warps themselves)
+  static constexpr int NT_SCALE_BYTES = BM * 4;
   static constexpr int OFF_STAGE =
-      ((OFF_SCALE + (KG ? SCALE_SLOTS * SCALE_BYTES : SRING_FLOATS * 4) + 1023) / 1024) * 1024;
+      ((OFF_SCALE + SCALE_SLOTS * (KG ? SCALE_BYTES : NT_SCALE_BYTES) + 1023) / 1024) * 1024;
   // output staging for the TMA-store epilogue: one 32-row x 64-byte chunk
   // (32 bf16 or 16 fp32 columns) per promotion warp, 64-byte swizzled
   static constexpr int STAGE_BYTES_PER_WARP = 32 * 64;
@@ -447,7 +448,7 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t s = it % S;
           bool ok = mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort_flag, tmo, SITE_PRODUCER_EMPTY);
           if (!__all_sync(0xffffffffu, ok)) goto producer_done;
-          if constexpr (Cfg::KG) {
+          {
             // take the scale slot before arming anything, so an abort here
             // leaves no uncounted copy in flight
             const uint32_t ss = sit % SS;
@@ -491,8 +492,26 @@ __global__ void __launch_bounds__(320, 1)
               tma_load_2d(slot, &tm_sfa, &sfull[ss], tl.m0, tl.kb0 + kb);
               tma_load_2d(slot + Cfg::BM, &tm_sfb, &sfull[ss], tl.n0, tl.kb0 + kb);
             }
-            ++sit;
+          } else {
+            // sfa of the tile's rows for this K-block: BM contiguous floats of
+            // the MN-major [K/128][ld] layout ([G][K/128][ld] when masked),
+            // cut at ld so the copy stays inside the tensor (ld % 4 == 0, so
+            // the size is a multiple of 16 bytes); rows the copy leaves out
+            // lie past M and get zero scales in the promotion
+            const uint32_t ss = sit % SS;
+            if (lane == 0) {
+              const int nrows = min(Cfg::BM, args.ld_sfa - tl.m0);
+              const uint32_t bytes = nrows > 0 ? static_cast<uint32_t>(nrows) * 4u : 0u;
+              mbar_arrive_expect_tx(&sfull[ss], bytes);
+              if (bytes > 0) {
+                long long off = static_cast<long long>(tl.kb0 + kb) * args.ld_sfa + tl.m0;
+                if constexpr (MODE == MODE_MASKED)
+                  off += static_cast<long long>(tl.g) * (args.K / Cfg::BK) * args.ld_sfa;
+                bulk_load(sScale + ss * Cfg::BM, args.sfa + off, bytes, &sfull[ss]);
+              }
+            }
           }
+          ++sit;
           __syncwarp();
         }
       }
@@ -507,11 +526,9 @@ __global__ void __launch_bounds__(320, 1)
         volatile int never = 0;
         mbar_wait(&full[j % S], (j / S) & 1, &never, tmo, SITE_TEARDOWN_TMA);
       }
-      if constexpr (Cfg::KG) {
-        for (uint32_t j = (sit > SS ? sit - SS : 0); j < sit; ++j) {
-          volatile int never = 0;
-          mbar_wait(&sfull[j % SS], (j / SS) & 1, &never, tmo, SITE_TEARDOWN_TMA);
-        }
+      for (uint32_t j = (sit > SS ? sit - SS : 0); j < sit; ++j) {
+        volatile int never = 0;
+        mbar_wait(&sfull[j % SS], (j / SS) & 1, &never, tmo, SITE_TEARDOWN_TMA);
       }
     }
     __syncwarp();
@@ -607,48 +624,27 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int j = 0; j < EC; ++j) acc[j] = 0.0f;
 
-      // NT scale streams: sfa for this thread's row, sfb for its column half,
-      // prefetched 4 K-blocks ahead in registers.
+      // NT scales: sfa of the tile's rows arrives per K-block in the shared
+      // ring the producer fills; sfb (one value per K-block for this warp's
+      // column half, consecutive floats unless B is stored [K][N]) is read
+      // here, one K-block ahead.
       // (rows past M and column halves past N get zero scales; they are
       // never stored, and their scale rows may not exist)
-      const float* pa = args.sfa;
-      const float* pb = args.sfb;
+      int pb = 0;  // offset of this column half's first sfb value (sfb < 2^31 floats)
       bool row_in = false, half_in = false;
+      float sb_next = 0.f;
+      auto sfb_at = [&](int kb) {
+        if constexpr (Cfg::B_MN) return __ldg(args.sfb + pb + kb * nbN);
+        else return __ldg(args.sfb + pb + kb);
+      };
       if constexpr (!Cfg::KG) {
-        const int m_local = tl.m0 + r_in_tile;
-        row_in = m_local < args.M;
-        if constexpr (MODE == MODE_MASKED)
-          pa = args.sfa + static_cast<long long>(tl.g) * KBn * args.ld_sfa + m_local;
-        else
-          pa = args.sfa + m_local;
+        row_in = tl.m0 + r_in_tile < args.M;
         const int col_first = tl.n0 + static_cast<int>(h) * EC;
         half_in = col_first < args.N;
         // sfb is [G][ceil(N/128)][K/128], or [K/128][ceil(N/128)] for B stored [K][N]
-        pb = Cfg::B_MN ? args.sfb + col_first / 128
-                       : args.sfb + (static_cast<long long>(tl.g) * nbN + col_first / 128) * KBn;
-        if constexpr (SPLITK) {  // this part starts at K-block kb0
-          pa += static_cast<long long>(tl.kb0) * args.ld_sfa;
-          pb += tl.kb0;
-        }
-      }
-      // NT scales stream through this warp's shared-memory ring by cp.async,
-      // SRING K-blocks ahead: lane l copies sfa for its row, lane 0 also the
-      // sfb value of the warp's column half. Every iteration commits exactly
-      // one cp.async group, so wait_group<SRING-1> means "K-block kb landed".
-      constexpr int SR = Cfg::SRING;
-      float* ring = reinterpret_cast<float*>(sScale) + (warp - 2) * (SR * 33);
-      auto issue_scales = [&](int kb) {
-        if (kb < tl.nkb) {
-          float* slot = ring + (kb % SR) * 33;
-          if (row_in) cp_async_4(slot + lane, pa + static_cast<long long>(kb) * args.ld_sfa);
-          if (lane == 0 && half_in)
-            cp_async_4(slot + 32, pb + (Cfg::B_MN ? static_cast<long long>(kb) * nbN : kb));
-        }
-        cp_async_commit();
-      };
-      if constexpr (!Cfg::KG) {
-#pragma unroll 1
-        for (int u = 0; u < SR; ++u) issue_scales(u);
+        pb = Cfg::B_MN ? col_first / 128 : (tl.g * nbN + col_first / 128) * KBn;
+        if constexpr (SPLITK) pb += tl.kb0;  // this part starts at K-block kb0
+        if (half_in && tl.nkb > 0) sb_next = sfb_at(0);
       }
 
       for (int kb = 0; kb < tl.nkb; ++kb) {
@@ -658,12 +654,16 @@ __global__ void __launch_bounds__(320, 1)
         if (!ok) goto epi_done;
         tc_fence_after();
         if constexpr (!Cfg::KG) {
-          cp_async_wait<SR - 1>();
+          const uint32_t ss = sit % SS;
+          bool ok2 = mbar_wait(&sfull[ss], (sit / SS) & 1, abort_flag, tmo, SITE_EPI_SCALE_FULL);
+          ok2 = __all_sync(0xffffffffu, ok2);
+          if (!ok2) goto epi_done;
+          const float sa = row_in ? sScale[ss * Cfg::BM + r_in_tile] : 0.f;
           __syncwarp();
-          const float* slot = ring + (kb % SR) * 33;
-          const float sc = (row_in ? slot[lane] : 0.f) * (half_in ? slot[32] : 0.f);
-          __syncwarp();
-          issue_scales(kb + SR);
+          if (lane == 0) mbar_arrive(&sempty[ss]);  // the slot may be refilled
+          ++sit;
+          const float sc = sa * sb_next;
+          sb_next = (half_in && kb + 1 < tl.nkb) ? sfb_at(kb + 1) : 0.f;
           auto release_tmem = [&]() {
             tc_fence_before();
             __syncwarp();
@@ -738,7 +738,6 @@ __global__ void __launch_bounds__(320, 1)
         }
         ++acc_it;
       }
-      if constexpr (!Cfg::KG) cp_async_wait<0>();
 
       // ------------------------------------------------ split-K tail
       if constexpr (SPLITK) {
@@ -903,7 +902,6 @@ __global__ void __launch_bounds__(320, 1)
         cluster_sync_all();
       }
     }
-    cp_async_wait<0>();  // no shared-memory copy may land after the CTA exits
     if (lane == 0) bulk_wait0();  // every TMA store of this warp has completed
     __syncwarp();
   }

@@ -73,10 +73,13 @@ def test_host_validation_before_any_cuda_call():
                                                  8, 128, 2, None) == dg.DG_ERR_UNSUPPORTED_SHAPE
     assert L.dg_m_grouped_fp8_gemm_nt_contiguous(fake, fake, fake, fake, fake, None, fake, 128,
                                                  8, 128, 0, None) == dg.DG_ERR_INVALID_ARG
-    assert L.dg_m_grouped_fp8_gemm_nt_masked(fake, fake, fake, fake, fake, fake, 2000, 64, 8,
+    assert L.dg_m_grouped_fp8_gemm_nt_masked(fake, fake, fake, fake, fake, fake, 2000, 64, 0, 8,
                                              128, None) == dg.DG_ERR_UNSUPPORTED_SHAPE
-    assert L.dg_m_grouped_fp8_gemm_nt_masked(fake, fake, fake, fake, fake, fake, 0, 64, 8,
+    assert L.dg_m_grouped_fp8_gemm_nt_masked(fake, fake, fake, fake, fake, fake, 0, 64, 0, 8,
                                              128, None) == dg.DG_ERR_INVALID_ARG
+    # expected_m is a hint only: any value passes validation
+    assert L.dg_m_grouped_fp8_gemm_nt_masked(fake, fake, fake, fake, fake, fake, 2, 0, -5, 8,
+                                             128, None) == dg.DG_OK
     ks = (ctypes.c_int * 2)(128, 100)
     assert L.dg_k_grouped_fp8_gemm_tn_contiguous(fake, fake, fake, fake, ks, None, fake, 2, 16,
                                                  16, None) == dg.DG_ERR_UNSUPPORTED_SHAPE

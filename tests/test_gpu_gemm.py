@@ -193,6 +193,29 @@ def test_masked_vs_oracle(G, max_m, N, K):
         assert np.all(raw[g, w.masked_m[g]:] == SENTINEL), f"group {g}: masked rows written"
 
 
+def test_masked_expected_m_hint_changes_plan_not_results():
+    """expected_m only steers the host's tile-width plan. For 8 groups of up
+    to 1024 rows, N=1024, the bound (64 row blocks) plans 128x256 tiles and
+    the hint expected_m=128 (8 row blocks) plans 128x128 tiles; the results
+    must be bit-identical and meet the bar."""
+    G, max_m, N, K = 8, 1024, 1024, 256
+    w = wl.masked(G=G, max_m=max_m, N=N, K=K, lo=1, hi=128, cfg=86)
+    qa, sa = dg.dg_quantize_fp8(to_dev(w.A), dg.DG_QUANT_ROW_1x128)
+    qb, sb = dg.dg_quantize_fp8(to_dev(w.B), dg.DG_QUANT_BLOCK_128x128)
+    mm = to_dev(w.masked_m)
+    outs = []
+    for hint in (None, 128, 1, 5000):
+        D = sentinel_bf16((G, max_m, N))
+        dg.dg_m_grouped_fp8_gemm_nt_masked(qa, sa, qb, sb, mm, D, expected_m=hint)
+        outs.append(D)
+    for D in outs[1:]:
+        assert torch.equal(D.view(torch.int16), outs[0].view(torch.int16))
+    oqa, osa = oracle.quantize(w.A, oracle.ROW_1x128)
+    oqb, osb = oracle.quantize(w.B, oracle.BLOCK_128x128)
+    check_close(as_f64(outs[1]), oracle.m_grouped_masked(oqa, osa, oqb, osb, w.masked_m),
+                "masked with hint")
+
+
 def test_masked_counts_above_max_are_clamped():
     G, max_m, N, K = 2, 128, 128, 128
     w = wl.masked(G=G, max_m=max_m, N=N, K=K, cfg=85)
