@@ -532,6 +532,24 @@ def run_fp8fp4(args):
     return 0
 
 
+# ----------------------------------------------------------------- ranks
+def max_over_ranks(dist, values, device):
+    """Element-wise maximum of per-rank timings (ms); every rank calls it in
+    the same order. Identity on one process (dist None)."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_tflops(world, flops_per_rank_step, ms_per_step):
+    """Whole-job throughput of `world` replicas that each do
+    `flops_per_rank_step` per step, timed by the slowest rank."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -635,10 +653,7 @@ def run_ours(args):
     t_q /= split_steps
     t_g /= split_steps
     ms_outer = outer0.elapsed_time(outer1) / args.steps
-    if dist:
-        t = torch.tensor([ms_step, ms_outer], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, ms_outer = float(t[0]), float(t[1])
+    ms_step, ms_outer = max_over_ranks(dist, [ms_step, ms_outer], device)
 
     # ---- end to end through the public API with host buffers
     if args.quick:
@@ -679,10 +694,7 @@ def run_ours(args):
     e1.record()
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1) / e2e_steps
-    if dist:
-        t = torch.tensor([ms_e2e], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t[0])
+    ms_e2e, = max_over_ranks(dist, [ms_e2e], device)
 
     flops_step = sum(shape_flops(*s) for s in shapes)
     pk = peaks()
@@ -717,7 +729,7 @@ def run_ours(args):
                     "shapes": "M in {64,128} (12 decode shapes), GEMM kernel only"}
 
     line = {
-        "metric": METRIC, "value": round(world * flops_step / (ms_step * 1e-3) / 1e12, 2),
+        "metric": METRIC, "value": round(job_tflops(world, flops_step, ms_step), 2),
         "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32 accumulate, bf16 out",
@@ -733,7 +745,7 @@ def run_ours(args):
         "fp8_pct_of_nominal_peak": round(100 * flops_step / (ms_step * 1e-3) / 1e12
                                          / NOMINAL_FP8_TFLOPS, 2),
         "roofline": roofline, "roofline_hbm": roofline_hbm,
-        "e2e": {"value": round(world * flops_step / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        "e2e": {"value": round(job_tflops(world, flops_step, ms_e2e), 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e, 3)},
         "gpu_launches": int(launches), "gpu_launches_per_step": int(launches // max(args.steps, 1)),
