@@ -311,6 +311,21 @@ void dg_debug_drop_next_arrive(int enable);
 /* Number of kernels this library has launched since load (all devices). */
 uint64_t dg_get_launch_count(void);
 
+/* Environment variables (README summary, section "ユーティリティと環境変数",
+ * names its DG_PRINT_CONFIGS; the rest override this library's planner, for
+ * comparisons; none is needed for correct results):
+ *   DG_PRINT_CONFIGS=1   print each launch's plan (tiles, widths, splits) to
+ *                        stderr; read once.
+ *   DG_FORCE_BN=128|256  tile width of the M > 128 dense and grouped kernels;
+ *                        read once.
+ *   DG_TAIL_SPLIT=0      no split-K launch for a dense call's partial last
+ *                        wave; read once.
+ *   DG_PAIR=1            dense M > 128 on CTA pairs (256-row tiles); read once.
+ *   DG_PAIR_BN=128|256   tile width of the pair kernel; read once.
+ *   DG_DECODE_MINB=1|2, DG_DECODE_SPLITS=s
+ *                        CTAs per SM and split count of the M <= 128 kernels;
+ *                        read on every call. */
+
 #ifdef __cplusplus
 }
 #endif

@@ -11,6 +11,10 @@
 // (The pages' promotion exists because Hopper's FP8 accumulator is imprecise;
 // this path measures what the B200 tensor core's own accumulation gives.)
 //
+// The FP4B instantiation is the FP8 x FP4 GEMM: B in E2M1 with one UE8M0
+// scale per 1x32 K-strip of each row (see MxCfgT for its tile and scale
+// layout); A keeps E4M3 with 1x128 power-of-two scales.
+//
 // Packed scale layout (written by the UE8M0 quantiser): for an operand with
 // R rows (M for A, N for B) and K columns,
 //   packed[q][rb][i][j]  (int32, q < ceil(K/512), rb < ceil(R/128), i < 32, j < 4)
