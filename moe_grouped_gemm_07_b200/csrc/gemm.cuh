@@ -710,26 +710,26 @@ __global__ void __launch_bounds__(320, 1)
           const float* slot = sScale + ss * (Cfg::BM + BN);
           const float sav = slot[r_in_tile];
           const float* sbv = slot + Cfg::BM + h * EC;
+          constexpr int KC = 16;  // columns per TMEM load (fewer live registers)
 #pragma unroll
-          for (int c = 0; c < EC / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(t_lane + b * BN + h * EC + c * 32, r);
+          for (int c = 0; c < EC / KC; ++c) {
+            uint32_t r[KC];
+            tmem_ld_32x32b<KC>(t_lane + b * BN + h * EC + c * KC, r);
             tmem_ld_wait();
-            if (c == EC / 32 - 1) {
+            if (c == EC / KC - 1) {
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&tempty[b]);
             }
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const float4 sb4 = *reinterpret_cast<const float4*>(sbv + c * 32 + i);
-              float t0, t1, t2, t3;
-              mul2(t0, t1, sav, sav, sb4.x, sb4.y);
-              mul2(t2, t3, sav, sav, sb4.z, sb4.w);
-              fma2(acc[c * 32 + i], acc[c * 32 + i + 1], t0, t1, __uint_as_float(r[i]),
-                   __uint_as_float(r[i + 1]));
-              fma2(acc[c * 32 + i + 2], acc[c * 32 + i + 3], t2, t3, __uint_as_float(r[i + 2]),
-                   __uint_as_float(r[i + 3]));
+            for (int i = 0; i < KC; i += 4) {
+              // acc += sav * (sb * P): the column-scaled products reuse P's registers
+              const float4 sb4 = *reinterpret_cast<const float4*>(sbv + c * KC + i);
+              float u0, u1, u2, u3;
+              mul2(u0, u1, sb4.x, sb4.y, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+              mul2(u2, u3, sb4.z, sb4.w, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+              fma2(acc[c * KC + i], acc[c * KC + i + 1], sav, sav, u0, u1);
+              fma2(acc[c * KC + i + 2], acc[c * KC + i + 3], sav, sav, u2, u3);
             }
           }
           __syncwarp();
