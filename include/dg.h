@@ -90,6 +90,9 @@ dg_status dg_quantize_fp8(const void* x, int in_dtype, int batch, int rows, int 
  *   D    [M][N] BF16, rounded to nearest even from the FP32 accumulator.
  * Shapes: M >= 0, N >= 0 (either 0: no-op), K % 128 == 0 (K == 0: D = C),
  * N % 8 == 0.
+ * M <= 128 (decode) runs a swap-AB kernel with split-K over a thread-block
+ * cluster; its partial sums are added in a fixed order, so results repeat
+ * bit for bit from run to run.
  * ------------------------------------------------------------------------- */
 dg_status dg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb,
                          const void* C, void* D, int M, int N, int K, void* stream);
@@ -207,7 +210,8 @@ dg_status dg_quantize_fp8_ue8m0(const void* x, int in_dtype, int rows, int cols,
 /* Dense NT GEMM on the block-scaled MMA: D = C + A @ B.T with sfa / sfb the
  * packed UE8M0 scales of A (ROW mode, rows = M) and B (BLOCK mode, rows = N)
  * from dg_quantize_fp8_ue8m0. A [M][K], B [N][K] E4M3; C [M][N] BF16 or NULL
- * (may alias D); D [M][N] BF16. K % 128 == 0, N % 8 == 0. */
+ * (may alias D); D [M][N] BF16. K % 128 == 0, N % 8 == 0. M <= 128 runs a
+ * swap-AB kernel with split-K over a cluster (partials added in rank order). */
 dg_status dg_fp8_gemm_nt_ue8m0(const void* A, const int32_t* sfa, const void* B,
                                const int32_t* sfb, const void* C, void* D, int M, int N, int K,
                                void* stream);
@@ -246,7 +250,9 @@ dg_status dg_fp8_gemm_nt_ue8m0(const void* A, const int32_t* sfa, const void* B,
  *       dg_quantize_fp4_e2m1 (rows = N); B 32-byte aligned;
  *   C   [M][N] BF16 or NULL (may alias D); D [M][N] BF16.
  *   K % 128 == 0, N % 8 == 0. Accumulation is the tensor core's FP32 across
- *   all K (no per-K-block promotion). Errors as dg_fp8_gemm_nt_ue8m0.
+ *   all K (no per-K-block promotion). M <= 128 runs the block-scaled swap-AB
+ *   split-K kernel, as dg_fp8_gemm_nt_ue8m0 does. Errors as
+ *   dg_fp8_gemm_nt_ue8m0.
  * ------------------------------------------------------------------------- */
 dg_status dg_quantize_fp4_e2m1(const void* x, int in_dtype, int rows, int cols, void* codes,
                                float* scales, int32_t* packed, void* stream);
