@@ -129,3 +129,13 @@ def test_fp4_entry_validation_before_any_cuda_call():
     assert g(None, None, None, None, None, None, 0, 8, 128, None) == dg.DG_OK
     # the packed E2M1 operand must be 32-byte aligned (4-bit TMA loads)
     assert g(fake, fake, vp(0x1010), fake, None, fake, 8, 8, 128, None) == dg.DG_ERR_MISALIGNED
+
+
+def test_every_environment_variable_read_is_documented():
+    import re as _re
+    src = os.path.join(ROOT, "moe_grouped_gemm_07_b200", "csrc", "dg_api.cu")
+    read = set(_re.findall(r'getenv\("(DG_[A-Z_]+)"\)', open(src).read()))
+    assert read, "no environment variables found"
+    header = open(HEADER).read()
+    missing = sorted(v for v in read if v not in header)
+    assert not missing, missing
