@@ -125,3 +125,26 @@ def test_gemm_reduces_to_matmul(M, N, K, with_c):
     np.testing.assert_allclose(R, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
     rows = [M - 1, 0, M // 2]
     assert np.array_equal(oracle.gemm_fp8_fp4_nt(A, sfa, B, sfb, C, rows=rows), R[rows])
+
+
+def test_gemm_equals_fp8_gemm_when_fp4_values_are_fp8_values():
+    """Every E2M1 value is exactly an E4M3 value. With B's four 1x32 scales of
+    each 128-block equal (per row, per K-block) and the same across the rows
+    of each 128-row block, the FP8 x FP4 GEMM must equal the FP8 x FP8 GEMM
+    on the same values with that block scale, element for element."""
+    rng = np.random.default_rng(77)
+    M, N, K = 7, 130, 256
+    A = rng.integers(0, 256, (M, K), dtype=np.uint8)
+    A[(A & 0x7F) == 0x7F] = 0x40
+    nib = rng.integers(0, 16, (N, K), dtype=np.uint8)
+    B4 = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    # the same values as E4M3 codes, via the oracle's own encoder
+    vals = lib_decode(nib)
+    B8 = np.array([[oracle.e4m3_encode(v) for v in row] for row in vals], dtype=np.uint8)
+    assert np.array_equal(_e4m3(B8), vals)
+    sfa = np.ldexp(1.0, rng.integers(-4, 5, (K // 128, M + 1))).astype(np.float32)
+    sfb8 = np.ldexp(1.0, rng.integers(-4, 5, ((N + 127) // 128, K // 128))).astype(np.float32)
+    sfb4 = np.repeat(np.repeat(sfb8, 128, axis=0)[:N], 4, axis=1)  # [N][K/32]
+    R4 = oracle.gemm_fp8_fp4_nt(A, sfa, B4, np.ascontiguousarray(sfb4))
+    R8 = oracle.gemm_nt(A, sfa, B8, sfb8)
+    np.testing.assert_allclose(R4, R8, rtol=1e-13, atol=1e-13 * np.abs(R8).max())
