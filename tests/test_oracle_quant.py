@@ -9,7 +9,12 @@ What is pinned and by what:
     of 3 mantissa bits, or half the subnormal step);
   * the amax element always lands on +-448;
   * all-zero strips (scale floor 1e-4/448, codes zero), ragged 128x128 blocks,
-    bf16 inputs.
+    bf16 inputs;
+  * the quotient itself, in all three modes: scales recomputed with numpy's
+    float32 division and codes equal to torch's cast of numpy's float32 x / s
+    (clipped to +-448), on N(0,1) data, heavy tails and zeros, and values on
+    s x midpoint rounding boundaries where multiplying by 1 / s instead would
+    change codes (the case set checks that it does).
 """
 import numpy as np
 import pytest
@@ -208,3 +213,127 @@ def test_pow2_scales_dequantise_within_bound():
     codes, s = oracle.quantize(x, oracle.ROW_1x128_POW2)
     sf = np.repeat(s[:, :64].T, 128, axis=1)
     assert dequant_err_ok(x, codes, sf)
+
+
+# ------------------------------------------------------------ the quotient x / s
+# The scale rule fixes s = max(amax, 1e-4) / 448 and code = E4M3_RN_sat(x / s),
+# both IEEE float32 divisions. These pins recompute s and the quotient with
+# numpy's float32 division (IEEE round-to-nearest) and encode with torch's
+# float8_e4m3fn cast (a library routine), after clipping to +-448 as the
+# saturating encoder does; neither side shares code with the oracle.
+def _groups_to_layout(g, mode, n_groups):
+    """g [n_groups, 128 * 128 or 128]: one quantisation group per row, element
+    0 first. Returns x laid out so that every group is one strip (ROW), one
+    128x128 block (BLOCK) or one 128-row column strip (COL)."""
+    if mode == oracle.ROW_1x128:
+        return g.reshape(n_groups, 128)
+    if mode == oracle.COL_128x1:
+        return np.ascontiguousarray(g.reshape(n_groups, 128).T)
+    # BLOCK: n_groups blocks side by side along the columns
+    return np.ascontiguousarray(g.reshape(n_groups, 128, 128).transpose(1, 0, 2).reshape(128, -1))
+
+
+def _numpy_scales(x, mode):
+    """Element-wise float32 scale of x under `mode`, computed in numpy."""
+    rows, cols = x.shape
+    a = np.abs(x)
+    if mode == oracle.ROW_1x128:
+        amax = a.reshape(rows, cols // 128, 128).max(axis=2)
+        s = (np.maximum(amax, F32(1e-4)).astype(F32) / F32(448.0)).astype(F32)
+        return np.repeat(s, 128, axis=1)
+    if mode == oracle.COL_128x1:
+        amax = a.reshape(rows // 128, 128, cols).max(axis=1)
+        s = (np.maximum(amax, F32(1e-4)).astype(F32) / F32(448.0)).astype(F32)
+        return np.repeat(s, 128, axis=0)
+    nb = (rows + 127) // 128
+    pad = np.zeros((nb * 128, cols), dtype=F32)
+    pad[:rows] = a
+    amax = pad.reshape(nb, 128, cols // 128, 128).max(axis=(1, 3))
+    s = (np.maximum(amax, F32(1e-4)).astype(F32) / F32(448.0)).astype(F32)
+    return np.repeat(np.repeat(s, 128, axis=0), 128, axis=1)[:rows]
+
+
+def _expected_codes(x, s):
+    y = (x.astype(F32) / s).astype(F32)              # IEEE float32 quotient
+    return torch_e4m3(np.clip(y, F32(-448.0), F32(448.0)))
+
+
+def _check_quotient(x, mode):
+    codes, sf = oracle.quantize(x, mode)
+    s = _numpy_scales(x, mode)
+    if mode == oracle.ROW_1x128:
+        got_s = np.repeat(sf[:, :x.shape[0]].T, 128, axis=1)
+    elif mode == oracle.COL_128x1:
+        got_s = np.repeat(sf, 128, axis=0)
+    else:
+        got_s = np.repeat(np.repeat(sf, 128, axis=0), 128, axis=1)[:x.shape[0]]
+    assert np.array_equal(got_s.view(np.uint32), s.view(np.uint32))
+    assert np.array_equal(codes, _expected_codes(x, s))
+
+
+MODES3 = [oracle.ROW_1x128, oracle.BLOCK_128x128, oracle.COL_128x1]
+
+
+@pytest.mark.parametrize("mode", MODES3)
+def test_quotient_codes_random(mode):
+    """N(0,1) data, a ragged 128x128 block in BLOCK mode (200 rows)."""
+    rows = 200 if mode == oracle.BLOCK_128x128 else 256
+    x = synth.normal((rows, 512), synth.seed(9, 10, mode))
+    _check_quotient(x, mode)
+
+
+@pytest.mark.parametrize("mode", MODES3)
+def test_quotient_codes_heavy_tails(mode):
+    """Heavy tails and zeros: scales spread over many binades, strips under
+    the 1e-4 floor, float32 subnormals, exact zeros and negative zeros."""
+    u = (synth.u64(256 * 512, synth.seed(9, 11, mode)) >> np.uint64(11)).astype(np.float64)
+    e = (np.floor(u / 2.0 ** 53 * 80.0) - 60.0).reshape(256, 512)   # binades 2^-60 .. 2^19
+    x = (synth.normal((256, 512), synth.seed(9, 12, mode)) * np.ldexp(1.0, e.astype(np.int64))
+         ).astype(F32)
+    x[:, 0:128:3] = F32(0.0)
+    x[:, 1:128:5] = F32(-0.0)
+    x[7] = F32(0.0)                                     # all-zero row / strips
+    x[9, :] = np.float32(1e-40)                         # float32 subnormals, under the floor
+    x[11, 128:256] = F32(3e30)
+    x[11, 130] = F32(1e-30)                             # underflows to a zero code
+    _check_quotient(x, mode)
+
+
+def _boundary_groups(n_groups, gsize, seed):
+    """Groups whose element 0 is a random amax (so s is not a power of two)
+    and whose other elements sit within four float32 ulps of s times an E4M3
+    rounding boundary (a midpoint between neighbouring codes), either sign."""
+    t = oracle.e4m3_table()
+    pos = np.array(sorted(set(float(v) for v in t[:0x7F])))
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(F32)
+    n = n_groups * gsize
+    u = synth.u64(3 * n + 2 * n_groups, seed)
+    amax = np.ldexp(0.5 + (u[:n_groups] >> np.uint64(11)).astype(np.float64) / 2.0 ** 53,
+                    (u[n_groups:2 * n_groups] % np.uint64(40)).astype(np.int64) - 20).astype(F32)
+    s = (np.maximum(amax, F32(1e-4)) / F32(448.0)).astype(F32)
+    r = u[2 * n_groups:]
+    pick = (r[:n] % np.uint64(mids.size)).astype(np.int64).reshape(n_groups, gsize)
+    base = (mids[pick] * s[:, None]).astype(F32)
+    nudge = ((r[n:2 * n] % np.uint64(9)).astype(np.int64) - 4).reshape(n_groups, gsize)
+    vals = (base.view(np.int32) + nudge.astype(np.int32)).view(F32)
+    vals = np.minimum(vals, amax[:, None])
+    sign = np.where((r[2 * n:3 * n] >> np.uint64(7)) & np.uint64(1), -1.0, 1.0).astype(F32)
+    g = vals * sign.reshape(n_groups, gsize)
+    g[:, 0] = amax
+    return g.astype(F32)
+
+
+@pytest.mark.parametrize("mode", MODES3)
+def test_quotient_codes_on_rounding_boundaries(mode):
+    """Values placed on s x (E4M3 midpoint) boundaries. The case set is
+    checked to contain quotients whose code changes when x / s is replaced
+    by x * (1 / s), so a reciprocal-multiply quantiser fails it."""
+    gsize = 128 * 128 if mode == oracle.BLOCK_128x128 else 128
+    n_groups = 8 if mode == oracle.BLOCK_128x128 else 1024
+    g = _boundary_groups(n_groups, gsize, synth.seed(9, 13, mode))
+    x = _groups_to_layout(g, mode, n_groups)
+    s = _numpy_scales(x, mode)
+    recip = (F32(1.0) / s).astype(F32)
+    by_recip = torch_e4m3(np.clip((x * recip).astype(F32), F32(-448.0), F32(448.0)))
+    assert np.count_nonzero(by_recip != _expected_codes(x, s)) > 10
+    _check_quotient(x, mode)
