@@ -5,18 +5,25 @@ Workload (the dense sweep the pages' headline numbers are quoted on): M in
 (7168,16384), (4096,7168), (7168,2048)}; A, B ~ N(0,1) float32 from seeded
 streams. Weights B are quantised once at set-up (128x128 blocks, static FP8
 weights). One step = for every shape: quantise A (1x128 strips) on the GPU and
-run D = A @ B.T (BF16 out), i.e. the whole hot path per shape. L2 is flushed
-(256 MiB write) before every shape, outside the per-shape timing.
+run D = A @ B.T (BF16 out), i.e. the whole hot path per shape. K steps run back
+to back between two CUDA events; one step streams several GB, so every shape's
+operands have left the 126 MB L2 before the shape comes around again (inputs
+larger than L2, no flush).
 
 Reported (one JSON line, rank 0):
-  value        whole-job TFLOP/s = sum of GEMM FLOPs / device time of the step
-               (events around each shape's quantise + GEMM pair; the per-kernel
-               split comes from a separate pass with an event between them)
+  value        whole-job TFLOP/s = sum of GEMM FLOPs / device time of a step
   e2e          same metric through the public API with the activations copied
                from pinned host memory and D copied back inside the timed loop
   roofline     dominant kernel (the GEMM on its largest shape): achieved TFLOP/s
-               vs the measured-derived FP8 peak; plus an HBM block for the
-               decode shapes (M <= 128)
+               vs the measured-derived FP8 peak, from the kernel's average
+               launch duration over back-to-back launches; roofline_hbm: the
+               same for the decode shapes (M <= 128) against HBM bandwidth,
+               launches back to back over rotating weight copies (>= 3x L2),
+               with the single-launch-after-a-flush figure beside it
+  shapes       per shape: GEMM, quantiser and pair launch durations, and the
+               isolated single-launch GEMM time
+  moe          (one GPU) the MoE workloads: contiguous, masked (two weight
+               shapes), K-grouped -- quantise + grouped GEMM steps
   cpu_baseline the CPU oracle on a bounded row sample of the same workload
 --impl reference times that oracle as the reference arm (no GPU work).
 Multi-GPU (--gpus N under torchrun): N independent replicas (the path has no
@@ -228,20 +235,56 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------- grouped workloads
-def run_grouped(args):
-    """--workload contiguous | masked | kgrouped: the MoE variants at their
-    benchmark sizes (parity cases of the dense sweep's bench line, timed here
-    for the record). One step = quantise the activations on the GPU + the
-    grouped GEMM, inputs resident in HBM and larger than L2 (no flush needed).
-    value = useful TFLOP/s (real rows only); one GPU, rank 0."""
+L2_BYTES = 126 << 20
+
+
+def n_copies(nbytes, min_copies=1):
+    """Rotating copies so that consecutive launches never find their operand
+    in L2: the copies together span at least three times the L2."""
+    return max(min_copies, -(-3 * L2_BYTES // max(1, int(nbytes))))
+
+
+def time_batch(fn, reps, warm=2, graph=False):
+    """Average device time (ms) of one call of fn(i) over `reps` calls issued
+    back to back on the current stream, CUDA events around the batch. With
+    graph=True the batch is captured once into a CUDA graph and the events
+    bracket one replay, so the host's per-call cost (Python, argument
+    marshalling) cannot starve the device of short kernels."""
+    import torch
+    for i in range(warm):
+        fn(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(reps):
+                fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) / reps
+    torch.cuda._sleep(200_000)  # the host queues the batch while the device spins
+    e0.record()
+    for i in range(reps):
+        fn(i)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def moe_workload(kind, dev, masked_index=0):
+    """Builds one MoE workload at its benchmark size (synth inputs, weights
+    quantised once) and returns (quant, gemm, info): quant() quantises the
+    activations, gemm() runs the grouped GEMM, info holds FLOPs, algorithmic
+    bytes, bound and config."""
     import torch
     import moe_grouped_gemm_07_b200 as dg
-
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
-    torch.cuda.set_device(dev)
-    pk = peaks()
-    fp8_peak = 2.0 * pk["bf16_tflops"]
-    kind = args.workload
 
     def put(x):
         return torch.from_numpy(x).to(dev)
@@ -254,11 +297,10 @@ def run_grouped(args):
         qa = torch.empty(A.shape, dtype=torch.uint8, device=dev)
         sa = torch.zeros((w.K // 128, (w.Mt + 3) // 4 * 4), dtype=torch.float32, device=dev)
         D = torch.empty((w.Mt, w.N), dtype=torch.bfloat16, device=dev)
-        flops = 2.0 * w.N * w.K * float(sum(w.rows))
-        algo_bytes = w.Mt * w.K + w.G * w.N * w.K + 2 * w.Mt * w.N
-        bound = "tensor"
-        cfg = {"workload": "m_grouped_contiguous", "G": w.G, "N": w.N, "K": w.K, "Mt": w.Mt,
-               "rows": [int(r) for r in w.rows]}
+        info = {"flops": 2.0 * w.N * w.K * float(sum(w.rows)),
+                "bytes": w.Mt * w.K + w.G * w.N * w.K + 2 * w.Mt * w.N, "bound": "tensor",
+                "config": {"workload": "m_grouped_contiguous", "G": w.G, "N": w.N, "K": w.K,
+                           "Mt": w.Mt, "rows": [int(r) for r in w.rows]}}
 
         def quant():
             dg.dg_quantize_fp8(A, dg.DG_QUANT_ROW_1x128, codes=qa, scales=sa)
@@ -266,8 +308,8 @@ def run_grouped(args):
         def gemm():
             dg.dg_m_grouped_fp8_gemm_nt_contiguous(qa, sa, qb, sb, mi, None, D)
     elif kind == "masked":
-        NK = wl.MASKED_NK[args.masked_index]
-        w = wl.masked(N=NK[0], K=NK[1], shape=args.masked_index)
+        NK = wl.MASKED_NK[masked_index]
+        w = wl.masked(N=NK[0], K=NK[1], shape=masked_index)
         A = put(w.A)
         qb, sb = dg.dg_quantize_fp8(put(w.B), dg.DG_QUANT_BLOCK_128x128)
         mm = put(w.masked_m)
@@ -275,11 +317,10 @@ def run_grouped(args):
         sa = torch.zeros((w.G, w.K // 128, (w.max_m + 3) // 4 * 4), dtype=torch.float32, device=dev)
         D = torch.empty((w.G, w.max_m, w.N), dtype=torch.bfloat16, device=dev)
         tot = float(np.sum(w.masked_m))
-        flops = 2.0 * w.N * w.K * tot
-        algo_bytes = w.G * w.N * w.K + tot * (w.K + 2 * w.N)
-        bound = "hbm"
-        cfg = {"workload": "m_grouped_masked", "G": w.G, "max_m": w.max_m, "N": w.N, "K": w.K,
-               "sum_masked_m": int(tot)}
+        info = {"flops": 2.0 * w.N * w.K * tot,
+                "bytes": w.G * w.N * w.K + tot * (w.K + 2 * w.N), "bound": "hbm",
+                "config": {"workload": "m_grouped_masked", "G": w.G, "max_m": w.max_m, "N": w.N,
+                           "K": w.K, "sum_masked_m": int(tot)}}
 
         def quant():
             dg.dg_quantize_fp8(A, dg.DG_QUANT_ROW_1x128, codes=qa, scales=sa)
@@ -295,11 +336,10 @@ def run_grouped(args):
         sb = torch.empty((w.sumK // 128, w.N), dtype=torch.float32, device=dev)
         C = put(w.C)
         D = torch.empty_like(C)
-        flops = 2.0 * w.M * w.N * w.sumK
-        algo_bytes = w.sumK * (w.M + w.N) + 2 * C.numel() * 4
-        bound = "tensor"
-        cfg = {"workload": "k_grouped_tn_contiguous", "G": w.G, "M": w.M, "N": w.N,
-               "ks": [int(k) for k in w.ks]}
+        info = {"flops": 2.0 * w.M * w.N * w.sumK,
+                "bytes": w.sumK * (w.M + w.N) + 2 * C.numel() * 4, "bound": "tensor",
+                "config": {"workload": "k_grouped_tn_contiguous", "G": w.G, "M": w.M, "N": w.N,
+                           "ks": [int(k) for k in w.ks]}}
 
         def quant():
             dg.dg_quantize_fp8(A, dg.DG_QUANT_COL_128x1, codes=qa, scales=sa)
@@ -308,48 +348,66 @@ def run_grouped(args):
         def gemm():
             dg.dg_k_grouped_fp8_gemm_tn_contiguous(qa, sa, qb, sb, w.ks, C, D)
     torch.cuda.synchronize()
+    return quant, gemm, info
 
-    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    for _ in range(max(args.warmup, 3)):
+
+def measure_moe(kind, dev, steps, warmup, pk, masked_index=0):
+    """One MoE workload: step = quantise the activations + the grouped GEMM,
+    run back to back `steps` times (every operand is larger than L2, so no
+    flush is needed); the GEMM alone is timed the same way. Returns a dict."""
+    import torch
+    fp8_peak = 2.0 * pk["bf16_tflops"]
+    quant, gemm, info = moe_workload(kind, dev, masked_index)
+
+    def pair(_):
         quant()
         gemm()
-    torch.cuda.synchronize()
+    ms_step = time_batch(pair, steps, warm=max(warmup, 3))
+    ms_gemm = time_batch(lambda _: gemm(), steps, warm=2)
+    if info["bound"] == "tensor":
+        ach = info["flops"] / (ms_gemm * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
+                "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4)}
+    else:
+        ach = info["bytes"] / (ms_gemm * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / pk["hbm_gbs"], 4)}
+    out = {"step_ms": round(ms_step, 4), "gemm_ms": round(ms_gemm, 4),
+           "step_tflops": round(info["flops"] / (ms_step * 1e-3) / 1e12, 1),
+           "gemm_tflops": round(info["flops"] / (ms_gemm * 1e-3) / 1e12, 1),
+           "gemm_gbs": round(info["bytes"] / (ms_gemm * 1e-3) / 1e9, 1),
+           "algorithmic_bytes": int(info["bytes"]), "flops": info["flops"],
+           "roofline": roof, "config": info["config"]}
+    del quant, gemm
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_grouped(args):
+    """--workload contiguous | masked | kgrouped: one MoE variant at its
+    benchmark size (the default run reports all of them beside the dense
+    line). value = useful TFLOP/s of the quantise + GEMM step; one GPU."""
+    import torch
+    import moe_grouped_gemm_07_b200 as dg
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    pk = peaks()
     sampler = ClockSampler(dev.index)
     launches0 = dg.dg_get_launch_count()
     wall0 = time.time()
-    e[0].record()
-    for _ in range(args.steps):
-        quant()
-        gemm()
-    e[1].record()
-    torch.cuda.synchronize()
+    r = measure_moe(args.workload, dev, args.steps, args.warmup, pk, args.masked_index)
     wall1 = time.time()
-    launches = dg.dg_get_launch_count() - launches0
     clocks = sampler.stop(wall0, wall1)
-    ms_step = e[0].elapsed_time(e[1]) / args.steps
-    # GEMM alone (launch-averaged over the same number of launches)
-    e[0].record()
-    for _ in range(args.steps):
-        gemm()
-    e[1].record()
-    torch.cuda.synchronize()
-    ms_gemm = e[0].elapsed_time(e[1]) / args.steps
-    if bound == "tensor":
-        ach = flops / (ms_gemm * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
-                "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4), "traffic": None}
-    else:
-        ach = algo_bytes / (ms_gemm * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": round(ach / pk["hbm_gbs"], 4), "traffic": None}
-    line = {"metric": METRIC, "value": round(flops / (ms_step * 1e-3) / 1e12, 2),
-            "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": max(args.warmup, 3),
-            "ms_per_step": round(ms_step, 4), "gemm_ms": round(ms_gemm, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3 x e4m3 -> f32 accumulate", "data": "synthetic (seeded N(0,1))",
-            "config": dict(cfg, l2="inputs larger than L2, no flush"), "roofline": roof,
-            "gpu_launches": int(launches), "clocks": clocks,
-            "algorithmic_bytes_per_launch": int(algo_bytes), "flops_per_step": flops}
+    line = {"metric": METRIC, "value": r["step_tflops"], "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": r["step_ms"],
+            "gemm_ms": r["gemm_ms"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32 accumulate",
+            "data": "synthetic (seeded N(0,1))",
+            "config": dict(r["config"], l2="inputs larger than L2, steps back to back, no flush"),
+            "roofline": r["roofline"], "gpu_launches": int(dg.dg_get_launch_count() - launches0),
+            "clocks": clocks, "algorithmic_bytes_per_launch": r["algorithmic_bytes"],
+            "flops_per_step": r["flops"]}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -568,100 +626,133 @@ def run_ours(args):
     shapes = wl.dense_shapes()
     if args.shape:
         shapes = [tuple(int(x) for x in sh.split(",")) for sh in args.shape.split(";") if sh]
+    pk = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops"]  # nominal FP8:BF16 dense ratio is 2
 
-    # ---- set-up: weights quantised once, activations resident in HBM
+    # ---- set-up: weights quantised once (plus rotating copies for the
+    # per-kernel batches), activations resident in HBM
     weights = {}
     for (N, K) in sorted(set((s_[1], s_[2]) for s_ in shapes)):
         B = torch.from_numpy(synth.normal((N, K), synth.seed(2, nk_index(N, K), 1))).to(device)
-        weights[(N, K)] = dg.dg_quantize_fp8(B, dg.DG_QUANT_BLOCK_128x128)
+        qb, sb = dg.dg_quantize_fp8(B, dg.DG_QUANT_BLOCK_128x128)
         del B
+        weights[(N, K)] = ([qb] + [qb.clone() for _ in range(n_copies(N * K, 2) - 1)], sb)
     acts, outs, qbufs = [], [], []
+    step_bytes = 0
     for i, (M, N, K) in enumerate(shapes):
         A = torch.from_numpy(synth.normal((M, K), synth.seed(2, shape_index(M, N, K), 0))).to(device)
         acts.append(A)
-        outs.append(torch.empty((M, N), dtype=torch.bfloat16, device=device))
+        nd = min(len(weights[(N, K)][0]), n_copies(2 * M * N, 1))
+        outs.append([torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(nd)])
         qbufs.append((torch.empty((M, K), dtype=torch.uint8, device=device),
                       torch.zeros((K // 128, (M + 3) // 4 * 4), dtype=torch.float32,
                                   device=device)))
+        step_bytes += 4 * M * K + M * K + N * K + 2 * M * N
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     torch.cuda.synchronize()
-
     n = len(shapes)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
 
-    def step(record=False, split=False):
-        """One pass over the shapes. record: events around each shape's
-        quantise + GEMM pair (the step time); split: one more event between
-        the two kernels (per-kernel times; this can block the overlap of the
-        GEMM's prologue with the quantiser, so it is a separate pass)."""
-        for i, (M, N, K) in enumerate(shapes):
-            flush.fill_(i & 0xFF)
-            # ~50 us device spin (outside the per-shape events) so the host has
-            # queued the timed launches before the device reaches them: the
-            # events then bracket kernel time, not host submission gaps
-            torch.cuda._sleep(100_000)
-            if record:
-                ev[i][0].record()
-            qa, sa = qbufs[i]
-            dg.dg_quantize_fp8(acts[i], dg.DG_QUANT_ROW_1x128, codes=qa, scales=sa)
-            if split:
-                ev[i][1].record()
-            qb, sb = weights[(N, K)]
-            dg.dg_fp8_gemm_nt(qa, sa, qb, sb, None, outs[i])
-            if record:
-                ev[i][2].record()
+    def run_shape(i, copy=0):
+        M, N, K = shapes[i]
+        qa, sa = qbufs[i]
+        qbs, sb = weights[(N, K)]
+        dg.dg_quantize_fp8(acts[i], dg.DG_QUANT_ROW_1x128, codes=qa, scales=sa)
+        dg.dg_fp8_gemm_nt(qa, sa, qbs[copy % len(qbs)], sb, None, outs[i][copy % len(outs[i])])
+
+    def step():
+        """One pass of the hot path over the batch: per shape, quantise A
+        (1x128) and run the GEMM. Consecutive kernels overlap through PDL."""
+        for i in range(n):
+            run_shape(i)
 
     sampler = None if args.quick else ClockSampler(local)
     for _ in range(max(args.warmup, 0)):
         step()
     torch.cuda.synchronize()
 
-    # ---- timed region (device-resident inputs)
-    t_q = np.zeros(n)
-    t_g = np.zeros(n)
+    # ---- timed region: K whole steps back to back, device-resident inputs.
+    # A step streams step_bytes (several GB), so each shape's operands have
+    # left L2 before the shape comes around again: no flush is needed.
     launches0 = dg.dg_get_launch_count()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     wall0 = time.time()
-    outer0 = torch.cuda.Event(enable_timing=True)
-    outer1 = torch.cuda.Event(enable_timing=True)
-    t_pair = np.zeros(n)
-    outer0.record()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
     for _ in range(args.steps):
-        step(record=True)
-        torch.cuda.synchronize()
-        for i in range(n):
-            t_pair[i] += ev[i][0].elapsed_time(ev[i][2])
-    outer1.record()
+        step()
+    e1.record()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     wall1 = time.time()
     launches = dg.dg_get_launch_count() - launches0
     clocks = sampler.stop(wall0, wall1) if sampler else None
-    t_pair /= args.steps
-    ms_step = float(np.sum(t_pair))
-    # per-kernel split (separate, untimed-for-value pass)
-    split_steps = max(1, min(args.steps, 20))
-    for _ in range(split_steps):
-        step(record=True, split=True)
+    ms_step = e0.elapsed_time(e1) / args.steps
+    ms_step, = max_over_ranks(dist, [ms_step], device)
+
+    # ---- per-kernel launch durations, two ways:
+    # (1) in the step: a few more steps with CUDA events around each shape's
+    #     GEMM (the events hold the GEMM back from overlapping its
+    #     neighbours, so these are not part of the step time);
+    # (2) back to back: each kernel launched `reps` times over rotating weight
+    #     / output copies (together >= 3x L2, so every launch reads its
+    #     weights from DRAM), captured in a CUDA graph, events around a replay
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+    t_in = np.zeros(n)
+    ctx_steps = max(2, min(args.steps, 10))
+    for _ in range(ctx_steps):
+        for i in range(n):
+            M, N, K = shapes[i]
+            qa, sa = qbufs[i]
+            qbs, sb = weights[(N, K)]
+            dg.dg_quantize_fp8(acts[i], dg.DG_QUANT_ROW_1x128, codes=qa, scales=sa)
+            ev[i][0].record()
+            dg.dg_fp8_gemm_nt(qa, sa, qbs[0], sb, None, outs[i][0])
+            ev[i][1].record()
         torch.cuda.synchronize()
         for i in range(n):
-            t_q[i] += ev[i][0].elapsed_time(ev[i][1])
-            t_g[i] += ev[i][1].elapsed_time(ev[i][2])
-    t_q /= split_steps
-    t_g /= split_steps
-    ms_outer = outer0.elapsed_time(outer1) / args.steps
-    ms_step, ms_outer = max_over_ranks(dist, [ms_step, ms_outer], device)
+            t_in[i] += ev[i][0].elapsed_time(ev[i][1]) / ctx_steps
+    t_g, t_q, t_pair, t_iso = np.zeros(n), np.zeros(n), np.zeros(n), np.zeros(n)
+    for i, (M, N, K) in enumerate(shapes):
+        qa, sa = qbufs[i]
+        qbs, sb = weights[(N, K)]
+        reps = 32 if M <= 128 else 8
+        t_g[i] = time_batch(lambda j: dg.dg_fp8_gemm_nt(qa, sa, qbs[j % len(qbs)], sb, None,
+                                                        outs[i][j % len(outs[i])]), reps,
+                            graph=True)
+        t_q[i] = time_batch(lambda j: dg.dg_quantize_fp8(acts[i], dg.DG_QUANT_ROW_1x128, codes=qa,
+                                                         scales=sa), reps, graph=True)
+        t_pair[i] = time_batch(lambda j: run_shape(i, j), reps, graph=True)
+        # isolated: one launch after a 256 MiB flush write and a device spin
+        iso = []
+        for j in range(6):
+            flush.fill_(j & 0xFF)
+            torch.cuda._sleep(100_000)
+            e0.record()
+            dg.dg_fp8_gemm_nt(qa, sa, qbs[j % len(qbs)], sb, None, outs[i][j % len(outs[i])])
+            e1.record()
+            torch.cuda.synchronize()
+            if j >= 1:
+                iso.append(e0.elapsed_time(e1))
+        t_iso[i] = float(np.mean(iso))
+    t_all = max_over_ranks(dist, list(t_g) + list(t_q) + list(t_pair) + list(t_iso) + list(t_in),
+                           device)
+    t_g, t_q = np.array(t_all[:n]), np.array(t_all[n:2 * n])
+    t_pair, t_iso = np.array(t_all[2 * n:3 * n]), np.array(t_all[3 * n:4 * n])
+    t_in = np.array(t_all[4 * n:])
 
     # ---- end to end through the public API with host buffers
     if args.quick:
         if rank == 0:
-            print(json.dumps({"quick": True, "shapes": [list(x) for x in shapes],
+            print(json.dumps({"quick": True, "ms_per_step": round(ms_step, 4),
+                              "shapes": [list(x) for x in shapes],
                               "gemm_us": [round(x * 1e3, 2) for x in t_g],
                               "pair_us": [round(x * 1e3, 2) for x in t_pair],
-                              "quant_us": [round(x * 1e3, 2) for x in t_q]}), flush=True)
+                              "quant_us": [round(x * 1e3, 2) for x in t_q],
+                              "gemm_isolated_us": [round(x * 1e3, 2) for x in t_iso]}), flush=True)
         if dist:
             dist.destroy_process_group()
         return 0
@@ -676,15 +767,13 @@ def run_ours(args):
             acts[i].copy_(host_a[i], non_blocking=True)
             qa, sa = qbufs[i]
             dg.dg_quantize_fp8(acts[i], dg.DG_QUANT_ROW_1x128, codes=qa, scales=sa)
-            qb, sb = weights[(N, K)]
-            dg.dg_fp8_gemm_nt(qa, sa, qb, sb, None, outs[i])
-            host_d[i].copy_(outs[i], non_blocking=True)
+            qbs, sb = weights[(N, K)]
+            dg.dg_fp8_gemm_nt(qa, sa, qbs[0], sb, None, outs[i][0])
+            host_d[i].copy_(outs[i][0], non_blocking=True)
 
     for _ in range(max(1, min(args.warmup, 2))):
         e2e_step()
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
     e2e_steps = max(1, min(args.steps, 10))
     if dist:
         dist.barrier()
@@ -696,37 +785,46 @@ def run_ours(args):
     ms_e2e = e0.elapsed_time(e1) / e2e_steps
     ms_e2e, = max_over_ranks(dist, [ms_e2e], device)
 
-    flops_step = sum(shape_flops(*s) for s in shapes)
-    pk = peaks()
-    fp8_peak = 2.0 * pk["bf16_tflops"]  # nominal FP8:BF16 dense ratio is 2
+    flops_step = sum(shape_flops(*s_) for s_ in shapes)
     per_shape = []
     for i, (M, N, K) in enumerate(shapes):
-        tf = shape_flops(M, N, K) / (t_g[i] * 1e-3) / 1e12
-        gbs = shape_bytes(M, N, K) / (t_g[i] * 1e-3) / 1e9
         roof_ms = max(shape_flops(M, N, K) / (fp8_peak * 1e12),
                       shape_bytes(M, N, K) / (pk["hbm_gbs"] * 1e9)) * 1e3
-        per_shape.append({"M": M, "N": N, "K": K, "step_us": round(t_pair[i] * 1e3, 2),
-                          "gemm_us": round(t_g[i] * 1e3, 2),
-                          "quant_us": round(t_q[i] * 1e3, 2), "tflops": round(tf, 1),
-                          "gbs": round(gbs, 1), "roofline_frac": round(roof_ms / t_g[i], 3)})
-    # dominant kernel: the GEMM on its largest shape
-    big = max(range(n), key=lambda i: t_g[i])
+        per_shape.append({"M": M, "N": N, "K": K, "gemm_us": round(t_g[i] * 1e3, 2),
+                          "gemm_in_step_us": round(t_in[i] * 1e3, 2),
+                          "quant_us": round(t_q[i] * 1e3, 2), "pair_us": round(t_pair[i] * 1e3, 2),
+                          "gemm_isolated_us": round(t_iso[i] * 1e3, 2),
+                          "tflops": round(shape_flops(M, N, K) / (t_g[i] * 1e-3) / 1e12, 1),
+                          "gbs": round(shape_bytes(M, N, K) / (t_g[i] * 1e-3) / 1e9, 1),
+                          "roofline_frac": round(roof_ms / t_g[i], 3)})
+    # dominant kernel: the GEMM on its largest shape, timed in the step
+    big = max(range(n), key=lambda i: t_in[i])
     Mb, Nb, Kb = shapes[big]
-    ach = shape_flops(Mb, Nb, Kb) / (t_g[big] * 1e-3) / 1e12
+    ach = shape_flops(Mb, Nb, Kb) / (t_in[big] * 1e-3) / 1e12
     key = f"gemm_fp8_kernel:{Mb}x{Nb}x{Kb}"
     roofline = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
                 "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4),
                 "traffic": traffic_from_profile(key),
                 "kernel": key,
+                "timing": "CUDA events around this GEMM inside full steps (its neighbours in the "
+                          "step are the other shapes' kernels); back to back alone: "
+                          f"{t_g[big] * 1e3:.1f} us",
                 "peak_note": f"FP8 dense = 2 x {pk['source']} bf16 burst "
                              f"({pk['bf16_tflops']} TF/s); nominal FP8 {NOMINAL_FP8_TFLOPS} TF/s"}
-    dec = [i for i, s in enumerate(shapes) if s[0] <= 128]
-    dec_bytes = sum(shape_bytes(*shapes[i]) for i in dec)
-    dec_ms = float(sum(t_g[i] for i in dec))
-    roofline_hbm = {"bound": "hbm", "achieved": round(dec_bytes / (dec_ms * 1e-3) / 1e9, 1),
-                    "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(dec_bytes / (dec_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-                    "shapes": "M in {64,128} (12 decode shapes), GEMM kernel only"}
+    dec = [i for i, s_ in enumerate(shapes) if s_[0] <= 128]
+    roofline_hbm = None
+    if dec:
+        dec_bytes = sum(shape_bytes(*shapes[i]) for i in dec)
+        dec_ms = float(sum(t_g[i] for i in dec))
+        dec_iso_ms = float(sum(t_iso[i] for i in dec))
+        roofline_hbm = {"bound": "hbm", "achieved": round(dec_bytes / (dec_ms * 1e-3) / 1e9, 1),
+                        "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(dec_bytes / (dec_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                        "frac_isolated_launch": round(
+                            dec_bytes / (dec_iso_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                        "shapes": f"M in {{64,128}} ({len(dec)} decode shapes), GEMM kernel only, "
+                                  "average launch duration back to back over rotating weights; "
+                                  "frac_isolated_launch: one launch after a flush, events around it"}
 
     line = {
         "metric": METRIC, "value": round(job_tflops(world, flops_step, ms_step), 2),
@@ -737,10 +835,10 @@ def run_ours(args):
         "config": {"workload": WORKLOAD, "shapes": n, "M": list(wl.DENSE_M),
                    "NK": [list(x) for x in wl.DENSE_NK],
                    "step": "per shape: quantise A (1x128) + GEMM; B pre-quantised (128x128)",
-                   "l2": "flushed (256 MiB write) before every shape, flush excluded from timing",
-                   "host_gap": "a ~50 us device spin precedes each shape so events time kernels only",
+                   "l2": f"inputs larger than L2: a step streams {step_bytes / 1e9:.2f} GB, so "
+                         "every shape's operands leave L2 before it comes around again; no flush",
+                   "timing": "K steps back to back between two CUDA events",
                    "parallelism": f"replicas x{world}"},
-        "ms_per_step_incl_flush": round(ms_outer, 4),
         "fp8_pct_of_measured_peak": round(100 * flops_step / (ms_step * 1e-3) / 1e12 / fp8_peak, 2),
         "fp8_pct_of_nominal_peak": round(100 * flops_step / (ms_step * 1e-3) / 1e12
                                          / NOMINAL_FP8_TFLOPS, 2),
@@ -751,15 +849,23 @@ def run_ours(args):
         "gpu_launches": int(launches), "gpu_launches_per_step": int(launches // max(args.steps, 1)),
         "clocks": clocks, "shapes": per_shape,
     }
+    del weights, outs, flush
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_moe:
+        moe = {}
+        for name, kind, idx in (("contiguous", "contiguous", 0), ("masked_4096x7168", "masked", 0),
+                                ("masked_7168x2048", "masked", 1), ("kgrouped", "kgrouped", 0)):
+            moe[name] = measure_moe(kind, device, max(3, min(args.steps, 20)), args.warmup, pk, idx)
+        line["moe"] = moe
     if rank == 0 and not args.no_cpu_baseline:
         rows = args.cpu_rows
         inputs = prepare_oracle_inputs(shapes, rows)
-        f, s, cores = oracle_sample(shapes, rows, inputs)
-        line["cpu_baseline"] = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": cores,
+        f, s_, cores = oracle_sample(shapes, rows, inputs)
+        line["cpu_baseline"] = {"value": f / s_ / 1e12, "unit": "TFLOP/s", "cores": cores,
                                 "kind": "oracle",
                                 "sample": f"{rows} rows of each of the 18 shapes (A rows "
                                           f"quantised + those rows of D), weights pre-quantised; "
-                                          f"{s:.1f} s"}
+                                          f"{s_:.1f} s"}
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -777,6 +883,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-moe", action="store_true",
+                    help="skip the MoE workloads (contiguous, masked, K-grouped) of the default run")
     ap.add_argument("--shape", default="",
                     help="M,N,K[;M,N,K...]: time only these shapes (profiling)")
     ap.add_argument("--quick", action="store_true",

@@ -330,7 +330,13 @@ uint64_t dg_get_launch_count(void);
  *   DG_PAIR_BN=128|256   tile width of the pair kernel; read once.
  *   DG_DECODE_MINB=1|2, DG_DECODE_SPLITS=s
  *                        CTAs per SM and split count of the M <= 128 kernels;
- *                        read on every call. */
+ *                        read on every call.
+ *   DG_DECODE_KG=1|2|4   K-blocks per ring stage (one TMA box each for weights
+ *                        and tokens) of the FP8 M <= 128 kernel; read on every
+ *                        call.
+ *   DG_DECODE_PF=k       weight K-blocks the FP8 M <= 128 kernel keeps
+ *                        requested into L2 ahead of its loads (rounded up to
+ *                        a multiple of 8, default 64); read on every call. */
 
 #ifdef __cplusplus
 }

@@ -139,6 +139,30 @@ dg_status make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, 
   return DG_OK;
 }
 
+// 3-D tensor: dims {d0, d1, d2} (d0 contiguous), byte strides of dims 1 and
+// 2, box {b0, b1, b2}. A [rows][K] operand viewed as [K/128][rows][128] this
+// way lets one box carry several K-blocks of a tile, each landing as the
+// [rows][128] tile a 2-D box would give.
+dg_status make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t d0,
+                      uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0,
+                      uint32_t b1, uint32_t b2,
+                      CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return DG_ERR_CUDA;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1, stride2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    if (print_configs()) std::fprintf(stderr, "[dg] cuTensorMapEncodeTiled (3-D) failed: %d\n", (int)r);
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
+}
+
 // ---------------------------------------------------------------- launches
 template <int MODE, int BN>
 dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
@@ -538,7 +562,7 @@ int max_cluster(int dev) {
   static int best[kMaxDevices];
   std::call_once(once[dev], [&] {
     best[dev] = probe_max_cluster(reinterpret_cast<const void*>(dg::gemm_decode_kernel<BNP, MINB>),
-                                  dg::DecodeCfg<BNP, MINB>::SMEM_BYTES);
+                                  dg::DecodeCfg<BNP, MINB>::SMEM_BUDGET);
   });
   return best[dev];
 }
@@ -555,46 +579,115 @@ int max_cluster_mx(int dev) {
   return best[dev];
 }
 
-// Decode plan: CTAs per SM (MINB) and split count. From a sweep of both
-// configurations x 1..8 splits over the decode shapes on B200: more than 4-5
-// splits lose (each CTA keeps too few K-blocks and the reduction grows); with
-// at least one tile per SM a single split on two CTAs per SM is best; M > 64
-// prefers one CTA per SM (all TMEM and registers for the 128-token tile) with
-// at most one CTA per SM in total; M <= 64 prefers two CTAs per SM.
+// Decode plan: CTAs per SM (MINB) and split count, from a sweep of both
+// configurations x 1..8 splits x 1/2/4 K-blocks per stage over the decode
+// shapes on B200, timed back to back. Tokens up to 64 take the half-SM
+// configuration (two CTAs per SM; a CTA of the next launch can also sit
+// beside one of this launch and prefetch its weights early) with about 256
+// CTAs; 128-token tiles need the whole SM, about 128 CTAs. A CTA streams at
+// most ~85 GB/s through TMA, so the grid must be wide; more splits than that
+// lose to their exchange. At most 8 splits (the portable cluster size and the
+// co-schedulable cluster size) and at least 2 K-blocks per split.
 struct DecodePlan {
   int minb, splits;
 };
 
+// Weight K-blocks each decode CTA keeps requested into L2 ahead of its TMA
+// loads, a multiple of 8 (DG_DECODE_PF overrides, read on every call).
+int decode_prefetch_kblocks() {
+  int pf = 64;
+  if (const char* e = std::getenv("DG_DECODE_PF")) {
+    const int f = std::atoi(e);
+    if (f >= 0) pf = f;
+  }
+  return (pf + 7) / 8 * 8;
+}
+
 DecodePlan plan_decode(int M, int n_tiles, int KB, int sms, int cap1, int cap2) {
+  auto clampi = [](int v, int lo, int hi) { return std::max(lo, std::min(v, hi)); };
+  const int minb = M <= 64 ? 2 : 1;
+  const int cap = minb == 1 ? cap1 : cap2;
+  const int target = (minb == 2 ? 256 : 128) * sms / 148;
+  const int splits = clampi(target / n_tiles, 1, std::min(std::min(8, cap), std::max(1, KB / 2)));
+  return {minb, splits};
+}
+
+// Plan of the block-scaled decode kernel (gemm_mx_decode.cuh), from a sweep
+// of both configurations x 1..8 splits over the decode shapes on B200: more
+// than 4-5 splits lose (each CTA keeps too few K-blocks and its cluster-barrier
+// reduction grows); with at least one tile per SM a single split on two CTAs
+// per SM is best; M > 64 prefers one CTA per SM, M <= 64 two.
+DecodePlan plan_mx_decode(int M, int n_tiles, int KB, int sms, int cap1, int cap2) {
   auto clampi = [](int v, int lo, int hi) { return std::max(lo, std::min(v, hi)); };
   if (n_tiles >= sms) return {2, 1};
   if (M > 64) return {1, clampi(std::min(sms / n_tiles, KB / 2), 1, std::min(5, cap1))};
   return {2, clampi(std::min(2 * sms / n_tiles, KB / 2), 1, std::min(4, cap2))};
 }
 
+// Shared-memory layout of one decode launch: the deepest W/X ring (2..8
+// stages) that fits beside the sfa chunk slots, the split-K receive slots and
+// the barriers in the configuration's share of the SM. False if it does not fit.
+template <int BNP, int MINB>
+bool decode_layout(int M, int splits, int kg, dg::DecodeArgs* a, int* smem_bytes) {
+  using Cfg = dg::DecodeCfg<BNP, MINB>;
+  const int R = (M + splits - 1) / splits;
+  const int recv = splits > 1 ? (splits - 1) * R * 512 : 0;
+  const int sfa = 2 * Cfg::SFA_CHUNK_BYTES;
+  const int fixed = sfa + recv + Cfg::BAR_BYTES + 1024;  // + alignment slack of the base
+  const int stage = kg * Cfg::STAGE_BYTES;
+  int stages = (Cfg::SMEM_BUDGET - fixed) / stage;
+  stages = std::min(stages, Cfg::MAX_STAGES);
+  if (stages < 2 || stages * stage < Cfg::STAGE_OUT_BYTES) return false;
+  a->stages = stages;
+  a->kg = kg;
+  a->rows_per_owner = R;
+  a->off_x = static_cast<uint32_t>(stages * kg * Cfg::W_BYTES);
+  a->off_sfa = static_cast<uint32_t>(stages * stage);
+  a->off_recv = a->off_sfa + static_cast<uint32_t>(sfa);
+  a->off_bar = a->off_recv + static_cast<uint32_t>(recv);
+  *smem_bytes = static_cast<int>(a->off_bar) + Cfg::BAR_BYTES + 1024;
+  return *smem_bytes <= Cfg::SMEM_BUDGET;
+}
+
 template <int BNP, int MINB>
 dg_status run_decode(const void* A, const float* sfa, const void* B, const float* sfb,
-                     const void* C, void* D, int M, int N, int K, int splits, int sms, int dev,
-                     cudaStream_t st) {
+                     const void* C, void* D, int M, int N, int K, int splits, cudaStream_t st) {
   using Cfg = dg::DecodeCfg<BNP, MINB>;
   const int KB = K / 128;
   const int n_tiles = (N + 127) / 128;
-  (void)sms;
-  (void)dev;
   const int ld = (M + 3) / 4 * 4;
-  CUtensorMap tw, tx, tsa;
-  dg_status s;
-  if ((s = make_map_2d(&tw, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, 128, 128,
-                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
-    return s;
-  if ((s = make_map_2d(&tx, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, BNP,
-                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
-    return s;
-  if ((s = make_map_2d(&tsa, sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ld, KB, 4ull * ld, BNP, 1,
-                       CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
-    return s;
   dg::DecodeArgs args;
   std::memset(&args, 0, sizeof args);
+  int smem = 0;
+  // K-blocks per ring stage: the deepest box (4, 2, 1) that still leaves a
+  // ring of two stages; DG_DECODE_KG=1|2|4 forces it (read on every call)
+  int kg = 0;
+  if (const char* e = std::getenv("DG_DECODE_KG")) {
+    const int f = std::atoi(e);
+    if (f == 1 || f == 2 || f == 4) kg = f;
+  }
+  bool fits = false;
+  if (kg) {
+    fits = decode_layout<BNP, MINB>(M, splits, kg, &args, &smem);
+  } else {
+    for (kg = 4; kg >= 1 && !fits; kg /= 2) fits = decode_layout<BNP, MINB>(M, splits, kg, &args, &smem);
+  }
+  if (!fits) return DG_ERR_UNSUPPORTED_SHAPE;
+  CUtensorMap tw, twpf, tx, tsa;
+  dg_status s;
+  // weights and tokens viewed as [KB][rows][128]: one box = kg K-blocks of a tile
+  if ((s = make_map_3d(&tw, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, N, KB, K, 128, 128, 128,
+                       static_cast<uint32_t>(args.kg), CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  if ((s = make_map_3d(&twpf, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, N, KB, K, 128, 128, 128,
+                       Cfg::PF_BOX)) != DG_OK)
+    return s;
+  if ((s = make_map_3d(&tx, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, M, KB, K, 128, 128, BNP,
+                       static_cast<uint32_t>(args.kg), CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+    return s;
+  if ((s = make_map_2d(&tsa, sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ld, KB, 4ull * ld, BNP,
+                       Cfg::SCH, CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
+    return s;
   args.M = M;
   args.N = N;
   args.K = K;
@@ -605,13 +698,14 @@ dg_status run_decode(const void* A, const float* sfa, const void* B, const float
   args.D = D;
   args.timeout_ns = timeout_ns();
   args.drop_arrive = take_drop_flag();
+  args.pf = decode_prefetch_kblocks();
   if (print_configs())
     std::fprintf(stderr,
                  "[dg] fp8_gemm_nt decode M=%d N=%d K=%d: swap-AB BNP=%d (%d CTA/SM), n_tiles=%d x "
-                 "split-K %d (cluster), %d CTAs, %d stages\n",
-                 M, N, K, BNP, MINB, n_tiles, splits, n_tiles * splits, Cfg::STAGES);
+                 "split-K %d (cluster), %d CTAs, %d stages x %d K-blocks, %d B smem\n",
+                 M, N, K, BNP, MINB, n_tiles, splits, n_tiles * splits, args.stages, args.kg, smem);
   cudaError_t e = launch(dg::gemm_decode_kernel<BNP, MINB>, dim3(splits, n_tiles, 1), dim3(320),
-                         Cfg::SMEM_BYTES, st, splits, tw, tx, tsa, args);
+                         static_cast<size_t>(smem), st, splits, tw, twpf, tx, tsa, args);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   g_launches.fetch_add(1);
   return DG_OK;
@@ -628,34 +722,37 @@ dg_status dispatch_decode(const void* A, const float* sfa, const void* B, const 
     case 16: cap1 = max_cluster<16, 1>(dev); cap2 = max_cluster<16, 2>(dev); break;
     case 32: cap1 = max_cluster<32, 1>(dev); cap2 = max_cluster<32, 2>(dev); break;
     case 64: cap1 = max_cluster<64, 1>(dev); cap2 = max_cluster<64, 2>(dev); break;
-    default: cap1 = max_cluster<128, 1>(dev); cap2 = max_cluster<128, 2>(dev); break;
+    default: cap1 = max_cluster<128, 1>(dev); break;
   }
-  if (cap1 <= 0 || cap2 <= 0) return DG_ERR_CUDA;
+  if (cap1 <= 0 || (bnp < 128 && cap2 <= 0)) return DG_ERR_CUDA;
   DecodePlan p = plan_decode(M, n_tiles, KB, sms, cap1, cap2);
   // DG_DECODE_MINB=1|2 and DG_DECODE_SPLITS=s force the plan (comparisons;
-  // splits clamped to the cluster limit and to one K-block per split); read
-  // on every call
+  // splits clamped to the cluster limit and to one K-block per split; 128
+  // tokens always take the whole SM); read on every call
   if (const char* e = std::getenv("DG_DECODE_MINB")) {
     const int f = std::atoi(e);
     if (f == 1 || f == 2) p.minb = f;
   }
+  if (bnp == 128) p.minb = 1;
   const int cap = p.minb == 1 ? cap1 : cap2;
-  p.splits = std::min(p.splits, std::min(cap, 8));
+  p.splits = std::max(1, std::min(p.splits, std::min(cap, 8)));
   if (const char* e = std::getenv("DG_DECODE_SPLITS")) {
     const int f = std::atoi(e);
     if (f >= 1) p.splits = std::max(1, std::min(std::min(f, std::min(cap, 8)), KB));
   }
-#define DG_RUN_DECODE(BNP_)                                                                   \
-  return p.minb == 1                                                                          \
-             ? run_decode<BNP_, 1>(A, sfa, B, sfb, C, D, M, N, K, p.splits, sms, dev, st) \
-             : run_decode<BNP_, 2>(A, sfa, B, sfb, C, D, M, N, K, p.splits, sms, dev, st)
   switch (bnp) {
-    case 16: DG_RUN_DECODE(16);
-    case 32: DG_RUN_DECODE(32);
-    case 64: DG_RUN_DECODE(64);
-    default: DG_RUN_DECODE(128);
+    case 16:
+      return p.minb == 1 ? run_decode<16, 1>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st)
+                         : run_decode<16, 2>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st);
+    case 32:
+      return p.minb == 1 ? run_decode<32, 1>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st)
+                         : run_decode<32, 2>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st);
+    case 64:
+      return p.minb == 1 ? run_decode<64, 1>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st)
+                         : run_decode<64, 2>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st);
+    default:
+      return run_decode<128, 1>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st);
   }
-#undef DG_RUN_DECODE
 }
 
 // Block-scaled small-M launcher (swap-AB, cluster split-K; W4: E2M1 weights).
@@ -723,7 +820,7 @@ dg_status dispatch_mx_decode(const void* X, const int32_t* sfx, const void* W,
     default: cap1 = max_cluster_mx<128, 1, W4>(dev); cap2 = max_cluster_mx<128, 2, W4>(dev); break;
   }
   if (cap1 <= 0 || cap2 <= 0) return DG_ERR_CUDA;
-  DecodePlan p = plan_decode(M, n_tiles, KB, sms, cap1, cap2);
+  DecodePlan p = plan_mx_decode(M, n_tiles, KB, sms, cap1, cap2);
   if (W4 && n_tiles < sms) {
     // E2M1 weights (from a sweep of both configurations x 1..8 splits over
     // the decode shapes): two CTAs per SM at every M, and a split keeps at

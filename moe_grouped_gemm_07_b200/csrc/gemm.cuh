@@ -270,6 +270,7 @@ enum : unsigned int {
   SITE_TEARDOWN_TMA = 7,
   SITE_TEARDOWN_MMA = 8,
   SITE_K_SIZES = 9,  // device-side K-group sizes were invalid (DG_ERR_INVALID_ARG)
+  SITE_SPLITK_RECV = 10,  // a split-K owner waited for its peers' partial sums
 };
 
 template <int MODE, int BN>

@@ -12,24 +12,30 @@
 //   * split-K across a thread-block cluster: the `splits` CTAs of a cluster
 //     share one N-tile and each streams its own slice of K-blocks, so
 //     n_tiles x splits CTAs keep HBM busy even when N/128 is small;
-//   * the partial tiles are reduced through distributed shared memory: CTA r
-//     owns units [16r/splits, 16(r+1)/splits) of the tile's sixteen 8-row
-//     units (splits <= 8, any count); after a cluster
-//     barrier (every ring is free) each CTA pushes, with remote stores, the
-//     rows of its FP32 partial that CTA o owns into o's receive slot for
-//     rank r; after a second barrier each CTA sums its units over the slots in
-//     rank order (deterministic) from its own shared memory, adds C and
-//     stores BF16. Remote stores need no round trip; remote loads, which an
-//     owner pulling the partials would issue, are latency-bound.
+//   * each CTA asks L2 for its whole weight slice (a window of `pf` K-blocks
+//     ahead, 8 K-blocks per prefetch instruction) before anything else, so
+//     the slice's DRAM reads are all in flight while the CTA sets up and
+//     while the previous launch finishes; the TMA loads then mostly hit L2;
+//   * the partial tiles are reduced by token rows: CTA r owns tokens
+//     [r R, r R + R), R = ceil(M / splits). Each CTA writes its FP32 partial
+//     to its own shared memory token-major, then one thread bulk-copies the
+//     rows every other CTA owns into that CTA's receive slot for this rank
+//     (cp.async.bulk shared::cta -> shared::cluster), completing bytes on the
+//     owner's mbarrier; the owner sums the slices in rank order
+//     (deterministic), adds C and stores whole BF16 rows of D. The receive
+//     slots are dedicated, so no cluster barrier waits for the slowest CTA's
+//     main loop; one split cluster barrier (arrive after barrier init, wait
+//     before the copies) makes the owners' mbarriers visible to the peers.
 //
 // Roles per CTA (320 threads): warp 0 TMA producer, warp 1 TMEM allocator and
 // tcgen05.mma issuer (both run their loops as converged warps, lane 0
 // issuing), warps 2..9 promotion (TMEM lane quadrant w % 4, column half
 // (w - 2) / 4). The MMA runs up to NACC - 1 K-blocks ahead of the promotion
-// (NACC accumulator buffers of BNP columns). All waits are bounded (see
-// ptx.cuh); both cluster barriers are reached unconditionally, also after a
-// timeout. With a single split the launch has no cluster and CTA barriers
-// replace them.
+// (NACC accumulator buffers of BNP columns). sfa comes in chunks of 16
+// K-blocks (one TMA box per chunk, two chunk slots). All waits are bounded
+// (see ptx.cuh); the cluster barrier and the copies are reached
+// unconditionally, also after a timeout, and a CTA that timed out stores
+// nothing.
 #pragma once
 
 #include <cstdint>
@@ -43,19 +49,30 @@ namespace dg {
 
 struct DecodeArgs {
   int M, N, K;
-  int KB;       // K / 128
-  int splits;   // CTAs per cluster along K
+  int KB;        // K / 128
+  int splits;    // CTAs per cluster along K
+  int stages;    // depth of the W/X ring (2..DecodeCfg::MAX_STAGES)
+  int kg;        // K-blocks per ring stage (1, 2 or 4): one TMA box each for W and X
+  int rows_per_owner;  // R = ceil(M / splits): token rows reduced by each CTA
+  uint32_t off_x, off_sfa, off_recv, off_bar;  // shared-memory layout (bytes)
   const float* sfb;  // [ceil(N/128)][KB]
   const void* C;     // [M][N] bf16 or null
   void* D;           // [M][N] bf16
   unsigned long long timeout_ns;
   int drop_arrive;
+  int pf;        // weight K-blocks kept requested into L2 ahead of the TMA loads
 };
 
 // MINB = CTAs per SM the configuration is built for: 2 (a CTA gets half of
-// shared memory, registers and TMEM) or 1 (the whole SM: every promotion
-// thread loads all its accumulator columns in one TMEM round trip, and twice
-// the accumulator buffers).
+// shared memory, registers and TMEM, and a CTA of the next launch can sit
+// beside it) or 1 (the whole SM: every promotion thread loads all its
+// accumulator columns in one TMEM round trip, and twice the accumulator
+// buffers). A ring stage holds kg consecutive K-blocks of W and of X, each
+// moved by one 3-D TMA box (a CTA's TMA throughput grows with the box size).
+// The ring depth, kg and the offsets of the other regions are chosen on the
+// host per launch (decode_layout in the launcher): ring [stages][kg] W tiles
+// then [stages][kg] X tiles, the two sfa chunk slots, the receive slots
+// ((splits - 1) x R token rows of 128 floats), then the barriers.
 template <int BNP_, int MINB_>
 struct DecodeCfg {
   static constexpr int BNP = BNP_;              // token columns (MMA N)
@@ -63,13 +80,11 @@ struct DecodeCfg {
   static constexpr int BK = 128;
   static constexpr int W_BYTES = 128 * BK;      // weight tile (MMA A operand)
   static constexpr int X_BYTES = BNP * BK;      // token tile (MMA B operand)
-  static constexpr int RING = MINB == 2 ? 96 * 1024 : 192 * 1024;
-  static constexpr int STAGES_RAW = RING / (W_BYTES + X_BYTES);
-  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
-  static constexpr int SS = 8;                  // sfa slots
-  // a TMA destination in shared memory must be 128-byte aligned, so each
-  // slot holds at least 32 floats even when BNP = 16
-  static constexpr int SLOT_FLOATS = BNP < 32 ? 32 : BNP;
+  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
+  static constexpr int MAX_STAGES = 8;
+  static constexpr int SCH = 16;                // K-blocks per sfa chunk
+  static constexpr int SFA_CHUNK_BYTES = SCH * BNP * 4;
+  static constexpr int PF_BOX = 8;              // K-blocks per L2 prefetch instruction
   static constexpr int EC = BNP / 2;            // accumulator columns per promotion thread
   // columns per tcgen05.ld; with one CTA per SM all EC columns are in flight
   // before a single wait, with two the loads go one 16-column chunk at a time
@@ -78,29 +93,16 @@ struct DecodeCfg {
   // accumulator buffers in this CTA's share of TMEM
   static constexpr int NACC = (512 / MINB) / BNP > 8 ? 8 : (512 / MINB) / BNP;
   static constexpr int TMEM_COLS = NACC * BNP;
-  static constexpr int OFF_W = 0;
-  static constexpr int OFF_X = OFF_W + STAGES * W_BYTES;
-  static constexpr int OFF_SCALE = OFF_X + STAGES * X_BYTES;
-  static constexpr int OFF_BAR = OFF_SCALE + SS * SLOT_FLOATS * 4;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * NACC + 2 * SS + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  // receive slots of the split-K reduction, overlaying the ring:
-  // [src rank][owned unit (< ceil(16/splits))][row in unit (8)][RECV_PITCH]
-  // floats, tokens along the row; at most 168 rows (splits = 7: 7 x 3 x 8).
-  // The pitch is padded by 4 floats so that consecutive rows start in
-  // different banks.
-  static constexpr int MAX_SPLITS = 8;
-  static constexpr int RECV_PITCH = BNP + 4;
-  static constexpr int RECV_ROWS = 168;
-  static constexpr int RECV_BYTES = RECV_ROWS * RECV_PITCH * 4;
-  static_assert(RECV_BYTES <= STAGES * (W_BYTES + X_BYTES), "receive slots fit the ring");
+  // barriers: full[8] empty[8] tfull[NACC] tempty[NACC] sfull[2] sempty[2]
+  // mma_done recv; then the TMEM base address and the abort flag
+  static constexpr int NUM_BARS = 2 * MAX_STAGES + 2 * NACC + 4 + 2;
+  static constexpr int BAR_BYTES = NUM_BARS * 8 + 16;
+  static constexpr int STAGE_OUT_BYTES = BNP * 128 * 4;  // token-major FP32 partial
+  static constexpr int SMEM_BUDGET = MINB == 2 ? 113 * 1024 : 227 * 1024;
   static_assert((NACC & (NACC - 1)) == 0 && TMEM_COLS >= 32 && (TMEM_COLS & (TMEM_COLS - 1)) == 0,
                 "TMEM allocation is a power of two >= 32 columns");
   static_assert(BNP == 16 || BNP == 32 || BNP == 64 || BNP == 128, "BNP");
-  static_assert(OFF_SCALE % 1024 == 0 && (SLOT_FLOATS * 4) % 128 == 0, "TMA smem alignment");
-  static_assert(OFF_X % 1024 == 0 && X_BYTES % 1024 == 0, "SW128 tiles are 1024-byte aligned");
-  static_assert(SMEM_BYTES <= (MINB == 2 ? 113 : 227) * 1024, "MINB CTAs per SM");
+  static_assert(X_BYTES % 1024 == 0, "SW128 tiles are 1024-byte aligned");
 };
 
 // Split-K reduction of a cluster's partial 128 x BNP tiles (swap-AB decode
@@ -180,81 +182,88 @@ __device__ __forceinline__ void splitk_reduce_store(const float (&acc)[EC], floa
 
 template <int BNP, int MINB>
 __global__ void __launch_bounds__(320, MINB)
-    gemm_decode_kernel(const __grid_constant__ CUtensorMap tm_w,    // B: [N][K] e4m3
-                       const __grid_constant__ CUtensorMap tm_x,    // A: [M][K] e4m3
-                       const __grid_constant__ CUtensorMap tm_sfa,  // sfa: [KB][ld] f32
+    gemm_decode_kernel(const __grid_constant__ CUtensorMap tm_w,    // B as [KB][N][128], kg-deep boxes
+                       const __grid_constant__ CUtensorMap tm_wpf,  // B as [KB][N][128], L2 prefetch
+                       const __grid_constant__ CUtensorMap tm_x,    // A as [KB][M][128], kg-deep boxes
+                       const __grid_constant__ CUtensorMap tm_sfa,  // sfa: [KB][ld] f32, 16-row boxes
                        const __grid_constant__ DecodeArgs args) {
   using Cfg = DecodeCfg<BNP, MINB>;
-  constexpr int S = Cfg::STAGES;
-  constexpr int SS = Cfg::SS;
+  constexpr int NA = Cfg::NACC;
   constexpr int EC = Cfg::EC;
   constexpr int CH = Cfg::CH;
+  constexpr int SCH = Cfg::SCH;
+  constexpr int MS = Cfg::MAX_STAGES;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-  uint8_t* sW = smem + Cfg::OFF_W;
-  uint8_t* sX = smem + Cfg::OFF_X;
-  float* sScale = reinterpret_cast<float*>(smem + Cfg::OFF_SCALE);
-  float* recv = reinterpret_cast<float*>(smem);  // receive slots, after the main loop
-  constexpr int NA = Cfg::NACC;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+  uint8_t* sW = smem;
+  uint8_t* sX = smem + args.off_x;
+  float* sSfa = reinterpret_cast<float*>(smem + args.off_sfa);
+  float* recv = reinterpret_cast<float*>(smem + args.off_recv);
+  float* stage_out = reinterpret_cast<float*>(smem);  // over the ring, after the main loop
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + args.off_bar);
   uint64_t* full = bars;
-  uint64_t* empty = bars + S;
-  uint64_t* tfull = bars + 2 * S;
-  uint64_t* tempty = bars + 2 * S + NA;
-  uint64_t* sfull = bars + 2 * S + 2 * NA;
-  uint64_t* sempty = bars + 2 * S + 2 * NA + SS;
-  uint64_t* mma_done = bars + 2 * S + 2 * NA + 2 * SS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
+  uint64_t* empty = bars + MS;
+  uint64_t* tfull = bars + 2 * MS;
+  uint64_t* tempty = tfull + NA;
+  uint64_t* sfull = tempty + NA;
+  uint64_t* sempty = sfull + 2;
+  uint64_t* mma_done = sempty + 2;
+  uint64_t* rbar = mma_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t warp = warp_id_uniform();
   const uint32_t lane = lane_id();
   const uint64_t tmo = args.timeout_ns;
   const uint32_t rank = cluster_ctarank();
   const int splits = args.splits;
+  const int S = args.stages;
+  const int KG = args.kg;
   const int n_tile = blockIdx.y;
   const int n0 = n_tile * 128;
   const int kb_begin = static_cast<int>((static_cast<long long>(rank) * args.KB) / splits);
   const int kb_end = static_cast<int>((static_cast<long long>(rank + 1) * args.KB) / splits);
   const int nkb = kb_end - kb_begin;
+  const int R = args.rows_per_owner;
+  const int m_lo = min(args.M, static_cast<int>(rank) * R);
+  const int m_hi = min(args.M, m_lo + R);
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+  if (warp == 0) {
+    // The weight slice goes to L2 before anything else (an L2 prefetch reads
+    // nothing into the kernel, so it may precede the PDL wait).
+    const int pf0 = min(args.pf, nkb);
+    for (int j = static_cast<int>(lane) * Cfg::PF_BOX; j < pf0; j += 32 * Cfg::PF_BOX)
+      tma_prefetch_l2_3d(&tm_wpf, 0, n0, kb_begin + j);
+    // lane i initialises barrier i (tempty / sempty count the 8 promotion warps)
+    for (int i = static_cast<int>(lane); i < Cfg::NUM_BARS; i += 32) {
+      const bool by_warps = (i >= 2 * MS + NA && i < 2 * MS + 2 * NA) ||
+                            i == 2 * MS + 2 * NA + 2 || i == 2 * MS + 2 * NA + 3;
+      mbar_init(&bars[i], by_warps ? 8u : 1u);
     }
-    for (int i = 0; i < NA; ++i) {
-      mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 8);
-    }
-    for (int i = 0; i < SS; ++i) {
-      mbar_init(&sfull[i], 1);
-      mbar_init(&sempty[i], 8);
-    }
-    mbar_init(mma_done, 1);
-    *abort_flag = 0;
     fence_mbarrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm_w);
-    tma_prefetch_desc(&tm_x);
-    tma_prefetch_desc(&tm_sfa);
-  }
-  if (warp == 1) {
+    __syncwarp();
+    if (lane == 0) {
+      *abort_flag = 0;
+      // this CTA receives (splits - 1) slices of its token rows
+      if (splits > 1) mbar_arrive_expect_tx(rbar, static_cast<uint32_t>((splits - 1) * (m_hi - m_lo) * 512));
+      tma_prefetch_desc(&tm_w);
+      tma_prefetch_desc(&tm_x);
+      tma_prefetch_desc(&tm_sfa);
+    }
+  } else if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
+  if (splits > 1) cluster_arrive_relaxed();  // matched by cluster_wait() before the copies
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // The first weight tiles of this CTA go to L2 while the previous kernel on
-  // the stream (typically the activation quantiser) finishes: their DRAM
-  // latency leaves the critical path. Only a prefetch happens before the wait.
-  if (warp == 0 && lane == 0) {
-    for (int j = 0; j < S && j < nkb; ++j) tma_prefetch_l2(&tm_w, (kb_begin + j) * Cfg::BK, n0);
-  }
+  // The next launch on the stream may start (its prologue and weight
+  // prefetch) once every CTA of this grid has passed here; its PDL wait
+  // still waits for this grid to complete.
+  pdl_trigger();
   pdl_wait();  // inputs may come from the previous launch on the stream
 
   float acc[EC];
@@ -265,63 +274,96 @@ __global__ void __launch_bounds__(320, MINB)
 
   if (warp == 0) {
     // ======================= TMA producer (converged warp, lane 0 issues) ===
-    int it = 0;
-    int dropped = -1;
-    for (; it < nkb; ++it) {
-      const int s = it % S;
-      const int ss = it % SS;
-      bool ok = mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort_flag, tmo, SITE_PRODUCER_EMPTY);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      ok = mbar_wait(&sempty[ss], ((it / SS) & 1) ^ 1, abort_flag, tmo, SITE_PRODUCER_SCALE_EMPTY);
-      if (!__all_sync(0xffffffffu, ok)) break;
+    // stage i holds K-blocks [i kg, i kg + kg) of this CTA's range (the last
+    // stage's box may run past it: those K-blocks are loaded, not used)
+    const int nst = (nkb + KG - 1) / KG;
+    int i = 0;
+    int s = 0;
+    uint32_t ph = 0;
+    int nchunks = 0;  // sfa chunks loaded
+    bool dropped = false;
+    for (; i < nst; ++i) {
+      const int it = i * KG;
       const int kb = kb_begin + it;
-      if (args.drop_arrive && it == 0) {
-        dropped = 0;  // test hook: never arm stage 0
+      if (it % SCH == 0) {  // kg divides SCH: a stage never straddles two chunks
+        const int c = (it / SCH) & 1;
+        bool ok = mbar_wait(&sempty[c], ((it / (2 * SCH)) & 1) ^ 1, abort_flag, tmo,
+                            SITE_PRODUCER_SCALE_EMPTY);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sfull[c], Cfg::SFA_CHUNK_BYTES);
+          tma_load_2d(sSfa + c * (SCH * BNP), &tm_sfa, &sfull[c], 0, kb);
+        }
+        ++nchunks;
+      }
+      bool ok = mbar_wait(&empty[s], ph ^ 1, abort_flag, tmo, SITE_PRODUCER_EMPTY);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (args.drop_arrive && i == 0) {
+        dropped = true;  // test hook: never arm stage 0
       } else if (lane == 0) {
-        mbar_arrive_expect_tx(&full[s], Cfg::W_BYTES + Cfg::X_BYTES);
-        tma_load_2d(sW + s * Cfg::W_BYTES, &tm_w, &full[s], kb * Cfg::BK, n0);
-        tma_load_2d(sX + s * Cfg::X_BYTES, &tm_x, &full[s], kb * Cfg::BK, 0);
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(KG * Cfg::STAGE_BYTES));
+        tma_load_3d(sW + s * KG * Cfg::W_BYTES, &tm_w, &full[s], 0, n0, kb);
+        tma_load_3d(sX + s * KG * Cfg::X_BYTES, &tm_x, &full[s], 0, 0, kb);
       }
       if (lane == 0) {
-        mbar_arrive_expect_tx(&sfull[ss], BNP * 4);
-        tma_load_2d(sScale + ss * Cfg::SLOT_FLOATS, &tm_sfa, &sfull[ss], 0, kb);
+        // keep the L2 prefetch window `pf` K-blocks ahead, one box of 8 at a time
+        const int lo = it + args.pf;
+        for (int j = (lo + Cfg::PF_BOX - 1) / Cfg::PF_BOX * Cfg::PF_BOX; j < lo + KG && j < nkb;
+             j += Cfg::PF_BOX)
+          tma_prefetch_l2_3d(&tm_wpf, 0, n0, kb_begin + j);
       }
       __syncwarp();
+      if (++s == S) {
+        s = 0;
+        ph ^= 1;
+      }
     }
-    // bounded wait for every copy still in flight
-    for (int j = (it > S ? it - S : 0); j < it; ++j) {
-      if (j == dropped) continue;
+    // bounded wait for every copy still in flight: the last min(i, S) stages
+    // and the last two sfa chunks (earlier ones were consumed before their
+    // slot was reloaded)
+    {
       volatile int never = 0;
-      mbar_wait(&full[j % S], (j / S) & 1, &never, tmo, SITE_TEARDOWN_TMA);
-    }
-    for (int j = (it > SS ? it - SS : 0); j < it; ++j) {
-      volatile int never = 0;
-      mbar_wait(&sfull[j % SS], (j / SS) & 1, &never, tmo, SITE_TEARDOWN_TMA);
+      for (int j = (i > S ? i - S : 0); j < i; ++j) {
+        if (dropped && j == 0) continue;
+        mbar_wait(&full[j % S], (j / S) & 1, &never, tmo, SITE_TEARDOWN_TMA);
+      }
+      for (int ci = (nchunks > 2 ? nchunks - 2 : 0); ci < nchunks; ++ci)
+        mbar_wait(&sfull[ci & 1], (ci >> 1) & 1, &never, tmo, SITE_TEARDOWN_TMA);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ======================= MMA issuer (converged warp, lane 0 issues) =====
     constexpr uint32_t idesc = idesc_e4m3_f32(128, BNP, 0, 0);
-    for (int it = 0; it < nkb; ++it) {
-      const uint32_t b = static_cast<uint32_t>(it) % NA;
-      bool ok = mbar_wait(&tempty[b], ((it / NA) & 1) ^ 1, abort_flag, tmo, SITE_MMA_TMEM_EMPTY);
+    const int nst = (nkb + KG - 1) / KG;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int i = 0; i < nst; ++i) {
+      bool ok = mbar_wait(&full[s], ph, abort_flag, tmo, SITE_MMA_FULL);
       if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      const int s = it % S;
-      ok = mbar_wait(&full[s], (it / S) & 1, abort_flag, tmo, SITE_MMA_FULL);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t w_base = smem_addr(sW + s * Cfg::W_BYTES);
-        const uint32_t x_base = smem_addr(sX + s * Cfg::X_BYTES);
+      for (int j = 0; j < KG && i * KG + j < nkb; ++j) {
+        const int it = i * KG + j;
+        const uint32_t b = static_cast<uint32_t>(it) % NA;
+        ok = mbar_wait(&tempty[b], ((it / NA) & 1) ^ 1, abort_flag, tmo, SITE_MMA_TMEM_EMPTY);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t w_base = smem_addr(sW + (s * KG + j) * Cfg::W_BYTES);
+          const uint32_t x_base = smem_addr(sX + (s * KG + j) * Cfg::X_BYTES);
 #pragma unroll
-        for (int k = 0; k < Cfg::BK / 32; ++k)
-          mma_f8f6f4(tmem_base + b * BNP, smem_desc_sw128(w_base + k * 32, 16, 1024),
-                     smem_desc_sw128(x_base + k * 32, 16, 1024), idesc, k > 0 ? 1u : 0u);
-        mma_commit(&empty[s]);
-        mma_commit(&tfull[b]);
+          for (int k = 0; k < Cfg::BK / 32; ++k)
+            mma_f8f6f4(tmem_base + b * BNP, smem_desc_sw128(w_base + k * 32, 16, 1024),
+                       smem_desc_sw128(x_base + k * 32, 16, 1024), idesc, k > 0 ? 1u : 0u);
+          mma_commit(&tfull[b]);
+        }
+        __syncwarp();
       }
+      if (!ok) break;
+      if (lane == 0) mma_commit(&empty[s]);
       __syncwarp();
+      if (++s == S) {
+        s = 0;
+        ph ^= 1;
+      }
     }
     if (lane == 0) mma_commit(mma_done);
     __syncwarp();
@@ -343,27 +385,30 @@ __global__ void __launch_bounds__(320, MINB)
         const int it = it0 + u;
         if (it >= nkb) break;
         const uint32_t b = static_cast<uint32_t>(it) % NA;
+        const int c = (it / SCH) & 1;
         bool ok = mbar_wait(&tfull[b], (it / NA) & 1, abort_flag, tmo, SITE_EPI_TMEM_FULL);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) goto promo_done;
-        const int ss = it % SS;
-        bool ok2 = mbar_wait(&sfull[ss], (it / SS) & 1, abort_flag, tmo, SITE_EPI_SCALE_FULL);
-        ok2 = __all_sync(0xffffffffu, ok2);
-        if (!ok2) goto promo_done;
+        if (it % SCH == 0) {
+          bool ok2 = mbar_wait(&sfull[c], (it / (2 * SCH)) & 1, abort_flag, tmo,
+                               SITE_EPI_SCALE_FULL);
+          ok2 = __all_sync(0xffffffffu, ok2);
+          if (!ok2) goto promo_done;
+        }
         tc_fence_after();
         const float sb = sbr[u];
         if (it + 4 < nkb) sbr[u] = __ldg(pb + it + 4);
-        const float* sa = sScale + ss * Cfg::SLOT_FLOATS + h * EC;
-        auto fma_chunk = [&](int c, const uint32_t (&r)[CH]) {
+        const float* sa = sSfa + c * (SCH * BNP) + (it % SCH) * BNP + h * EC;
+        auto fma_chunk = [&](int cc, const uint32_t (&r)[CH]) {
 #pragma unroll
           for (int i = 0; i < CH; i += 4) {
-            const float4 s4 = *reinterpret_cast<const float4*>(sa + c * CH + i);
+            const float4 s4 = *reinterpret_cast<const float4*>(sa + cc * CH + i);
             float t0, t1, t2, t3;
             mul2(t0, t1, s4.x, s4.y, sb, sb);
             mul2(t2, t3, s4.z, s4.w, sb, sb);
-            fma2(acc[c * CH + i], acc[c * CH + i + 1], t0, t1, __uint_as_float(r[i]),
+            fma2(acc[cc * CH + i], acc[cc * CH + i + 1], t0, t1, __uint_as_float(r[i]),
                  __uint_as_float(r[i + 1]));
-            fma2(acc[c * CH + i + 2], acc[c * CH + i + 3], t2, t3, __uint_as_float(r[i + 2]),
+            fma2(acc[cc * CH + i + 2], acc[cc * CH + i + 3], t2, t3, __uint_as_float(r[i + 2]),
                  __uint_as_float(r[i + 3]));
           }
         };
@@ -375,37 +420,104 @@ __global__ void __launch_bounds__(320, MINB)
         if constexpr (Cfg::ALL_IN_FLIGHT) {
           uint32_t r[EC / CH][CH];
 #pragma unroll
-          for (int c = 0; c < EC / CH; ++c)
-            tmem_ld_32x32b<CH>(t_lane + b * BNP + h * EC + c * CH, r[c]);
+          for (int cc = 0; cc < EC / CH; ++cc)
+            tmem_ld_32x32b<CH>(t_lane + b * BNP + h * EC + cc * CH, r[cc]);
           tmem_ld_wait();
           release_tmem();
 #pragma unroll
-          for (int c = 0; c < EC / CH; ++c) fma_chunk(c, r[c]);
+          for (int cc = 0; cc < EC / CH; ++cc) fma_chunk(cc, r[cc]);
         } else {
 #pragma unroll
-          for (int c = 0; c < EC / CH; ++c) {
+          for (int cc = 0; cc < EC / CH; ++cc) {
             uint32_t r[CH];
-            tmem_ld_32x32b<CH>(t_lane + b * BNP + h * EC + c * CH, r);
+            tmem_ld_32x32b<CH>(t_lane + b * BNP + h * EC + cc * CH, r);
             tmem_ld_wait();
-            if (c == EC / CH - 1) release_tmem();
-            fma_chunk(c, r);
+            if (cc == EC / CH - 1) release_tmem();
+            fma_chunk(cc, r);
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sempty[ss]);
+        if (it % SCH == SCH - 1 || it == nkb - 1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sempty[c]);
+        }
       }
     }
   promo_done:;
   }
 
   // ---------------------------------------------------------- split-K reduction
-  // Every role is done and every copy / MMA has landed, so this CTA's ring is
-  // free; the first barrier (inside) makes that true for every CTA of the cluster.
+  // Every role is done and every copy / MMA of this CTA has landed, so its
+  // ring is free: the FP32 partial goes there token-major ([token][128 rows]).
   tc_fence_before();
-  pdl_trigger();
-  splitk_reduce_store<BNP, EC, Cfg::RECV_PITCH>(acc, recv, rank, splits, warp, lane, n0, args.M,
-                                                args.N, args.C, args.D);
-  // no peer touches this CTA's shared memory after the second barrier
+  __syncthreads();
+  if (warp >= 2) {
+    float* col = stage_out + h * EC * 128 + q * 32 + lane;
+#pragma unroll
+    for (int j = 0; j < EC; ++j) col[j * 128] = acc[j];
+    fence_proxy_async_smem();  // the bulk copies below read it through the async proxy
+  }
+  __syncthreads();
+  if (splits > 1) {
+    cluster_wait();  // every owner's receive barrier is initialised
+    if (threadIdx.x == 0) {
+      for (int o = 0; o < splits; ++o) {
+        if (o == static_cast<int>(rank)) continue;
+        const int lo = min(args.M, o * R);
+        const int hi = min(args.M, lo + R);
+        if (hi <= lo) continue;
+        const int slot = static_cast<int>(rank) < o ? static_cast<int>(rank) : static_cast<int>(rank) - 1;
+        const uint32_t dst = dsmem_addr(smem_addr(recv + slot * R * 128), static_cast<uint32_t>(o));
+        const uint32_t mb = dsmem_addr(smem_addr(rbar), static_cast<uint32_t>(o));
+        bulk_copy_to_cluster(dst, stage_out + lo * 128, static_cast<uint32_t>((hi - lo) * 512), mb);
+      }
+      bulk_commit();
+    }
+  }
+  bool ok = true;
+  if (splits > 1 && m_hi > m_lo) {
+    volatile int never = 0;
+    ok = mbar_wait(rbar, 0, &never, tmo, SITE_SPLITK_RECV);
+  }
+  if (ok && !*abort_flag) {
+    // this CTA's token rows: item = (token m, 8 weight rows), weight rows fastest
+    const int items = (m_hi - m_lo) * 16;
+    for (int itm = threadIdx.x; itm < items; itm += blockDim.x) {
+      const int m = m_lo + (itm >> 4);
+      const int c8 = (itm & 15) << 3;
+      const int gn = n0 + c8;
+      if (gn >= args.N) continue;  // N % 8 == 0: a group of 8 is wholly in or out
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int src = 0; src < splits; ++src) {  // rank order: deterministic
+        const float* p;
+        if (src == static_cast<int>(rank)) {
+          p = stage_out + m * 128 + c8;
+        } else {
+          const int slot = src < static_cast<int>(rank) ? src : src - 1;
+          p = recv + (slot * R + (m - m_lo)) * 128 + c8;
+        }
+        const float4 a = *reinterpret_cast<const float4*>(p);
+        const float4 b = *reinterpret_cast<const float4*>(p + 4);
+        v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+        v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+      }
+      const long long o = static_cast<long long>(m) * args.N + gn;
+      if (args.C) {
+        const uint4 c4 = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(args.C) + o);
+        v[0] += bf16_lo(c4.x); v[1] += bf16_hi(c4.x);
+        v[2] += bf16_lo(c4.y); v[3] += bf16_hi(c4.y);
+        v[4] += bf16_lo(c4.z); v[5] += bf16_hi(c4.z);
+        v[6] += bf16_lo(c4.w); v[7] += bf16_hi(c4.w);
+      }
+      uint4 out;
+      out.x = pack_bf16x2(v[0], v[1]);
+      out.y = pack_bf16x2(v[2], v[3]);
+      out.z = pack_bf16x2(v[4], v[5]);
+      out.w = pack_bf16x2(v[6], v[7]);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.D) + o) = out;
+    }
+  }
+  // this CTA's partial must stay until the copies to its peers have read it
+  if (splits > 1 && threadIdx.x == 0) bulk_wait_read0();
 
   if (warp == 1) {
     tc_fence_after();

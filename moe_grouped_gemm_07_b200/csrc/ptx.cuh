@@ -116,6 +116,15 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m, uint64_t* bar,
+                                            int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_addr(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // Untiled bulk copy global -> shared of `bytes` bytes (both addresses 16-byte
 // aligned, bytes a multiple of 16), completing on `bar` with complete_tx.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes,
@@ -134,6 +143,16 @@ __device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* m, int32_t x,
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
                    reinterpret_cast<uint64_t>(m)),
                "r"(x), "r"(y)
+               : "memory");
+}
+
+// 3-D variant of tma_prefetch_l2 (one instruction covers a box of several
+// K-blocks of a weight tile).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int32_t x, int32_t y,
+                                                   int32_t z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(z)
                : "memory");
 }
 
@@ -368,6 +387,30 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile(
       "barrier.cluster.arrive.release.aligned;\n\t"
       "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Split cluster barrier: every thread of every CTA arrives (no ordering of
+// earlier memory operations beyond what a preceding fence gives, e.g.
+// fence_mbarrier_init for barrier initialisation) and later waits.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// Bulk copy of `bytes` bytes (multiple of 16, both addresses 16-byte aligned)
+// from this CTA's shared memory into shared memory of a CTA of the cluster
+// (`dst_cluster`, a shared::cluster address), completing `bytes` transaction
+// bytes on the destination CTA's mbarrier at `mbar_cluster`. Tracked by the
+// issuing thread's bulk async group (bulk_commit / bulk_wait_read0).
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, const void* src,
+                                                     uint32_t bytes, uint32_t mbar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster),
+      "r"(smem_addr(src)), "r"(bytes), "r"(mbar_cluster)
+      : "memory");
 }
 
 // Address of the same shared-memory offset in CTA `rank` of this cluster.

@@ -147,8 +147,8 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
                                                         float* __restrict__ scales, int ld,
                                                         uint8_t* __restrict__ packed) {
   constexpr int U = 2;  // rounds of 4 strips in flight per warp
+  pdl_trigger();  // the next launch's PDL wait still waits for this grid
   pdl_wait();
-  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int g = lane >> 3;   // strip of this lane within a round
   const int li = lane & 7;   // 16-value slice of the strip
@@ -220,8 +220,8 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
                                                           float* __restrict__ scales,
                                                           uint8_t* __restrict__ packed) {
   __shared__ float red[8];
+  pdl_trigger();  // the next launch's PDL wait still waits for this grid
   pdl_wait();
-  pdl_trigger();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int kbs = cols >> 7, nbs = (rows + 127) >> 7;
   const int64_t blk = blockIdx.x;
@@ -280,8 +280,8 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const void* __restrict__
   __shared__ float red[16][64];
   __shared__ float sc_s[64];
   __shared__ float rc_s[64];
+  pdl_trigger();  // the next launch's PDL wait still waits for this grid
   pdl_wait();
-  pdl_trigger();
   const int cg = threadIdx.x & 15, rg = threadIdx.x >> 4;
   const int slabs = (cols + 63) >> 6, rbs = rows >> 7;
   const int64_t blk = blockIdx.x;
@@ -365,8 +365,8 @@ __global__ void __launch_bounds__(256) quant_fp4_kernel(const void* __restrict__
                                                         float* __restrict__ scales,
                                                         uint8_t* __restrict__ packed) {
   constexpr int U = 2;
+  pdl_trigger();  // the next launch's PDL wait still waits for this grid
   pdl_wait();
-  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int g = lane >> 3;
   const int li = lane & 7;

@@ -27,6 +27,12 @@ def sample_rows(M, extra, seed):
     return np.array(sorted(base | set(int(r) for r in rnd)), dtype=np.int64)
 
 
+def stripe(M, seed):
+    """One whole 128-row tile of an M-row output at a seeded tile position."""
+    t = int(synth.u64(1, seed)[0] % np.uint64((M + 127) // 128))
+    return np.arange(128 * t, min(M, 128 * t + 128), dtype=np.int64)
+
+
 @pytest.mark.parametrize("NK", wl.DENSE_NK)
 def test_dense_sweep_full_size(NK):
     """Workload 2: every M of the sweep for one (N, K) weight."""
@@ -58,10 +64,15 @@ def test_contiguous_full_size():
     D = torch.full((w.Mt, w.N), SENTINEL, dtype=torch.int16, device=dev()).view(torch.bfloat16)
     dg.dg_m_grouped_fp8_gemm_nt_contiguous(qa, sa, qb, sb, to_dev(w.m_indices), None, D)
     oqb, osb = oracle.quantize(w.B, oracle.BLOCK_128x128)
+    # per expert: its first, middle and last row, plus one whole 128-row tile
+    # (every row a tile holds) at a seeded tile position inside the expert
     rows = []
     off = 0
+    pick = synth.u64(w.G, synth.seed(62, 0))
     for g, r in enumerate(w.rows):
         rows += [off, off + r - 1, off + r // 2]
+        t = int(pick[g] % np.uint64((r + 127) // 128))
+        rows += [x for x in range(off + 128 * t, off + 128 * t + 128) if x < off + r]
         off += wl.align(r)
     rows = np.array(sorted(set(rows)), dtype=np.int64)
     oqa, osa = oracle.quantize(np.ascontiguousarray(w.A[rows]), oracle.ROW_1x128)
@@ -104,7 +115,7 @@ def test_k_grouped_full_size():
     qb, sb = dg.dg_quantize_fp8(to_dev(w.B), dg.DG_QUANT_COL_128x1)
     D = to_dev(w.C)
     dg.dg_k_grouped_fp8_gemm_tn_contiguous(qa, sa, qb, sb, w.ks, D, D)
-    rows = sample_rows(w.M, 4, synth.seed(61, 0))
+    rows = np.union1d(sample_rows(w.M, 4, synth.seed(61, 0)), stripe(w.M, synth.seed(61, 1)))
     # the oracle quantises the sampled columns of A (COL mode is per column)
     oqa_s, osa_s = oracle.quantize(np.ascontiguousarray(w.A[:, rows]), oracle.COL_128x1)
     oqb, osb = oracle.quantize(w.B, oracle.COL_128x1)
@@ -112,3 +123,21 @@ def test_k_grouped_full_size():
     R = oracle.k_grouped_tn(oqa_s, osa_s, oqb, osb, w.ks, Cs)
     Dn = D.cpu().numpy()[:, rows, :].astype(np.float64)
     check_close(Dn, R, "k-grouped full")
+
+
+def test_dense_weight_gradient_full_size():
+    """The dense weight gradient dW = C + dY^T X (both operands stored
+    K-outer, FP32 accumulated onto C) is the K-grouped TN entry point with a
+    single group: M=4096, N=7168, K=4096, in place on C."""
+    w = wl.k_grouped(G=1, M=4096, N=7168, ks=[4096], cfg=5, shape=1)
+    qa, sa = dg.dg_quantize_fp8(to_dev(w.A), dg.DG_QUANT_COL_128x1)
+    qb, sb = dg.dg_quantize_fp8(to_dev(w.B), dg.DG_QUANT_COL_128x1)
+    D = to_dev(w.C)
+    dg.dg_k_grouped_fp8_gemm_tn_contiguous(qa, sa, qb, sb, w.ks, D, D)
+    rows = np.union1d(sample_rows(w.M, 4, synth.seed(61, 2)), stripe(w.M, synth.seed(61, 3)))
+    oqa_s, osa_s = oracle.quantize(np.ascontiguousarray(w.A[:, rows]), oracle.COL_128x1)
+    oqb, osb = oracle.quantize(w.B, oracle.COL_128x1)
+    Cs = np.ascontiguousarray(w.C[:, rows, :])
+    R = oracle.k_grouped_tn(oqa_s, osa_s, oqb, osb, w.ks, Cs)
+    Dn = D.cpu().numpy()[:, rows, :].astype(np.float64)
+    check_close(Dn, R, "dense weight gradient (G = 1)")
