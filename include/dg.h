@@ -23,7 +23,9 @@
  *     and launches nothing.
  *   - Device-side waits are bounded: a wait that exceeds the timeout (default
  *     2 s) records DG_ERR_TIMEOUT in a per-device error word, and the kernel
- *     exits cleanly; read it with dg_get_last_device_error().
+ *     exits cleanly; read it with dg_get_last_device_error(). The output of a
+ *     launch that timed out is undefined (some tiles may be written, others
+ *     not); inputs are never written.
  *   - E4M3 bytes are the OCP OFP8 "E4M3FN" encoding (torch.float8_e4m3fn).
  */
 #ifndef DG_H
@@ -306,7 +308,12 @@ int dg_get_pdl(void);
 /* Synchronises `stream`, then reads and clears this device's error word.
  * Returns DG_OK, DG_ERR_TIMEOUT (a bounded wait ran out; *site gets the code
  * of the wait that gave up, if site != NULL), DG_ERR_INVALID_ARG (device-side
- * sizes were invalid, site 9) or DG_ERR_CUDA. Debug/test use. */
+ * sizes were invalid, site 9) or DG_ERR_CUDA. Debug/test use.
+ * The error word is one per device, shared by every stream: it holds the
+ * first error any launch on the device recorded since the last read. Call
+ * this when no other stream has work of this library in flight; otherwise an
+ * error recorded by a launch on another stream may be reported here (or
+ * recorded between the read and the clear and lost). */
 dg_status dg_get_last_device_error(void* stream, int* site);
 
 /* Test hook: when nonzero, the next GEMM launch drops one producer arrive so

@@ -6,7 +6,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -256,6 +258,13 @@ int tail_split_for(long long tiles, int grid, int KB) {
   return KB - KB / k >= 40 ? k : 1;
 }
 
+// The occupancy probes below may leave an error of their own in the
+// runtime's last-error slot, which they clear. So that this never swallows an
+// error of the caller's earlier asynchronous work, a probe runs only when no
+// error is pending (otherwise it reports "unknown" and caches nothing, and
+// the caller's error stays pending for its own check).
+bool no_pending_error() { return cudaPeekAtLastError() == cudaSuccess; }
+
 // How many k-CTA clusters of the split-K kernel the device runs at once
 // (cached per device and k; 0 on error).
 int splitk_clusters(int dev, int k) {
@@ -265,6 +274,7 @@ int splitk_clusters(int dev, int k) {
   static bool done[kMaxDevices][9];
   std::lock_guard<std::mutex> lock(mu);
   if (!done[dev][k]) {
+    if (!no_pending_error()) return 0;
     done[dev][k] = true;
     cache[dev][k] = 0;
     auto kern = dg::gemm_fp8_kernel<dg::MODE_SPLITK, 256>;
@@ -287,6 +297,20 @@ int splitk_clusters(int dev, int k) {
     cudaGetLastError();
   }
   return cache[dev][k];
+}
+
+// NT scale ring: sfb viewed as [G * ceil(N/128)][K/128] FP32 with 4 x 2
+// boxes (four K-blocks of two 128-column blocks), when its rows are a
+// multiple of 16 bytes long (K/128 % 4 == 0); otherwise the kernel reads sfb
+// with plain loads. Sets args->sfb_tma accordingly.
+void make_sfb_box_map(CUtensorMap* m, const float* sfb, int N, int K, int G, GemmArgs* args) {
+  const int kbn = K / 128;
+  const int nbn = (N + 127) / 128;
+  args->sfb_tma = 0;
+  if (kbn % 4 != 0) return;
+  if (make_map_2d(m, sfb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, kbn, static_cast<uint64_t>(G) * nbn,
+                  4ull * kbn, 4, 2, CU_TENSOR_MAP_SWIZZLE_NONE) == DG_OK)
+    args->sfb_tma = 1;
 }
 
 template <int MODE>
@@ -337,6 +361,8 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
   args.D = D;
   args.timeout_ns = timeout_ns();
   args.drop_arrive = take_drop_flag();
+  CUtensorMap tsb = dummy;
+  make_sfb_box_map(&tsb, sfb, N, K, G, &args);
   const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(sms, tiles)));
   // Dense: a partial last wave of R tiles runs as a second launch that
   // splits each tile along K over a cluster of k CTAs (MODE_SPLITK); the
@@ -354,17 +380,17 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
   if (split > 1) {
     GemmArgs tail = args;
     args.total_tiles = static_cast<int>(tiles - R);
-    dg_status s2 = launch_gemm<MODE, 256>(ta, tb, dummy, dummy, td, args, grid, st, dev);
+    dg_status s2 = launch_gemm<MODE, 256>(ta, tb, dummy, tsb, td, args, grid, st, dev);
     if (s2 != DG_OK) return s2;
     tail.total_tiles = static_cast<int>(R);
     tail.split_tile0 = static_cast<int>(tiles - R);
     tail.split = split;
     tail.drop_arrive = 0;
-    return launch_gemm<dg::MODE_SPLITK, 256>(ta, tb, dummy, dummy, td, tail,
+    return launch_gemm<dg::MODE_SPLITK, 256>(ta, tb, dummy, tsb, td, tail,
                                              static_cast<int>(R) * split, st, dev, split);
   }
-  if (bn == 256) return launch_gemm<MODE, 256>(ta, tb, dummy, dummy, td, args, grid, st, dev);
-  return launch_gemm<MODE, 128>(ta, tb, dummy, dummy, td, args, grid, st, dev);
+  if (bn == 256) return launch_gemm<MODE, 256>(ta, tb, dummy, tsb, td, args, grid, st, dev);
+  return launch_gemm<MODE, 128>(ta, tb, dummy, tsb, td, args, grid, st, dev);
 }
 
 // Dense GEMM with A and/or B stored MN-major (NN, TN, TT); 128 x 256 tiles.
@@ -414,11 +440,13 @@ dg_status run_layout(const void* A, const float* sfa, int ld_sfa, const void* B,
   args.D = D;
   args.timeout_ns = timeout_ns();
   args.drop_arrive = take_drop_flag();
+  CUtensorMap tsb = dummy;
+  if (MODE == dg::MODE_TT) make_sfb_box_map(&tsb, sfb, N, K, 1, &args);  // B stored [N][K]
   const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(sms, tiles)));
   if (print_configs())
     std::fprintf(stderr, "[dg] %s M=%d N=%d K=%d: BM=128 BN=256 tiles=%lld grid=%d\n", name, M, N,
                  K, tiles, grid);
-  return launch_gemm<MODE, 256>(ta, tb, dummy, dummy, td, args, grid, st, dev);
+  return launch_gemm<MODE, 256>(ta, tb, dummy, tsb, td, args, grid, st, dev);
 }
 
 // Shared argument checks of the dense entry points. a_mn / b_mn: the operand
@@ -515,14 +543,16 @@ dg_status run_pair(const void* A, const float* sfa, int ld_sfa, const void* B, c
   args.d_rows = M;
   args.timeout_ns = timeout_ns();
   args.drop_arrive = take_drop_flag();
+  CUtensorMap tsb = dummy;
+  make_sfb_box_map(&tsb, sfb, N, K, 1, &args);
   const int pairs = static_cast<int>(std::max<long long>(1, std::min<long long>(sms / 2, tiles)));
   if (print_configs())
     std::fprintf(stderr,
                  "[dg] fp8_gemm_nt pairs M=%d N=%d K=%d: 256x%d tiles=%lld on %d CTA pairs\n", M,
                  N, K, bn, tiles, pairs);
   if (bn == 256)
-    return launch_gemm<dg::MODE_PAIR, 256>(ta, tb, dummy, dummy, td, args, 2 * pairs, st, dev, 2);
-  return launch_gemm<dg::MODE_PAIR, 128>(ta, tb, dummy, dummy, td, args, 2 * pairs, st, dev, 2);
+    return launch_gemm<dg::MODE_PAIR, 256>(ta, tb, dummy, tsb, td, args, 2 * pairs, st, dev, 2);
+  return launch_gemm<dg::MODE_PAIR, 128>(ta, tb, dummy, tsb, td, args, 2 * pairs, st, dev, 2);
 }
 
 // ---------------------------------------------------------------- decode path
@@ -532,6 +562,7 @@ dg_status run_pair(const void* A, const float* sfa, int ld_sfa, const void* B, c
 // Largest cluster size (<= 16, or 8 without non-portable sizes) of which
 // enough co-resident clusters fit to fill most of the GPU; 0 on failure.
 int probe_max_cluster(const void* kern, int smem) {
+  if (!no_pending_error()) return -1;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return 0;
   const bool nonportable =
@@ -556,27 +587,42 @@ int probe_max_cluster(const void* kern, int smem) {
   return 0;
 }
 
+// Caches a probe's answer per device unless the probe could not run (-1: an
+// earlier error was pending).
+template <typename Probe>
+int cached_probe(std::mutex& mu, int (&best)[kMaxDevices], bool (&done)[kMaxDevices], int dev,
+                 Probe probe) {
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
+    const int r = probe();
+    if (r < 0) return r;
+    best[dev] = r;
+    done[dev] = true;
+  }
+  return best[dev];
+}
+
 template <int BNP, int MINB>
 int max_cluster(int dev) {
-  static std::once_flag once[kMaxDevices];
+  static std::mutex mu;
   static int best[kMaxDevices];
-  std::call_once(once[dev], [&] {
-    best[dev] = probe_max_cluster(reinterpret_cast<const void*>(dg::gemm_decode_kernel<BNP, MINB>),
-                                  dg::DecodeCfg<BNP, MINB>::SMEM_BUDGET);
+  static bool done[kMaxDevices];
+  return cached_probe(mu, best, done, dev, [] {
+    return probe_max_cluster(reinterpret_cast<const void*>(dg::gemm_decode_kernel<BNP, MINB>),
+                             dg::DecodeCfg<BNP, MINB>::SMEM_BUDGET);
   });
-  return best[dev];
 }
 
 template <int BNP, int MINB, bool W4>
 int max_cluster_mx(int dev) {
-  static std::once_flag once[kMaxDevices];
+  static std::mutex mu;
   static int best[kMaxDevices];
-  std::call_once(once[dev], [&] {
-    best[dev] = probe_max_cluster(
+  static bool done[kMaxDevices];
+  return cached_probe(mu, best, done, dev, [] {
+    return probe_max_cluster(
         reinterpret_cast<const void*>(dg::gemm_mx_decode_kernel<BNP, MINB, W4>),
         dg::MxDecodeCfg<BNP, MINB, W4>::SMEM_BYTES);
   });
-  return best[dev];
 }
 
 // Decode plan: CTAs per SM (MINB) and split count, from a sweep of both
@@ -601,6 +647,51 @@ int decode_prefetch_kblocks() {
     if (f >= 0) pf = f;
   }
   return (pf + 7) / 8 * 8;
+}
+
+// How many clusters of `s` CTAs of this decode configuration, with `smem`
+// bytes of shared memory each, the device runs at once (cached per device,
+// configuration, s and smem; 0 on error). A cluster lives inside one GPC, so
+// e.g. clusters of 7 one-CTA-per-SM CTAs leave SMs of every GPC idle and
+// fewer of them fit than SMs / 7.
+template <int BNP, int MINB>
+int decode_cluster_capacity(int dev, int s, int smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  if (s < 1 || s > 8) return 0;
+  const auto key = std::make_tuple(dev, s, smem);
+  auto f = cache.find(key);
+  if (f != cache.end()) return f->second;
+  if (!no_pending_error()) return 0;
+  int cap = 0;
+  const void* kern = reinterpret_cast<const void*>(dg::gemm_decode_kernel<BNP, MINB>);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           dg::DecodeCfg<BNP, MINB>::SMEM_BUDGET) == cudaSuccess) {
+    if (s > 1) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(s, 1, 1);
+      cfg.blockDim = dim3(320, 1, 1);
+      cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = s;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess) cap = n;
+    } else {
+      int per_sm = 0, sms = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 320, smem) == cudaSuccess &&
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+        cap = per_sm * sms;
+    }
+  }
+  cudaGetLastError();  // only the queries' own errors can be pending here
+  cache[key] = cap;
+  return cap;
 }
 
 DecodePlan plan_decode(int M, int n_tiles, int KB, int sms, int cap1, int cap2) {
@@ -647,6 +738,20 @@ bool decode_layout(int M, int splits, int kg, dg::DecodeArgs* a, int* smem_bytes
   a->off_bar = a->off_recv + static_cast<uint32_t>(recv);
   *smem_bytes = static_cast<int>(a->off_bar) + Cfg::BAR_BYTES + 1024;
   return *smem_bytes <= Cfg::SMEM_BUDGET;
+}
+
+// Lowers `splits` until every cluster of the launch (with its shared-memory
+// layout) is resident at once.
+template <int BNP, int MINB>
+int fit_splits(int dev, int M, int n_tiles, int splits) {
+  for (; splits > 1; --splits) {
+    dg::DecodeArgs a;
+    int smem = 0;
+    bool fits = false;
+    for (int kg = 4; kg >= 1 && !fits; kg /= 2) fits = decode_layout<BNP, MINB>(M, splits, kg, &a, &smem);
+    if (fits && decode_cluster_capacity<BNP, MINB>(dev, splits, smem) >= n_tiles) break;
+  }
+  return splits;
 }
 
 template <int BNP, int MINB>
@@ -740,19 +845,24 @@ dg_status dispatch_decode(const void* A, const float* sfa, const void* B, const 
     const int f = std::atoi(e);
     if (f >= 1) p.splits = std::max(1, std::min(std::min(f, std::min(cap, 8)), KB));
   }
+  const bool forced = std::getenv("DG_DECODE_SPLITS") != nullptr;
+#define DG_RUN_DECODE(BNP_, MINB_)                                                         \
+  return run_decode<BNP_, MINB_>(A, sfa, B, sfb, C, D, M, N, K,                            \
+                                 forced ? p.splits : fit_splits<BNP_, MINB_>(dev, M, n_tiles, p.splits), st)
   switch (bnp) {
     case 16:
-      return p.minb == 1 ? run_decode<16, 1>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st)
-                         : run_decode<16, 2>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st);
+      if (p.minb == 1) DG_RUN_DECODE(16, 1);
+      DG_RUN_DECODE(16, 2);
     case 32:
-      return p.minb == 1 ? run_decode<32, 1>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st)
-                         : run_decode<32, 2>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st);
+      if (p.minb == 1) DG_RUN_DECODE(32, 1);
+      DG_RUN_DECODE(32, 2);
     case 64:
-      return p.minb == 1 ? run_decode<64, 1>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st)
-                         : run_decode<64, 2>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st);
+      if (p.minb == 1) DG_RUN_DECODE(64, 1);
+      DG_RUN_DECODE(64, 2);
     default:
-      return run_decode<128, 1>(A, sfa, B, sfb, C, D, M, N, K, p.splits, st);
+      DG_RUN_DECODE(128, 1);
   }
+#undef DG_RUN_DECODE
 }
 
 // Block-scaled small-M launcher (swap-AB, cluster split-K; W4: E2M1 weights).

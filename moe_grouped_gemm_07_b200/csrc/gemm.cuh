@@ -73,6 +73,7 @@ struct GemmArgs {
   const int32_t* ks_dev;        // K-grouped, device sizes: [G] K per group (else null)
   int kb_cap;                   // K-grouped, device sizes: K-blocks the operands hold
   int split_tile0, split;       // MODE_SPLITK: first tail tile, CTAs per tile
+  int sfb_tma;                  // NT: sfb comes through the scale ring (tm_sfb), else __ldg
 };
 
 template <int MODE, int BN_>
@@ -102,9 +103,14 @@ struct GemmCfg {
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_SCALE = OFF_B + STAGES * B_BYTES;
   // NT modes: a ring of SCALE_SLOTS K-blocks of sfa for the tile's BM rows,
-  // filled by the producer's bulk copies (the sfb value of a column half is
-  // one float per K-block, read by the promotion warps themselves)
-  static constexpr int NT_SCALE_BYTES = BM * 4;
+  // filled by the producer's bulk copies, each slot followed (at a 128-byte
+  // boundary) by a 2 x 4 box of sfb: the two column halves' 128-column
+  // blocks x the four K-blocks around this one, loaded by TMA (when the sfb
+  // rows are a multiple of 16 bytes long; otherwise the promotion warps read
+  // sfb themselves)
+  static constexpr int NT_SLOT_FLOATS = BM + 32;
+  static constexpr int NT_SCALE_BYTES = NT_SLOT_FLOATS * 4;
+  static constexpr int SFB_BOX_BYTES = 2 * 4 * 4;
   static constexpr int OFF_STAGE =
       ((OFF_SCALE + SCALE_SLOTS * (KG ? SCALE_BYTES : NT_SCALE_BYTES) + 1023) / 1024) * 1024;
   // output staging for the TMA-store epilogue: one 32-row x 64-byte chunk
@@ -345,6 +351,8 @@ __global__ void __launch_bounds__(320, 1)
     if constexpr (Cfg::KG) {
       tma_prefetch_desc(&tm_sfa);
       tma_prefetch_desc(&tm_sfb);
+    } else if (args.sfb_tma) {
+      tma_prefetch_desc(&tm_sfb);
     }
   }
   if (warp == 1) {
@@ -457,42 +465,52 @@ __global__ void __launch_bounds__(320, 1)
                            SITE_PRODUCER_SCALE_EMPTY);
             if (!__all_sync(0xffffffffu, ok)) goto producer_done;
           }
+          // One thread's TMA copies are processed one after another (about
+          // 60 GB/s per thread with 16 KB boxes on B200); copies issued by
+          // different lanes proceed side by side. So lane 0 arms the
+          // barrier, then lane 0 loads A and lane 1 (lanes 1..2 for an
+          // MN-major B) the B tile, in parallel.
           if (args.drop_arrive && it == 0) {  // test hook: never arm stage 0
             dropped = 0;
-          } else if (lane == 0) {
+          } else {
             if constexpr (PAIR) {
               // the leader's barrier counts the bytes of both CTAs' loads
-              if (leader) mbar_arrive_expect_tx(&full[s], 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
+              if (lane == 0 && leader)
+                mbar_arrive_expect_tx(&full[s], 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
+              __syncwarp();
               const uint32_t fb = dsmem_addr(smem_addr(&full[s]), 0);
               const int kk = kb * Cfg::BK;
-              tma_load_2d_pair(sA + s * Cfg::A_BYTES, &tm_a, fb, kk, tl.a_row);
-              tma_load_2d_pair(sB + s * Cfg::B_BYTES, &tm_b, fb, kk, tl.b_row);
+              if (lane == 0) tma_load_2d_pair(sA + s * Cfg::A_BYTES, &tm_a, fb, kk, tl.a_row);
+              if (lane == 1) tma_load_2d_pair(sB + s * Cfg::B_BYTES, &tm_b, fb, kk, tl.b_row);
             } else {
-              mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES);
+              if (lane == 0) mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES);
+              __syncwarp();
               const int kk = (tl.kb0 + kb) * Cfg::BK;
               // MN-major operands: 128-element-wide boxes of BK K-rows (x = MN)
-              if constexpr (Cfg::A_MN)
-                tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], tl.a_row, kk);
-              else
-                tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], kk, tl.a_row);
+              if (lane == 0) {
+                if constexpr (Cfg::A_MN)
+                  tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], tl.a_row, kk);
+                else
+                  tma_load_2d(sA + s * Cfg::A_BYTES, &tm_a, &full[s], kk, tl.a_row);
+              }
               if constexpr (Cfg::B_MN) {
-#pragma unroll
-                for (int h = 0; h < BN / 128; ++h)
+                if (lane >= 1 && lane <= BN / 128) {
+                  const int h = static_cast<int>(lane) - 1;
                   tma_load_2d(sB + s * Cfg::B_BYTES + h * 128 * Cfg::BK, &tm_b, &full[s],
                               tl.b_row + h * 128, kk);
+                }
               } else {
-                tma_load_2d(sB + s * Cfg::B_BYTES, &tm_b, &full[s], kk, tl.b_row);
+                if (lane == 1) tma_load_2d(sB + s * Cfg::B_BYTES, &tm_b, &full[s], kk, tl.b_row);
               }
             }
           }
           if constexpr (Cfg::KG) {
             const uint32_t ss = sit % SS;
-            if (lane == 0) {
-              mbar_arrive_expect_tx(&sfull[ss], Cfg::SCALE_BYTES);
-              float* slot = sScale + ss * (Cfg::BM + BN);
-              tma_load_2d(slot, &tm_sfa, &sfull[ss], tl.m0, tl.kb0 + kb);
-              tma_load_2d(slot + Cfg::BM, &tm_sfb, &sfull[ss], tl.n0, tl.kb0 + kb);
-            }
+            if (lane == 0) mbar_arrive_expect_tx(&sfull[ss], Cfg::SCALE_BYTES);
+            __syncwarp();
+            float* slot = sScale + ss * (Cfg::BM + BN);
+            if (lane == 3) tma_load_2d(slot, &tm_sfa, &sfull[ss], tl.m0, tl.kb0 + kb);
+            if (lane == 4) tma_load_2d(slot + Cfg::BM, &tm_sfb, &sfull[ss], tl.n0, tl.kb0 + kb);
           } else {
             // sfa of the tile's rows for this K-block: BM contiguous floats of
             // the MN-major [K/128][ld] layout ([G][K/128][ld] when masked),
@@ -500,16 +518,24 @@ __global__ void __launch_bounds__(320, 1)
             // the size is a multiple of 16 bytes); rows the copy leaves out
             // lie past M and get zero scales in the promotion
             const uint32_t ss = sit % SS;
-            if (lane == 0) {
-              const int nrows = min(Cfg::BM, args.ld_sfa - tl.m0);
-              const uint32_t bytes = nrows > 0 ? static_cast<uint32_t>(nrows) * 4u : 0u;
-              mbar_arrive_expect_tx(&sfull[ss], bytes);
-              if (bytes > 0) {
-                long long off = static_cast<long long>(tl.kb0 + kb) * args.ld_sfa + tl.m0;
-                if constexpr (MODE == MODE_MASKED)
-                  off += static_cast<long long>(tl.g) * (args.K / Cfg::BK) * args.ld_sfa;
-                bulk_load(sScale + ss * Cfg::BM, args.sfa + off, bytes, &sfull[ss]);
-              }
+            const int nrows = min(Cfg::BM, args.ld_sfa - tl.m0);
+            const uint32_t bytes = nrows > 0 ? static_cast<uint32_t>(nrows) * 4u : 0u;
+            const bool sfb_box = !Cfg::B_MN && args.sfb_tma;
+            if (lane == 0)
+              mbar_arrive_expect_tx(&sfull[ss], bytes + (sfb_box ? Cfg::SFB_BOX_BYTES : 0u));
+            __syncwarp();
+            float* slot = sScale + ss * Cfg::NT_SLOT_FLOATS;
+            if (lane == 3 && bytes > 0) {
+              long long off = static_cast<long long>(tl.kb0 + kb) * args.ld_sfa + tl.m0;
+              if constexpr (MODE == MODE_MASKED)
+                off += static_cast<long long>(tl.g) * (args.K / Cfg::BK) * args.ld_sfa;
+              bulk_load(slot, args.sfa + off, bytes, &sfull[ss]);
+            }
+            if (lane == 4 && sfb_box) {
+              // sfb viewed as [G * ceil(N/128)][K/128]: rows of the tile's two
+              // column halves, the 4 K-blocks whose group holds this one
+              const int row = tl.g * ((args.N + 127) / 128) + tl.n0 / 128;
+              tma_load_2d(slot + Cfg::BM, &tm_sfb, &sfull[ss], (tl.kb0 + kb) & ~3, row);
             }
           }
           ++sit;
@@ -645,7 +671,7 @@ __global__ void __launch_bounds__(320, 1)
         // sfb is [G][ceil(N/128)][K/128], or [K/128][ceil(N/128)] for B stored [K][N]
         pb = Cfg::B_MN ? col_first / 128 : (tl.g * nbN + col_first / 128) * KBn;
         if constexpr (SPLITK) pb += tl.kb0;  // this part starts at K-block kb0
-        if (half_in && tl.nkb > 0) sb_next = sfb_at(0);
+        if (half_in && tl.nkb > 0 && (Cfg::B_MN || !args.sfb_tma)) sb_next = sfb_at(0);
       }
 
       for (int kb = 0; kb < tl.nkb; ++kb) {
@@ -659,12 +685,17 @@ __global__ void __launch_bounds__(320, 1)
           bool ok2 = mbar_wait(&sfull[ss], (sit / SS) & 1, abort_flag, tmo, SITE_EPI_SCALE_FULL);
           ok2 = __all_sync(0xffffffffu, ok2);
           if (!ok2) goto epi_done;
-          const float sa = row_in ? sScale[ss * Cfg::BM + r_in_tile] : 0.f;
+          const float* slot = sScale + ss * Cfg::NT_SLOT_FLOATS;
+          const float sa = row_in ? slot[r_in_tile] : 0.f;
+          float sb = sb_next;
+          if (!Cfg::B_MN && args.sfb_tma)  // this half's 128-column block (both halves of a 128-wide tile share one)
+            sb = half_in ? slot[Cfg::BM + (h * EC / 128) * 4 + ((tl.kb0 + kb) & 3)] : 0.f;
           __syncwarp();
           if (lane == 0) mbar_arrive(&sempty[ss]);  // the slot may be refilled
           ++sit;
-          const float sc = sa * sb_next;
-          sb_next = (half_in && kb + 1 < tl.nkb) ? sfb_at(kb + 1) : 0.f;
+          const float sc = sa * sb;
+          if (Cfg::B_MN || !args.sfb_tma)
+            sb_next = (half_in && kb + 1 < tl.nkb) ? sfb_at(kb + 1) : 0.f;
           auto release_tmem = [&]() {
             tc_fence_before();
             __syncwarp();
