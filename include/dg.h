@@ -338,6 +338,9 @@ uint64_t dg_get_launch_count(void);
  *   DG_DECODE_MINB=1|2, DG_DECODE_SPLITS=s
  *                        CTAs per SM and split count of the M <= 128 kernels;
  *                        read on every call.
+ *   DG_DECODE_BNP=64     65..128 tokens as two 64-token tiles on half an SM
+ *                        each instead of one 128-token tile (FP8 M <= 128
+ *                        kernel); read on every call.
  *   DG_DECODE_KG=1|2|4   K-blocks per ring stage (one TMA box each for weights
  *                        and tokens) of the FP8 M <= 128 kernel; read on every
  *                        call.

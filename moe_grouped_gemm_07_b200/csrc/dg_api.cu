@@ -694,12 +694,13 @@ int decode_cluster_capacity(int dev, int s, int smem) {
   return cap;
 }
 
-DecodePlan plan_decode(int M, int n_tiles, int KB, int sms, int cap1, int cap2) {
+DecodePlan plan_decode(int bnp, int m_tiles, int n_tiles, int KB, int sms, int cap1, int cap2) {
   auto clampi = [](int v, int lo, int hi) { return std::max(lo, std::min(v, hi)); };
-  const int minb = M <= 64 ? 2 : 1;
+  const int minb = bnp <= 64 ? 2 : 1;
   const int cap = minb == 1 ? cap1 : cap2;
   const int target = (minb == 2 ? 256 : 128) * sms / 148;
-  const int splits = clampi(target / n_tiles, 1, std::min(std::min(8, cap), std::max(1, KB / 2)));
+  const int splits =
+      clampi(target / (n_tiles * m_tiles), 1, std::min(std::min(8, cap), std::max(1, KB / 2)));
   return {minb, splits};
 }
 
@@ -743,13 +744,14 @@ bool decode_layout(int M, int splits, int kg, dg::DecodeArgs* a, int* smem_bytes
 // Lowers `splits` until every cluster of the launch (with its shared-memory
 // layout) is resident at once.
 template <int BNP, int MINB>
-int fit_splits(int dev, int M, int n_tiles, int splits) {
+int fit_splits(int dev, int M, int clusters, int splits) {
   for (; splits > 1; --splits) {
     dg::DecodeArgs a;
     int smem = 0;
     bool fits = false;
-    for (int kg = 4; kg >= 1 && !fits; kg /= 2) fits = decode_layout<BNP, MINB>(M, splits, kg, &a, &smem);
-    if (fits && decode_cluster_capacity<BNP, MINB>(dev, splits, smem) >= n_tiles) break;
+    for (int kg = 4; kg >= 1 && !fits; kg /= 2)
+      fits = decode_layout<BNP, MINB>(std::min(M, BNP), splits, kg, &a, &smem);
+    if (fits && decode_cluster_capacity<BNP, MINB>(dev, splits, smem) >= clusters) break;
   }
   return splits;
 }
@@ -760,7 +762,9 @@ dg_status run_decode(const void* A, const float* sfa, const void* B, const float
   using Cfg = dg::DecodeCfg<BNP, MINB>;
   const int KB = K / 128;
   const int n_tiles = (N + 127) / 128;
+  const int m_tiles = (M + BNP - 1) / BNP;
   const int ld = (M + 3) / 4 * 4;
+  const int Mt = std::min(M, BNP);  // tokens of the largest token tile
   dg::DecodeArgs args;
   std::memset(&args, 0, sizeof args);
   int smem = 0;
@@ -773,9 +777,9 @@ dg_status run_decode(const void* A, const float* sfa, const void* B, const float
   }
   bool fits = false;
   if (kg) {
-    fits = decode_layout<BNP, MINB>(M, splits, kg, &args, &smem);
+    fits = decode_layout<BNP, MINB>(Mt, splits, kg, &args, &smem);
   } else {
-    for (kg = 4; kg >= 1 && !fits; kg /= 2) fits = decode_layout<BNP, MINB>(M, splits, kg, &args, &smem);
+    for (kg = 4; kg >= 1 && !fits; kg /= 2) fits = decode_layout<BNP, MINB>(Mt, splits, kg, &args, &smem);
   }
   if (!fits) return DG_ERR_UNSUPPORTED_SHAPE;
   CUtensorMap tw, twpf, tx, tsa;
@@ -807,9 +811,10 @@ dg_status run_decode(const void* A, const float* sfa, const void* B, const float
   if (print_configs())
     std::fprintf(stderr,
                  "[dg] fp8_gemm_nt decode M=%d N=%d K=%d: swap-AB BNP=%d (%d CTA/SM), n_tiles=%d x "
-                 "split-K %d (cluster), %d CTAs, %d stages x %d K-blocks, %d B smem\n",
-                 M, N, K, BNP, MINB, n_tiles, splits, n_tiles * splits, args.stages, args.kg, smem);
-  cudaError_t e = launch(dg::gemm_decode_kernel<BNP, MINB>, dim3(splits, n_tiles, 1), dim3(320),
+                 "token tiles %d x split-K %d (cluster), %d CTAs, %d stages x %d K-blocks, %d B smem\n",
+                 M, N, K, BNP, MINB, n_tiles, m_tiles, splits, n_tiles * m_tiles * splits,
+                 args.stages, args.kg, smem);
+  cudaError_t e = launch(dg::gemm_decode_kernel<BNP, MINB>, dim3(splits, m_tiles, n_tiles), dim3(320),
                          static_cast<size_t>(smem), st, splits, tw, twpf, tx, tsa, args);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   g_launches.fetch_add(1);
@@ -821,7 +826,16 @@ dg_status dispatch_decode(const void* A, const float* sfa, const void* B, const 
                           cudaStream_t st) {
   const int KB = K / 128;
   const int n_tiles = (N + 127) / 128;
-  const int bnp = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  // token tile: up to 64 tokens in one tile of the half-SM configuration,
+  // 65..128 tokens in one 128-token tile on the whole SM. DG_DECODE_BNP=64
+  // cuts 65..128 tokens into two 64-token tiles instead (measured slower on
+  // B200: the second token tile re-reads every weight tile through L2); read
+  // on every call
+  int bnp = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  if (M > 64)
+    if (const char* e = std::getenv("DG_DECODE_BNP"))
+      if (std::atoi(e) == 64) bnp = 64;
+  const int m_tiles = (M + bnp - 1) / bnp;
   int cap1 = 0, cap2 = 0;  // co-schedulable cluster sizes of the two configurations
   switch (bnp) {
     case 16: cap1 = max_cluster<16, 1>(dev); cap2 = max_cluster<16, 2>(dev); break;
@@ -830,7 +844,7 @@ dg_status dispatch_decode(const void* A, const float* sfa, const void* B, const 
     default: cap1 = max_cluster<128, 1>(dev); break;
   }
   if (cap1 <= 0 || (bnp < 128 && cap2 <= 0)) return DG_ERR_CUDA;
-  DecodePlan p = plan_decode(M, n_tiles, KB, sms, cap1, cap2);
+  DecodePlan p = plan_decode(bnp, m_tiles, n_tiles, KB, sms, cap1, cap2);
   // DG_DECODE_MINB=1|2 and DG_DECODE_SPLITS=s force the plan (comparisons;
   // splits clamped to the cluster limit and to one K-block per split; 128
   // tokens always take the whole SM); read on every call
@@ -845,10 +859,14 @@ dg_status dispatch_decode(const void* A, const float* sfa, const void* B, const 
     const int f = std::atoi(e);
     if (f >= 1) p.splits = std::max(1, std::min(std::min(f, std::min(cap, 8)), KB));
   }
-  const bool forced = std::getenv("DG_DECODE_SPLITS") != nullptr;
+  // with one CTA per SM a cluster needs `splits` whole SMs of one GPC, and
+  // some sizes (e.g. 7) leave SMs of every GPC idle: lower the split count
+  // until all clusters are resident at once (two CTAs per SM pack freely)
+  const bool fit = std::getenv("DG_DECODE_SPLITS") == nullptr && p.minb == 1;
+  const int clusters = n_tiles * m_tiles;
 #define DG_RUN_DECODE(BNP_, MINB_)                                                         \
   return run_decode<BNP_, MINB_>(A, sfa, B, sfb, C, D, M, N, K,                            \
-                                 forced ? p.splits : fit_splits<BNP_, MINB_>(dev, M, n_tiles, p.splits), st)
+                                 fit ? fit_splits<BNP_, MINB_>(dev, M, clusters, p.splits) : p.splits, st)
   switch (bnp) {
     case 16:
       if (p.minb == 1) DG_RUN_DECODE(16, 1);

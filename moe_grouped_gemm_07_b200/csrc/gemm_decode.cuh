@@ -16,8 +16,11 @@
 //     ahead, 8 K-blocks per prefetch instruction) before anything else, so
 //     the slice's DRAM reads are all in flight while the CTA sets up and
 //     while the previous launch finishes; the TMA loads then mostly hit L2;
+//   * more than BNP tokens are cut into token tiles of BNP (a grid
+//     dimension); the tiles of one N-tile run side by side, so the weight
+//     tile comes from DRAM once;
 //   * the partial tiles are reduced by token rows: CTA r owns tokens
-//     [r R, r R + R), R = ceil(M / splits). Each CTA writes its FP32 partial
+//     [r R, r R + R) of its token tile, R = ceil(min(M, BNP) / splits). Each CTA writes its FP32 partial
 //     to its own shared memory token-major, then one thread bulk-copies the
 //     rows every other CTA owns into that CTA's receive slot for this rank
 //     (cp.async.bulk shared::cta -> shared::cluster), completing bytes on the
@@ -53,7 +56,7 @@ struct DecodeArgs {
   int splits;    // CTAs per cluster along K
   int stages;    // depth of the W/X ring (2..DecodeCfg::MAX_STAGES)
   int kg;        // K-blocks per ring stage (1, 2 or 4): one TMA box each for W and X
-  int rows_per_owner;  // R = ceil(M / splits): token rows reduced by each CTA
+  int rows_per_owner;  // R = ceil(min(M, BNP) / splits): token rows reduced by each CTA
   uint32_t off_x, off_sfa, off_recv, off_bar;  // shared-memory layout (bytes)
   const float* sfb;  // [ceil(N/128)][KB]
   const void* C;     // [M][N] bf16 or null
@@ -220,14 +223,20 @@ __global__ void __launch_bounds__(320, MINB)
   const int splits = args.splits;
   const int S = args.stages;
   const int KG = args.kg;
-  const int n_tile = blockIdx.y;
+  // grid (splits, token tiles, N-tiles): this CTA's tokens are
+  // [m0, m0 + Mloc) -- more than BNP tokens are cut into token tiles that
+  // share each weight tile (read from DRAM once, the second time from L2:
+  // the tiles of one N-tile are neighbours in launch order)
+  const int m0 = static_cast<int>(blockIdx.y) * BNP;
+  const int Mloc = min(BNP, args.M - m0);
+  const int n_tile = blockIdx.z;
   const int n0 = n_tile * 128;
   const int kb_begin = static_cast<int>((static_cast<long long>(rank) * args.KB) / splits);
   const int kb_end = static_cast<int>((static_cast<long long>(rank + 1) * args.KB) / splits);
   const int nkb = kb_end - kb_begin;
   const int R = args.rows_per_owner;
-  const int m_lo = min(args.M, static_cast<int>(rank) * R);
-  const int m_hi = min(args.M, m_lo + R);
+  const int m_lo = min(Mloc, static_cast<int>(rank) * R);
+  const int m_hi = min(Mloc, m_lo + R);
 
   if (warp == 0) {
     // The weight slice goes to L2 before anything else (an L2 prefetch reads
@@ -292,7 +301,7 @@ __global__ void __launch_bounds__(320, MINB)
         if (!__all_sync(0xffffffffu, ok)) break;
         if (lane == 0) mbar_arrive_expect_tx(&sfull[c], Cfg::SFA_CHUNK_BYTES);
         __syncwarp();
-        if (lane == 2) tma_load_2d(sSfa + c * (SCH * BNP), &tm_sfa, &sfull[c], 0, kb);
+        if (lane == 2) tma_load_2d(sSfa + c * (SCH * BNP), &tm_sfa, &sfull[c], m0, kb);
         ++nchunks;
       }
       bool ok = mbar_wait(&empty[s], ph ^ 1, abort_flag, tmo, SITE_PRODUCER_EMPTY);
@@ -307,7 +316,7 @@ __global__ void __launch_bounds__(320, MINB)
         if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(KG * Cfg::STAGE_BYTES));
         __syncwarp();
         if (lane == 0) tma_load_3d(sW + s * KG * Cfg::W_BYTES, &tm_w, &full[s], 0, n0, kb);
-        if (lane == 1) tma_load_3d(sX + s * KG * Cfg::X_BYTES, &tm_x, &full[s], 0, 0, kb);
+        if (lane == 1) tma_load_3d(sX + s * KG * Cfg::X_BYTES, &tm_x, &full[s], 0, m0, kb);
       }
       if (lane == 3) {
         const int lo = it + args.pf;
@@ -465,8 +474,8 @@ __global__ void __launch_bounds__(320, MINB)
     if (threadIdx.x == 0) {
       for (int o = 0; o < splits; ++o) {
         if (o == static_cast<int>(rank)) continue;
-        const int lo = min(args.M, o * R);
-        const int hi = min(args.M, lo + R);
+        const int lo = min(Mloc, o * R);
+        const int hi = min(Mloc, lo + R);
         if (hi <= lo) continue;
         const int slot = static_cast<int>(rank) < o ? static_cast<int>(rank) : static_cast<int>(rank) - 1;
         const uint32_t dst = dsmem_addr(smem_addr(recv + slot * R * 128), static_cast<uint32_t>(o));
@@ -503,7 +512,7 @@ __global__ void __launch_bounds__(320, MINB)
         v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
         v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
       }
-      const long long o = static_cast<long long>(m) * args.N + gn;
+      const long long o = static_cast<long long>(m0 + m) * args.N + gn;
       if (args.C) {
         const uint4 c4 = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(args.C) + o);
         v[0] += bf16_lo(c4.x); v[1] += bf16_hi(c4.x);
