@@ -330,8 +330,10 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
   s = make_map_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, rows_total, K, 128, 128,
                   CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DG_OK) return s;
+  // B in 128-row boxes: the kernel loads a BN-row tile as BN/128 boxes from
+  // separate producer lanes
   s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, static_cast<uint64_t>(G) * N, K, 128,
-                  bn, CU_TENSOR_MAP_SWIZZLE_128B);
+                  128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DG_OK) return s;
   // D as [rows_total][N] bf16; 32x32 boxes, 64-byte swizzle (TMA-store epilogue)
   CUtensorMap td;
@@ -415,7 +417,7 @@ dg_status run_layout(const void* A, const float* sfa, int ld_sfa, const void* B,
     s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, N, 128, 128,
                     CU_TENSOR_MAP_SWIZZLE_128B);
   else
-    s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, 128, 256,
+    s = make_map_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, 128, 128,
                     CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DG_OK) return s;
   s = make_map_2d(&td, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, 2ull * N, 32, 32,

@@ -468,8 +468,8 @@ __global__ void __launch_bounds__(320, 1)
           // One thread's TMA copies are processed one after another (about
           // 60 GB/s per thread with 16 KB boxes on B200); copies issued by
           // different lanes proceed side by side. So lane 0 arms the
-          // barrier, then lane 0 loads A and lane 1 (lanes 1..2 for an
-          // MN-major B) the B tile, in parallel.
+          // barrier, then lane 0 loads A and lanes 1..BN/128 the B tile's
+          // 128-row boxes, in parallel.
           if (args.drop_arrive && it == 0) {  // test hook: never arm stage 0
             dropped = 0;
           } else {
@@ -500,7 +500,12 @@ __global__ void __launch_bounds__(320, 1)
                               tl.b_row + h * 128, kk);
                 }
               } else {
-                if (lane == 1) tma_load_2d(sB + s * Cfg::B_BYTES, &tm_b, &full[s], kk, tl.b_row);
+                // B in 128-row boxes, one lane each (the map's box is 128 rows)
+                if (lane >= 1 && lane <= BN / 128) {
+                  const int h = static_cast<int>(lane) - 1;
+                  tma_load_2d(sB + s * Cfg::B_BYTES + h * 128 * Cfg::BK, &tm_b, &full[s], kk,
+                              tl.b_row + h * 128);
+                }
               }
             }
           }
