@@ -412,6 +412,59 @@ def run_grouped(args):
     return 0
 
 
+# ----------------------------------------------------------------- operand layouts
+def run_layouts(args):
+    """--workload layouts: the dense GEMM in its four operand layouts (NT, NN,
+    TN, TT) at M in {64, 128, 4096} on two weight shapes, GEMM launches back
+    to back over rotating weight copies (>= 3x L2) in a CUDA graph. NT routes
+    M <= 128 to the swap-AB decode kernel; NN / TN / TT run the persistent
+    kernel at every M. One GPU."""
+    import torch
+    import moe_grouped_gemm_07_b200 as dg
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops"]
+    fns = {"nt": dg.dg_fp8_gemm_nt, "nn": dg.dg_fp8_gemm_nn, "tn": dg.dg_fp8_gemm_tn,
+           "tt": dg.dg_fp8_gemm_tt}
+    rows = []
+    for (N, K) in ((7168, 16384), (4096, 7168)):
+        Bf = torch.from_numpy(synth.normal((N, K), synth.seed(2, nk_index(N, K), 1))).to(dev)
+        for layout in ("nt", "nn", "tn", "tt"):
+            b_mn = layout[1] == "n"
+            src = Bf.t().contiguous() if b_mn else Bf
+            qb, sb = dg.dg_quantize_fp8(src, dg.DG_QUANT_BLOCK_128x128)
+            del src
+            qbs = [qb] + [qb.clone() for _ in range(n_copies(N * K, 2) - 1)]
+            for M in (64, 128, 4096):
+                a_mn = layout[0] == "t"
+                Af = torch.from_numpy(synth.normal((M, K), synth.seed(2, shape_index(M, N, K), 0))).to(dev)
+                A = Af.t().contiguous() if a_mn else Af
+                qa, sa = dg.dg_quantize_fp8(
+                    A, dg.DG_QUANT_COL_128x1 if a_mn else dg.DG_QUANT_ROW_1x128)
+                Ds = [torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+                      for _ in range(min(len(qbs), n_copies(2 * M * N, 1)))]
+                reps = 16 if M <= 128 else 4
+                fn = fns[layout]
+                ms = time_batch(lambda j: fn(qa, sa, qbs[j % len(qbs)], sb, None,
+                                             Ds[j % len(Ds)]), reps, graph=True)
+                roof_ms = max(shape_flops(M, N, K) / (fp8_peak * 1e12),
+                              shape_bytes(M, N, K) / (pk["hbm_gbs"] * 1e9)) * 1e3
+                rows.append({"layout": layout, "M": M, "N": N, "K": K,
+                             "gemm_us": round(ms * 1e3, 2),
+                             "tflops": round(shape_flops(M, N, K) / (ms * 1e-3) / 1e12, 1),
+                             "gbs": round(shape_bytes(M, N, K) / (ms * 1e-3) / 1e9, 1),
+                             "roofline_frac": round(roof_ms / ms, 3)})
+                del Af, A, qa, sa, Ds
+            del qbs, qb, sb
+            torch.cuda.empty_cache()
+    print(json.dumps({"metric": METRIC, "workload": "dense_fp8_gemm_layouts",
+                      "timing": "GEMM launches back to back in a CUDA graph over rotating "
+                                "weight copies (>= 3x L2)", "shapes": rows}), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------- UE8M0 comparison
 def run_ue8m0(args):
     """--workload ue8m0: the dense sweep with power-of-two scales, timing the
@@ -890,7 +943,8 @@ def main():
     ap.add_argument("--quick", action="store_true",
                     help="timed device loop only: no e2e leg, CPU baseline or clock sampling")
     ap.add_argument("--workload", default="dense",
-                    choices=["dense", "contiguous", "masked", "kgrouped", "ue8m0", "fp8fp4"],
+                    choices=["dense", "contiguous", "masked", "kgrouped", "ue8m0", "fp8fp4",
+                             "layouts"],
                     help="dense (the bench line) or one MoE variant at its benchmark size")
     ap.add_argument("--masked-index", type=int, default=0,
                     help="masked workload: index into the (N, K) pairs")
@@ -901,6 +955,8 @@ def main():
         return run_reference(args)
     if args.workload == "fp8fp4":
         return run_fp8fp4(args)
+    if args.workload == "layouts":
+        return run_layouts(args)
     if args.workload == "ue8m0":
         return run_ue8m0(args)
     if args.workload != "dense":

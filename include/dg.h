@@ -341,6 +341,9 @@ uint64_t dg_get_launch_count(void);
  *   DG_DECODE_BNP=64     65..128 tokens as two 64-token tiles on half an SM
  *                        each instead of one 128-token tile (FP8 M <= 128
  *                        kernel); read on every call.
+ *   DG_DECODE_PAIR=0|1   128-token tiles of the FP8 M <= 128 kernel on tcgen05
+ *                        CTA pairs (two N-tiles, tokens split between the
+ *                        pair); read on every call.
  *   DG_DECODE_KG=1|2|4   K-blocks per ring stage (one TMA box each for weights
  *                        and tokens) of the FP8 M <= 128 kernel; read on every
  *                        call.

@@ -604,14 +604,15 @@ int cached_probe(std::mutex& mu, int (&best)[kMaxDevices], bool (&done)[kMaxDevi
   return best[dev];
 }
 
-template <int BNP, int MINB>
+template <int BNP, int MINB, bool PAIR = false>
 int max_cluster(int dev) {
   static std::mutex mu;
   static int best[kMaxDevices];
   static bool done[kMaxDevices];
   return cached_probe(mu, best, done, dev, [] {
-    return probe_max_cluster(reinterpret_cast<const void*>(dg::gemm_decode_kernel<BNP, MINB>),
-                             dg::DecodeCfg<BNP, MINB>::SMEM_BUDGET);
+    return probe_max_cluster(
+        reinterpret_cast<const void*>(dg::gemm_decode_kernel<BNP, MINB, PAIR>),
+        dg::DecodeCfg<BNP, MINB, PAIR>::SMEM_BUDGET);
   });
 }
 
@@ -656,28 +657,29 @@ int decode_prefetch_kblocks() {
 // configuration, s and smem; 0 on error). A cluster lives inside one GPC, so
 // e.g. clusters of 7 one-CTA-per-SM CTAs leave SMs of every GPC idle and
 // fewer of them fit than SMs / 7.
-template <int BNP, int MINB>
+template <int BNP, int MINB, bool PAIR = false>
 int decode_cluster_capacity(int dev, int s, int smem) {
   static std::mutex mu;
   static std::map<std::tuple<int, int, int>, int> cache;
   std::lock_guard<std::mutex> lock(mu);
   if (s < 1 || s > 8) return 0;
   const auto key = std::make_tuple(dev, s, smem);
+  const int cs = PAIR ? 2 * s : s;  // CTAs per cluster
   auto f = cache.find(key);
   if (f != cache.end()) return f->second;
   if (!no_pending_error()) return 0;
   int cap = 0;
-  const void* kern = reinterpret_cast<const void*>(dg::gemm_decode_kernel<BNP, MINB>);
+  const void* kern = reinterpret_cast<const void*>(dg::gemm_decode_kernel<BNP, MINB, PAIR>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           dg::DecodeCfg<BNP, MINB>::SMEM_BUDGET) == cudaSuccess) {
-    if (s > 1) {
+                           dg::DecodeCfg<BNP, MINB, PAIR>::SMEM_BUDGET) == cudaSuccess) {
+    if (cs > 1) {
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(s, 1, 1);
+      cfg.gridDim = dim3(cs, 1, 1);
       cfg.blockDim = dim3(320, 1, 1);
       cfg.dynamicSmemBytes = static_cast<size_t>(smem);
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = s;
+      attr[0].val.clusterDim.x = cs;
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
       cfg.attrs = attr;
@@ -721,9 +723,9 @@ DecodePlan plan_mx_decode(int M, int n_tiles, int KB, int sms, int cap1, int cap
 // Shared-memory layout of one decode launch: the deepest W/X ring (2..8
 // stages) that fits beside the sfa chunk slots, the split-K receive slots and
 // the barriers in the configuration's share of the SM. False if it does not fit.
-template <int BNP, int MINB>
+template <int BNP, int MINB, bool PAIR = false>
 bool decode_layout(int M, int splits, int kg, dg::DecodeArgs* a, int* smem_bytes) {
-  using Cfg = dg::DecodeCfg<BNP, MINB>;
+  using Cfg = dg::DecodeCfg<BNP, MINB, PAIR>;
   const int R = (M + splits - 1) / splits;
   const int recv = splits > 1 ? (splits - 1) * R * 512 : 0;
   const int sfa = 2 * Cfg::SFA_CHUNK_BYTES;
@@ -745,23 +747,23 @@ bool decode_layout(int M, int splits, int kg, dg::DecodeArgs* a, int* smem_bytes
 
 // Lowers `splits` until every cluster of the launch (with its shared-memory
 // layout) is resident at once.
-template <int BNP, int MINB>
+template <int BNP, int MINB, bool PAIR = false>
 int fit_splits(int dev, int M, int clusters, int splits) {
   for (; splits > 1; --splits) {
     dg::DecodeArgs a;
     int smem = 0;
     bool fits = false;
     for (int kg = 4; kg >= 1 && !fits; kg /= 2)
-      fits = decode_layout<BNP, MINB>(std::min(M, BNP), splits, kg, &a, &smem);
-    if (fits && decode_cluster_capacity<BNP, MINB>(dev, splits, smem) >= clusters) break;
+      fits = decode_layout<BNP, MINB, PAIR>(std::min(M, BNP), splits, kg, &a, &smem);
+    if (fits && decode_cluster_capacity<BNP, MINB, PAIR>(dev, splits, smem) >= clusters) break;
   }
   return splits;
 }
 
-template <int BNP, int MINB>
+template <int BNP, int MINB, bool PAIR = false>
 dg_status run_decode(const void* A, const float* sfa, const void* B, const float* sfb,
                      const void* C, void* D, int M, int N, int K, int splits, cudaStream_t st) {
-  using Cfg = dg::DecodeCfg<BNP, MINB>;
+  using Cfg = dg::DecodeCfg<BNP, MINB, PAIR>;
   const int KB = K / 128;
   const int n_tiles = (N + 127) / 128;
   const int m_tiles = (M + BNP - 1) / BNP;
@@ -779,9 +781,10 @@ dg_status run_decode(const void* A, const float* sfa, const void* B, const float
   }
   bool fits = false;
   if (kg) {
-    fits = decode_layout<BNP, MINB>(Mt, splits, kg, &args, &smem);
+    fits = decode_layout<BNP, MINB, PAIR>(Mt, splits, kg, &args, &smem);
   } else {
-    for (kg = 4; kg >= 1 && !fits; kg /= 2) fits = decode_layout<BNP, MINB>(Mt, splits, kg, &args, &smem);
+    for (kg = 4; kg >= 1 && !fits; kg /= 2)
+      fits = decode_layout<BNP, MINB, PAIR>(Mt, splits, kg, &args, &smem);
   }
   if (!fits) return DG_ERR_UNSUPPORTED_SHAPE;
   CUtensorMap tw, twpf, tx, tsa;
@@ -793,8 +796,10 @@ dg_status run_decode(const void* A, const float* sfa, const void* B, const float
   if ((s = make_map_3d(&twpf, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, N, KB, K, 128, 128, 128,
                        Cfg::PF_BOX)) != DG_OK)
     return s;
-  if ((s = make_map_3d(&tx, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, M, KB, K, 128, 128, BNP,
-                       static_cast<uint32_t>(args.kg), CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+  // tokens: BNP rows per box, or the half a CTA of a pair holds
+  if ((s = make_map_3d(&tx, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, M, KB, K, 128, 128,
+                       PAIR ? BNP / 2 : BNP, static_cast<uint32_t>(args.kg),
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
     return s;
   if ((s = make_map_2d(&tsa, sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ld, KB, 4ull * ld, BNP,
                        Cfg::SCH, CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
@@ -812,12 +817,15 @@ dg_status run_decode(const void* A, const float* sfa, const void* B, const float
   args.pf = decode_prefetch_kblocks();
   if (print_configs())
     std::fprintf(stderr,
-                 "[dg] fp8_gemm_nt decode M=%d N=%d K=%d: swap-AB BNP=%d (%d CTA/SM), n_tiles=%d x "
+                 "[dg] fp8_gemm_nt decode M=%d N=%d K=%d: swap-AB BNP=%d (%d CTA/SM)%s, n_tiles=%d x "
                  "token tiles %d x split-K %d (cluster), %d CTAs, %d stages x %d K-blocks, %d B smem\n",
-                 M, N, K, BNP, MINB, n_tiles, m_tiles, splits, n_tiles * m_tiles * splits,
-                 args.stages, args.kg, smem);
-  cudaError_t e = launch(dg::gemm_decode_kernel<BNP, MINB>, dim3(splits, m_tiles, n_tiles), dim3(320),
-                         static_cast<size_t>(smem), st, splits, tw, twpf, tx, tsa, args);
+                 M, N, K, BNP, MINB, PAIR ? " CTA pairs" : "", n_tiles, m_tiles, splits,
+                 (PAIR ? (n_tiles + 1) / 2 * 2 : n_tiles) * m_tiles * splits, args.stages, args.kg,
+                 smem);
+  const int cs = PAIR ? 2 * splits : splits;
+  cudaError_t e = launch(dg::gemm_decode_kernel<BNP, MINB, PAIR>,
+                         dim3(cs, m_tiles, PAIR ? (n_tiles + 1) / 2 : n_tiles), dim3(320),
+                         static_cast<size_t>(smem), st, cs, tw, twpf, tx, tsa, args);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   g_launches.fetch_add(1);
   return DG_OK;
@@ -846,6 +854,15 @@ dg_status dispatch_decode(const void* A, const float* sfa, const void* B, const 
     default: cap1 = max_cluster<128, 1>(dev); break;
   }
   if (cap1 <= 0 || (bnp < 128 && cap2 <= 0)) return DG_ERR_CUDA;
+  // 128-token tiles on CTA pairs (DG_DECODE_PAIR=0|1; read on every call)
+  bool pair = false;
+  if (bnp == 128)
+    if (const char* e = std::getenv("DG_DECODE_PAIR")) pair = std::atoi(e) != 0;
+  if (pair) {
+    const int pc = max_cluster<128, 1, true>(dev);
+    if (pc < 2) return DG_ERR_CUDA;
+    cap1 = pc / 2;  // split count of a cluster of pairs
+  }
   DecodePlan p = plan_decode(bnp, m_tiles, n_tiles, KB, sms, cap1, cap2);
   // DG_DECODE_MINB=1|2 and DG_DECODE_SPLITS=s force the plan (comparisons;
   // splits clamped to the cluster limit and to one K-block per split; 128
@@ -865,7 +882,12 @@ dg_status dispatch_decode(const void* A, const float* sfa, const void* B, const 
   // some sizes (e.g. 7) leave SMs of every GPC idle: lower the split count
   // until all clusters are resident at once (two CTAs per SM pack freely)
   const bool fit = std::getenv("DG_DECODE_SPLITS") == nullptr && p.minb == 1;
-  const int clusters = n_tiles * m_tiles;
+  const int clusters = (pair ? (n_tiles + 1) / 2 : n_tiles) * m_tiles;
+  if (pair)
+    return run_decode<128, 1, true>(A, sfa, B, sfb, C, D, M, N, K,
+                                    fit ? fit_splits<128, 1, true>(dev, M, clusters, p.splits)
+                                        : p.splits,
+                                    st);
 #define DG_RUN_DECODE(BNP_, MINB_)                                                         \
   return run_decode<BNP_, MINB_>(A, sfa, B, sfb, C, D, M, N, K,                            \
                                  fit ? fit_splits<BNP_, MINB_>(dev, M, clusters, p.splits) : p.splits, st)

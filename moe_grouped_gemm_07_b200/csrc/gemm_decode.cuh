@@ -76,13 +76,20 @@ struct DecodeArgs {
 // host per launch (decode_layout in the launcher): ring [stages][kg] W tiles
 // then [stages][kg] X tiles, the two sfa chunk slots, the receive slots
 // ((splits - 1) x R token rows of 128 floats), then the barriers.
-template <int BNP_, int MINB_>
+// PAIR: two CTAs of the cluster (ranks 2i, 2i + 1) form a tcgen05 CTA pair
+// over two neighbouring N-tiles: one M = 256 MMA, issued by the even rank,
+// whose token operand is split between the two CTAs (each loads BNP / 2
+// token rows) while each keeps its own 128 weight rows and its own 128 x BNP
+// accumulator. A CTA then moves 16 KB of weights + BNP / 2 x 128 bytes of
+// tokens per K-block instead of 16 KB + BNP x 128.
+template <int BNP_, int MINB_, bool PAIR_ = false>
 struct DecodeCfg {
   static constexpr int BNP = BNP_;              // token columns (MMA N)
   static constexpr int MINB = MINB_;
+  static constexpr bool PAIR = PAIR_;
   static constexpr int BK = 128;
   static constexpr int W_BYTES = 128 * BK;      // weight tile (MMA A operand)
-  static constexpr int X_BYTES = BNP * BK;      // token tile (MMA B operand)
+  static constexpr int X_BYTES = (PAIR ? BNP / 2 : BNP) * BK;  // this CTA's token rows (MMA B)
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
   static constexpr int MAX_STAGES = 8;
   static constexpr int SCH = 16;                // K-blocks per sfa chunk
@@ -106,6 +113,7 @@ struct DecodeCfg {
                 "TMEM allocation is a power of two >= 32 columns");
   static_assert(BNP == 16 || BNP == 32 || BNP == 64 || BNP == 128, "BNP");
   static_assert(X_BYTES % 1024 == 0, "SW128 tiles are 1024-byte aligned");
+  static_assert(!PAIR || (BNP == 128 && MINB == 1), "CTA pairs: 128-token tiles, one CTA per SM");
 };
 
 // Split-K reduction of a cluster's partial 128 x BNP tiles (swap-AB decode
@@ -183,14 +191,14 @@ __device__ __forceinline__ void splitk_reduce_store(const float (&acc)[EC], floa
   }
 }
 
-template <int BNP, int MINB>
+template <int BNP, int MINB, bool PAIR = false>
 __global__ void __launch_bounds__(320, MINB)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tm_w,    // B as [KB][N][128], kg-deep boxes
                        const __grid_constant__ CUtensorMap tm_wpf,  // B as [KB][N][128], L2 prefetch
                        const __grid_constant__ CUtensorMap tm_x,    // A as [KB][M][128], kg-deep boxes
                        const __grid_constant__ CUtensorMap tm_sfa,  // sfa: [KB][ld] f32, 16-row boxes
                        const __grid_constant__ DecodeArgs args) {
-  using Cfg = DecodeCfg<BNP, MINB>;
+  using Cfg = DecodeCfg<BNP, MINB, PAIR>;
   constexpr int NA = Cfg::NACC;
   constexpr int EC = Cfg::EC;
   constexpr int CH = Cfg::CH;
@@ -219,7 +227,13 @@ __global__ void __launch_bounds__(320, MINB)
   const uint32_t warp = warp_id_uniform();
   const uint32_t lane = lane_id();
   const uint64_t tmo = args.timeout_ns;
-  const uint32_t rank = cluster_ctarank();
+  // cluster = splits CTAs (x 2 with CTA pairs): `rank` is this CTA's part of
+  // the K range; with pairs, `pc` its place in the pair (0 issues the MMAs)
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t pc = PAIR ? (crank & 1u) : 0u;
+  const uint32_t rank = PAIR ? (crank >> 1) : crank;
+  const uint32_t leader_rank = crank & ~1u;
+  const bool leader = !PAIR || pc == 0;
   const int splits = args.splits;
   const int S = args.stages;
   const int KG = args.kg;
@@ -229,8 +243,9 @@ __global__ void __launch_bounds__(320, MINB)
   // the tiles of one N-tile are neighbours in launch order)
   const int m0 = static_cast<int>(blockIdx.y) * BNP;
   const int Mloc = min(BNP, args.M - m0);
-  const int n_tile = blockIdx.z;
-  const int n0 = n_tile * 128;
+  const int n_tile = PAIR ? static_cast<int>(blockIdx.z) * 2 + static_cast<int>(pc)
+                          : static_cast<int>(blockIdx.z);
+  const int n0 = n_tile * 128;  // with pairs and an odd tile count, may lie past N
   const int kb_begin = static_cast<int>((static_cast<long long>(rank) * args.KB) / splits);
   const int kb_end = static_cast<int>((static_cast<long long>(rank + 1) * args.KB) / splits);
   const int nkb = kb_end - kb_begin;
@@ -246,9 +261,9 @@ __global__ void __launch_bounds__(320, MINB)
       tma_prefetch_l2_3d(&tm_wpf, 0, n0, kb_begin + j);
     // lane i initialises barrier i (tempty / sempty count the 8 promotion warps)
     for (int i = static_cast<int>(lane); i < Cfg::NUM_BARS; i += 32) {
-      const bool by_warps = (i >= 2 * MS + NA && i < 2 * MS + 2 * NA) ||
-                            i == 2 * MS + 2 * NA + 2 || i == 2 * MS + 2 * NA + 3;
-      mbar_init(&bars[i], by_warps ? 8u : 1u);
+      const bool tmem_rel = i >= 2 * MS + NA && i < 2 * MS + 2 * NA;  // pairs: both CTAs' warps
+      const bool by_warps = tmem_rel || i == 2 * MS + 2 * NA + 2 || i == 2 * MS + 2 * NA + 3;
+      mbar_init(&bars[i], tmem_rel && PAIR ? 16u : by_warps ? 8u : 1u);
     }
     fence_mbarrier_init();
     __syncwarp();
@@ -261,12 +276,24 @@ __global__ void __launch_bounds__(320, MINB)
       tma_prefetch_desc(&tm_sfa);
     }
   } else if (warp == 1) {
-    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
-  if (splits > 1) cluster_arrive_relaxed();  // matched by cluster_wait() before the copies
+  // pairs: the partner's copies and TMEM releases signal the even CTA's
+  // barriers from the first K-block on, so the whole cluster syncs here;
+  // otherwise a split arrive here, matched by cluster_wait() before the
+  // split-K copies
+  if (!PAIR && splits > 1) cluster_arrive_relaxed();
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // The next launch on the stream may start (its prologue and weight
@@ -312,6 +339,16 @@ __global__ void __launch_bounds__(320, MINB)
       // lane 3 keeps the L2 prefetch window `pf` K-blocks ahead.
       if (args.drop_arrive && i == 0) {
         dropped = true;  // test hook: never arm stage 0
+      } else if constexpr (PAIR) {
+        // both CTAs' copies complete on the even CTA's barrier, armed there
+        if (lane == 0 && leader)
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(2 * KG * Cfg::STAGE_BYTES));
+        __syncwarp();
+        const uint32_t fb = dsmem_addr(smem_addr(&full[s]), leader_rank);
+        if (lane == 0) tma_load_3d_pair(sW + s * KG * Cfg::W_BYTES, &tm_w, fb, 0, n0, kb);
+        if (lane == 1)
+          tma_load_3d_pair(sX + s * KG * Cfg::X_BYTES, &tm_x, fb, 0,
+                           m0 + static_cast<int>(pc) * (BNP / 2), kb);
       } else {
         if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(KG * Cfg::STAGE_BYTES));
         __syncwarp();
@@ -335,7 +372,9 @@ __global__ void __launch_bounds__(320, MINB)
     // slot was reloaded)
     {
       volatile int never = 0;
-      for (int j = (i > S ? i - S : 0); j < i; ++j) {
+      // (pairs: the even CTA's barriers count both CTAs' copies; the odd
+      // CTA leaves only after the closing cluster barrier)
+      for (int j = (i > S ? i - S : 0); j < i && leader; ++j) {
         if (dropped && j == 0) continue;
         mbar_wait(&full[j % S], (j / S) & 1, &never, tmo, SITE_TEARDOWN_TMA);
       }
@@ -343,9 +382,10 @@ __global__ void __launch_bounds__(320, MINB)
         mbar_wait(&sfull[ci & 1], (ci >> 1) & 1, &never, tmo, SITE_TEARDOWN_TMA);
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 1 && leader) {
     // ======================= MMA issuer (converged warp, lane 0 issues) =====
-    constexpr uint32_t idesc = idesc_e4m3_f32(128, BNP, 0, 0);
+    constexpr uint32_t idesc = idesc_e4m3_f32(PAIR ? 256 : 128, BNP, 0, 0);
+    const uint16_t pair_mask = static_cast<uint16_t>(3u << leader_rank);
     const int nst = (nkb + KG - 1) / KG;
     int s = 0;
     uint32_t ph = 0;
@@ -362,35 +402,54 @@ __global__ void __launch_bounds__(320, MINB)
           const uint32_t w_base = smem_addr(sW + (s * KG + j) * Cfg::W_BYTES);
           const uint32_t x_base = smem_addr(sX + (s * KG + j) * Cfg::X_BYTES);
 #pragma unroll
-          for (int k = 0; k < Cfg::BK / 32; ++k)
-            mma_f8f6f4(tmem_base + b * BNP, smem_desc_sw128(w_base + k * 32, 16, 1024),
-                       smem_desc_sw128(x_base + k * 32, 16, 1024), idesc, k > 0 ? 1u : 0u);
-          mma_commit(&tfull[b]);
+          for (int k = 0; k < Cfg::BK / 32; ++k) {
+            const uint64_t dw = smem_desc_sw128(w_base + k * 32, 16, 1024);
+            const uint64_t dx = smem_desc_sw128(x_base + k * 32, 16, 1024);
+            if constexpr (PAIR)
+              mma_f8f6f4_pair(tmem_base + b * BNP, dw, dx, idesc, k > 0 ? 1u : 0u);
+            else
+              mma_f8f6f4(tmem_base + b * BNP, dw, dx, idesc, k > 0 ? 1u : 0u);
+          }
+          if constexpr (PAIR)
+            mma_commit_pair_mc(&tfull[b], pair_mask);  // both accumulators are ready
+          else
+            mma_commit(&tfull[b]);
         }
         __syncwarp();
       }
       if (!ok) break;
-      if (lane == 0) mma_commit(&empty[s]);
+      if (lane == 0) {
+        if constexpr (PAIR)
+          mma_commit_pair_mc(&empty[s], pair_mask);  // frees the stage in both CTAs
+        else
+          mma_commit(&empty[s]);
+      }
       __syncwarp();
       if (++s == S) {
         s = 0;
         ph ^= 1;
       }
     }
-    if (lane == 0) mma_commit(mma_done);
+    if (lane == 0) {
+      if constexpr (PAIR)
+        mma_commit_pair_mc(mma_done, static_cast<uint16_t>(1u << crank));
+      else
+        mma_commit(mma_done);
+    }
     __syncwarp();
     volatile int never = 0;
     mbar_wait(mma_done, 0, &never, tmo, SITE_TEARDOWN_MMA);
     __syncwarp();
-  } else {
+  } else if (warp >= 2) {
     // ======================= promotion (8 warps) =======================
     const uint32_t t_lane = tmem_base + ((q * 32) << 16);
     const float* pb = args.sfb + static_cast<long long>(n_tile) * args.KB + kb_begin;
+    const bool n_in = n0 < args.N;  // a pair's odd CTA past the last N-tile reads no sfb
     // sfb prefetch ring of 4 K-blocks, loop unrolled by 4 (slot u refilled in place)
     float sbr[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-      if (u < nkb) sbr[u] = __ldg(pb + u);
+      if (u < nkb && n_in) sbr[u] = __ldg(pb + u);
     for (int it0 = 0; it0 < nkb; it0 += 4) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -409,7 +468,7 @@ __global__ void __launch_bounds__(320, MINB)
         }
         tc_fence_after();
         const float sb = sbr[u];
-        if (it + 4 < nkb) sbr[u] = __ldg(pb + it + 4);
+        if (it + 4 < nkb && n_in) sbr[u] = __ldg(pb + it + 4);
         const float* sa = sSfa + c * (SCH * BNP) + (it % SCH) * BNP + h * EC;
         auto fma_chunk = [&](int cc, const uint32_t (&r)[CH]) {
 #pragma unroll
@@ -427,7 +486,12 @@ __global__ void __launch_bounds__(320, MINB)
         auto release_tmem = [&]() {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[b]);
+          if (lane == 0) {
+            if constexpr (PAIR)
+              mbar_arrive_cluster(dsmem_addr(smem_addr(&tempty[b]), leader_rank));
+            else
+              mbar_arrive(&tempty[b]);
+          }
         };
         if constexpr (Cfg::ALL_IN_FLIGHT) {
           uint32_t r[EC / CH][CH];
@@ -470,7 +534,7 @@ __global__ void __launch_bounds__(320, MINB)
   }
   __syncthreads();
   if (splits > 1) {
-    cluster_wait();  // every owner's receive barrier is initialised
+    if (!PAIR) cluster_wait();  // every owner's receive barrier is initialised
     if (threadIdx.x == 0) {
       for (int o = 0; o < splits; ++o) {
         if (o == static_cast<int>(rank)) continue;
@@ -478,8 +542,10 @@ __global__ void __launch_bounds__(320, MINB)
         const int hi = min(Mloc, lo + R);
         if (hi <= lo) continue;
         const int slot = static_cast<int>(rank) < o ? static_cast<int>(rank) : static_cast<int>(rank) - 1;
-        const uint32_t dst = dsmem_addr(smem_addr(recv + slot * R * 128), static_cast<uint32_t>(o));
-        const uint32_t mb = dsmem_addr(smem_addr(rbar), static_cast<uint32_t>(o));
+        // the owner is the CTA at the same place in its pair
+        const uint32_t orank = PAIR ? static_cast<uint32_t>(2 * o) + pc : static_cast<uint32_t>(o);
+        const uint32_t dst = dsmem_addr(smem_addr(recv + slot * R * 128), orank);
+        const uint32_t mb = dsmem_addr(smem_addr(rbar), orank);
         bulk_copy_to_cluster(dst, stage_out + lo * 128, static_cast<uint32_t>((hi - lo) * 512), mb);
       }
       bulk_commit();
@@ -531,7 +597,16 @@ __global__ void __launch_bounds__(320, MINB)
   // this CTA's partial must stay until the copies to its peers have read it
   if (splits > 1 && threadIdx.x == 0) bulk_wait_read0();
 
-  if (warp == 1) {
+  if constexpr (PAIR) {
+    // the even CTA's MMAs wrote this CTA's TMEM and read its shared memory:
+    // neither is released before the whole cluster is here
+    tc_fence_before();
+    cluster_sync_all();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+    }
+  } else if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }

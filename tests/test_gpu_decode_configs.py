@@ -1,9 +1,9 @@
 """Every configuration of the small-M (decode) kernel against the oracle.
 
 The planner picks CTAs per SM (1 or 2), a split count and the token tile
-(one tile of up to 128 tokens); DG_DECODE_MINB, DG_DECODE_SPLITS and
-DG_DECODE_BNP=64 (two 64-token tiles for 65..128 tokens) force them for
-every call. Each
+(one tile of up to 128 tokens); DG_DECODE_MINB, DG_DECODE_SPLITS,
+DG_DECODE_BNP=64 (two 64-token tiles for 65..128 tokens) and DG_DECODE_PAIR
+(128-token tiles on CTA pairs) force them for every call. Each
 case re-runs the decode parity tests in a child process with one forced plan
 (split counts that do not divide a tile's tokens evenly included) and checks
 the config log.
@@ -18,17 +18,20 @@ pytestmark = pytest.mark.gpu
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
-PLANS = [("1", None, None), ("2", None, None), ("1", "7", None), ("2", "3", None),
-         ("2", "8", None), ("2", None, "64"), ("1", "5", "64")]
+PLANS = [("1", None, None, None), ("2", None, None, None), ("1", "7", None, None),
+         ("2", "3", None, None), ("2", "8", None, None), ("2", None, "64", None),
+         ("1", "5", "64", None), ("1", None, None, "1"), ("1", "3", None, "1")]
 
 
-@pytest.mark.parametrize("minb,splits,bnp", PLANS)
-def test_decode_kernel_configs_parity(minb, splits, bnp):
+@pytest.mark.parametrize("minb,splits,bnp,pair", PLANS)
+def test_decode_kernel_configs_parity(minb, splits, bnp, pair):
     env = dict(os.environ, DG_DECODE_MINB=minb, DG_PRINT_CONFIGS="1")
     if splits:
         env["DG_DECODE_SPLITS"] = splits
     if bnp:
         env["DG_DECODE_BNP"] = bnp
+    if pair:
+        env["DG_DECODE_PAIR"] = pair
     cmd = [sys.executable, "-m", "pytest", "-x", "-q", "-s", "-m", "gpu", "-p", "no:cacheprovider",
            "tests/test_gpu_gemm.py", "tests/test_gpu_failure.py",
            "-k", "decode or graph or dropped_arrive"]
@@ -40,3 +43,5 @@ def test_decode_kernel_configs_parity(minb, splits, bnp):
         assert f"split-K {splits} " in out, "forced split count did not run:\n" + out[-2000:]
     if bnp:
         assert f"BNP={bnp} " in out, "forced token tile did not run:\n" + out[-2000:]
+    if pair:
+        assert "CTA pairs" in out, "CTA-pair configuration did not run:\n" + out[-2000:]
