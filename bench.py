@@ -15,8 +15,9 @@ Reported (one JSON line, rank 0):
   e2e          same metric through the public API with the activations copied
                from pinned host memory and D copied back inside the timed loop
   roofline     dominant kernel (the GEMM on its largest shape): achieved TFLOP/s
-               vs the measured-derived FP8 peak, from the kernel's average
-               launch duration over back-to-back launches; roofline_hbm: the
+               vs the measured-derived FP8 peak, from CUDA events around that
+               GEMM inside full steps (its back-to-back time alone beside it);
+               roofline_hbm: the
                same for the decode shapes (M <= 128) against HBM bandwidth,
                launches back to back over rotating weight copies (>= 3x L2),
                with the single-launch-after-a-flush figure beside it
@@ -466,13 +467,56 @@ def run_layouts(args):
 
 
 # ----------------------------------------------------------------- UE8M0 comparison
+def _sweep_inputs(dev, shapes, quant_w, quant_a):
+    """Seeded weights (quantised once, rotating copies of the codes spanning
+    at least three times the L2) and activations for a dense sweep."""
+    import torch
+    weights, acts, outs, qbufs = {}, [], [], []
+    for (N, K) in sorted(set((s_[1], s_[2]) for s_ in shapes)):
+        B = torch.from_numpy(synth.normal((N, K), synth.seed(2, nk_index(N, K), 1))).to(dev)
+        qb, sb, pb = quant_w(B)
+        del B
+        weights[(N, K)] = ([qb] + [qb.clone() for _ in range(n_copies(qb.numel(), 2) - 1)], sb, pb)
+    for (M, N, K) in shapes:
+        A = torch.from_numpy(synth.normal((M, K), synth.seed(2, shape_index(M, N, K), 0))).to(dev)
+        acts.append(A)
+        outs.append(torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+        qbufs.append(quant_a(A))
+    torch.cuda.synchronize()
+    return weights, acts, outs, qbufs
+
+
+def batch_reps(shape):
+    """Launches per timed CUDA-graph batch of one GEMM shape."""
+    return 32 if shape[0] <= 128 else 8
+
+
+def _time_steps(step, steps, warmup):
+    """Average ms of one step over `steps` steps issued back to back between
+    two CUDA events, after `warmup` untimed steps."""
+    import torch
+    for j in range(max(warmup, 3)):
+        step(j)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(200_000)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for j in range(steps):
+        step(j)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
 def run_ue8m0(args):
     """--workload ue8m0: the dense sweep with power-of-two scales, timing the
     two GEMM paths on the same quantised inputs: explicit promotion
     (dg_fp8_gemm_nt, FP32 copies of the scales) and the tensor core's
     block-scaled MMA (dg_fp8_gemm_nt_ue8m0, packed UE8M0). One step = per
-    shape, quantise A (power-of-two 1x128) + the block-scaled GEMM; L2 flushed
-    before every shape as in the main line. One GPU."""
+    shape, quantise A (power-of-two 1x128) + the block-scaled GEMM, steps
+    back to back as in the main line; each GEMM is also timed alone, launches
+    back to back in a CUDA graph over rotating weight copies. One GPU."""
     import torch
     import moe_grouped_gemm_07_b200 as dg
 
@@ -483,52 +527,31 @@ def run_ue8m0(args):
     shapes = wl.dense_shapes()
     if args.shape:
         shapes = [tuple(int(x) for x in sh.split(",")) for sh in args.shape.split(";") if sh]
-    weights, acts, outs, qbufs = {}, [], [], []
-    for (N, K) in sorted(set((s_[1], s_[2]) for s_ in shapes)):
-        B = torch.from_numpy(synth.normal((N, K), synth.seed(2, nk_index(N, K), 1))).to(dev)
-        weights[(N, K)] = dg.dg_quantize_fp8_ue8m0(B, dg.DG_QUANT_BLOCK_128x128)
-        del B
-    for (M, N, K) in shapes:
-        A = torch.from_numpy(synth.normal((M, K), synth.seed(2, shape_index(M, N, K), 0))).to(dev)
-        acts.append(A)
-        outs.append(torch.empty((M, N), dtype=torch.bfloat16, device=dev))
-        qbufs.append(dg.dg_quantize_fp8_ue8m0(A, dg.DG_QUANT_ROW_1x128))
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    torch.cuda.synchronize()
+    weights, acts, outs, qbufs = _sweep_inputs(
+        dev, shapes, lambda B: dg.dg_quantize_fp8_ue8m0(B, dg.DG_QUANT_BLOCK_128x128),
+        lambda A: dg.dg_quantize_fp8_ue8m0(A, dg.DG_QUANT_ROW_1x128))
     n = len(shapes)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
 
-    def run(kind, record):
-        for i, (M, N, K) in enumerate(shapes):
-            flush.fill_(i & 0xFF)
-            torch.cuda._sleep(100_000)
+    def gemm(kind, i, j):
+        M, N, K = shapes[i]
+        qa, sa, pa = qbufs[i]
+        qbs, sb, pb = weights[(N, K)]
+        qb = qbs[j % len(qbs)]
+        if kind == "mx":
+            dg.dg_fp8_gemm_nt_ue8m0(qa, pa, qb, pb, None, outs[i])
+        else:
+            dg.dg_fp8_gemm_nt(qa, sa, qb, sb, None, outs[i])
+
+    def step(j):
+        for i in range(n):
             qa, sa, pa = qbufs[i]
-            qb, sb, pb = weights[(N, K)]
-            if record:
-                ev[i][0].record()
-            if kind == "step":
-                dg.dg_quantize_fp8_ue8m0(acts[i], dg.DG_QUANT_ROW_1x128, codes=qa, scales=sa,
-                                         packed=pa)
-                dg.dg_fp8_gemm_nt_ue8m0(qa, pa, qb, pb, None, outs[i])
-            elif kind == "mx":
-                dg.dg_fp8_gemm_nt_ue8m0(qa, pa, qb, pb, None, outs[i])
-            else:
-                dg.dg_fp8_gemm_nt(qa, sa, qb, sb, None, outs[i])
-            if record:
-                ev[i][1].record()
+            dg.dg_quantize_fp8_ue8m0(acts[i], dg.DG_QUANT_ROW_1x128, codes=qa, scales=sa, packed=pa)
+            gemm("mx", i, j)
 
-    res = {}
-    for kind in ("step", "mx", "promotion"):
-        for _ in range(max(args.warmup, 3)):
-            run(kind, False)
-        torch.cuda.synchronize()
-        t = np.zeros(n)
-        for _ in range(args.steps):
-            run(kind, True)
-            torch.cuda.synchronize()
-            for i in range(n):
-                t[i] += ev[i][0].elapsed_time(ev[i][1])
-        res[kind] = t / args.steps
+    ms_step = _time_steps(step, args.steps, args.warmup)
+    res = {kind: np.array([time_batch(lambda j, i=i: gemm(kind, i, j), batch_reps(shapes[i]),
+                                      graph=True) for i in range(n)])
+           for kind in ("mx", "promotion")}
     flops = [shape_flops(*sh) for sh in shapes]
     big = max(range(n), key=lambda i: flops[i])
     per = [{"M": M, "N": N, "K": K, "mx_us": round(res["mx"][i] * 1e3, 2),
@@ -538,9 +561,11 @@ def run_ue8m0(args):
            for i, (M, N, K) in enumerate(shapes)]
     ach = flops[big] / (res["mx"][big] * 1e-3) / 1e12
     line = {"metric": METRIC, "workload": "dense_fp8_gemm_nt_sweep_ue8m0",
-            "value": round(sum(flops) / (res["step"].sum() * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "ms_per_step": round(float(res["step"].sum()), 4), "steps": args.steps,
+            "value": round(sum(flops) / (ms_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms_step, 4), "steps": args.steps,
             "higher_is_better": True, "dtype": "e4m3 x e4m3 (UE8M0 scales) -> f32 accumulate, bf16 out",
+            "timing": "step: K steps back to back; per shape: GEMM launches back to back in a "
+                      "CUDA graph over rotating weight copies (>= 3x L2)",
             "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
                          "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4),
                          "kernel": f"gemm_mx_kernel:{shapes[big][0]}x{shapes[big][1]}x{shapes[big][2]}"},
@@ -556,8 +581,9 @@ def run_fp8fp4(args):
     """--workload fp8fp4: the dense sweep with E2M1 (FP4) weights, one
     power-of-two scale per 1x32 K-strip, against E4M3 activations with
     power-of-two 1x128 scales, on the block-scaled MMA. One step = per shape,
-    quantise A + the FP8 x FP4 GEMM; the FP8 x FP8 block-scaled GEMM on the
-    same activations is timed beside it. L2 flushed before every shape. One GPU."""
+    quantise A + the FP8 x FP4 GEMM, steps back to back; each GEMM (and the
+    FP8 x FP8 block-scaled GEMM on the same activations) is also timed alone,
+    launches back to back in a CUDA graph over rotating weight copies. One GPU."""
     import torch
     import moe_grouped_gemm_07_b200 as dg
 
@@ -568,53 +594,39 @@ def run_fp8fp4(args):
     shapes = wl.dense_shapes()
     if args.shape:
         shapes = [tuple(int(x) for x in sh.split(",")) for sh in args.shape.split(";") if sh]
-    w4, w8, acts, outs, qbufs = {}, {}, [], [], []
-    for (N, K) in sorted(set((s_[1], s_[2]) for s_ in shapes)):
+    w4, acts, outs, qbufs = _sweep_inputs(
+        dev, shapes, lambda B: dg.dg_quantize_fp4_e2m1(B, with_scales=False),
+        lambda A: dg.dg_quantize_fp8_ue8m0(A, dg.DG_QUANT_ROW_1x128, with_scales=False))
+    w8 = {}
+    for (N, K) in w4:  # FP8 weights of the same matrices, for the comparison
         B = torch.from_numpy(synth.normal((N, K), synth.seed(2, nk_index(N, K), 1))).to(dev)
-        w4[(N, K)] = dg.dg_quantize_fp4_e2m1(B, with_scales=False)
-        w8[(N, K)] = dg.dg_quantize_fp8_ue8m0(B, dg.DG_QUANT_BLOCK_128x128, with_scales=False)
+        qb, sb, pb = dg.dg_quantize_fp8_ue8m0(B, dg.DG_QUANT_BLOCK_128x128, with_scales=False)
         del B
-    for (M, N, K) in shapes:
-        A = torch.from_numpy(synth.normal((M, K), synth.seed(2, shape_index(M, N, K), 0))).to(dev)
-        acts.append(A)
-        outs.append(torch.empty((M, N), dtype=torch.bfloat16, device=dev))
-        qbufs.append(dg.dg_quantize_fp8_ue8m0(A, dg.DG_QUANT_ROW_1x128, with_scales=False))
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        w8[(N, K)] = ([qb] + [qb.clone() for _ in range(n_copies(qb.numel(), 2) - 1)], sb, pb)
     torch.cuda.synchronize()
     n = len(shapes)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
 
-    def run(kind, record):
-        for i, (M, N, K) in enumerate(shapes):
-            flush.fill_(i & 0xFF)
-            torch.cuda._sleep(100_000)
+    def gemm(kind, i, j):
+        M, N, K = shapes[i]
+        qa, _, pa = qbufs[i]
+        qbs, _, pb = (w4 if kind == "fp4" else w8)[(N, K)]
+        qb = qbs[j % len(qbs)]
+        if kind == "fp4":
+            dg.dg_fp8_fp4_gemm_nt(qa, pa, qb, pb, None, outs[i])
+        else:
+            dg.dg_fp8_gemm_nt_ue8m0(qa, pa, qb, pb, None, outs[i])
+
+    def step(j):
+        for i in range(n):
             qa, _, pa = qbufs[i]
-            if record:
-                ev[i][0].record()
-            if kind == "step":
-                dg.dg_quantize_fp8_ue8m0(acts[i], dg.DG_QUANT_ROW_1x128, codes=qa, packed=pa,
-                                         with_scales=False)
-            if kind in ("step", "fp4"):
-                qb, _, pb = w4[(N, K)]
-                dg.dg_fp8_fp4_gemm_nt(qa, pa, qb, pb, None, outs[i])
-            else:
-                qb, _, pb = w8[(N, K)]
-                dg.dg_fp8_gemm_nt_ue8m0(qa, pa, qb, pb, None, outs[i])
-            if record:
-                ev[i][1].record()
+            dg.dg_quantize_fp8_ue8m0(acts[i], dg.DG_QUANT_ROW_1x128, codes=qa, packed=pa,
+                                     with_scales=False)
+            gemm("fp4", i, j)
 
-    res = {}
-    for kind in ("step", "fp4", "fp8"):
-        for _ in range(max(args.warmup, 3)):
-            run(kind, False)
-        torch.cuda.synchronize()
-        t = np.zeros(n)
-        for _ in range(args.steps):
-            run(kind, True)
-            torch.cuda.synchronize()
-            for i in range(n):
-                t[i] += ev[i][0].elapsed_time(ev[i][1])
-        res[kind] = t / args.steps
+    ms_step = _time_steps(step, args.steps, args.warmup)
+    res = {kind: np.array([time_batch(lambda j, i=i: gemm(kind, i, j), batch_reps(shapes[i]),
+                                      graph=True) for i in range(n)])
+           for kind in ("fp4", "fp8")}
     flops = [shape_flops(*sh) for sh in shapes]
     # algorithmic bytes with FP4 weights: A + B/2 + scales (A 1 per 128, B 1 per 32) + D
     nbytes = [M * K + N * K // 2 + M * (K // 128) + N * (K // 32) + 2 * M * N
@@ -628,10 +640,12 @@ def run_fp8fp4(args):
            for i, (M, N, K) in enumerate(shapes)]
     ach = flops[big] / (res["fp4"][big] * 1e-3) / 1e12
     line = {"metric": METRIC, "workload": "dense_fp8_fp4_gemm_nt_sweep",
-            "value": round(sum(flops) / (res["step"].sum() * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "ms_per_step": round(float(res["step"].sum()), 4), "steps": args.steps,
+            "value": round(sum(flops) / (ms_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms_step, 4), "steps": args.steps,
             "higher_is_better": True,
             "dtype": "e4m3 x e2m1 (UE8M0 scales, 1x128 / 1x32) -> f32 accumulate, bf16 out",
+            "timing": "step: K steps back to back; per shape: GEMM launches back to back in a "
+                      "CUDA graph over rotating weight copies (>= 3x L2)",
             "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
                          "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4),
                          "kernel": f"gemm_mx_kernel<FP4B>:{shapes[big][0]}x{shapes[big][1]}x{shapes[big][2]}",
@@ -772,7 +786,7 @@ def run_ours(args):
     for i, (M, N, K) in enumerate(shapes):
         qa, sa = qbufs[i]
         qbs, sb = weights[(N, K)]
-        reps = 32 if M <= 128 else 8
+        reps = batch_reps((M, N, K))
         t_g[i] = time_batch(lambda j: dg.dg_fp8_gemm_nt(qa, sa, qbs[j % len(qbs)], sb, None,
                                                         outs[i][j % len(outs[i])]), reps,
                             graph=True)
