@@ -93,8 +93,11 @@ dg_status dg_quantize_fp8(const void* x, int in_dtype, int batch, int rows, int 
  * Shapes: M >= 0, N >= 0 (either 0: no-op), K % 128 == 0 (K == 0: D = C),
  * N % 8 == 0.
  * M <= 128 (decode) runs a swap-AB kernel with split-K over a thread-block
- * cluster; its partial sums are added in a fixed order, so results repeat
- * bit for bit from run to run.
+ * cluster, or, for 65..128 rows where a cost model expects it to be faster,
+ * 128 x 256 tiles with each tile split along K over a cluster (both
+ * reductions add the partial sums in a fixed order, so results repeat bit
+ * for bit from run to run). The test hook dg_debug_drop_next_arrive does not
+ * apply to such split tiles.
  * ------------------------------------------------------------------------- */
 dg_status dg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb,
                          const void* C, void* D, int M, int N, int K, void* stream);
@@ -349,7 +352,10 @@ uint64_t dg_get_launch_count(void);
  *                        call.
  *   DG_DECODE_PF=k       weight K-blocks the FP8 M <= 128 kernel keeps
  *                        requested into L2 ahead of its loads (rounded up to
- *                        a multiple of 8, default 64); read on every call. */
+ *                        a multiple of 8, default 64); read on every call.
+ *   DG_SMALL_M_TILES=1   FP8 NT with M <= 128 on the 128 x 256 tile kernel,
+ *                        every tile split along K over a cluster, instead of
+ *                        the swap-AB decode kernel; read on every call. */
 
 #ifdef __cplusplus
 }

@@ -234,6 +234,15 @@ struct Bf16Raw {
 };
 
 // Shared NT launcher for dense / contiguous / masked.
+// M <= 128 on 128 x 256 tiles, each split along K over a cluster when the
+// tiles leave SMs idle, instead of the swap-AB decode kernel:
+// DG_SMALL_M_TILES=1 always, =0 never, unset: the cost model in
+// dispatch_decode decides for 65..128 tokens (read on every call).
+int small_m_tiles_env() {
+  const char* e = std::getenv("DG_SMALL_M_TILES");
+  return e ? (e[0] == '1' ? 1 : 0) : -1;
+}
+
 // Split-K tail of a dense launch (MODE_SPLITK): DG_TAIL_SPLIT=0 turns it off.
 bool tail_split_enabled() {
   static const bool on = [] {
@@ -299,6 +308,16 @@ int splitk_clusters(int dev, int k) {
   return cache[dev][k];
 }
 
+// One wave of 128 x 256 tiles (few rows): every tile split along K over a
+// cluster of k CTAs, k the largest power of two <= 8 whose clusters all fit
+// at once with at least 4 K-blocks per part.
+int whole_split_k(long long tiles, int KB, int sms, int dev) {
+  int k = 1;
+  while (k < 8 && tiles * (2 * k) <= sms && KB / (2 * k) >= 4 && splitk_clusters(dev, 2 * k) >= tiles)
+    k *= 2;
+  return k;
+}
+
 // NT scale ring: sfb viewed as [G * ceil(N/128)][K/128] FP32 with 4 x 2
 // boxes (four K-blocks of two 128-column blocks), when its rows are a
 // multiple of 16 bytes long (K/128 % 4 == 0); otherwise the kernel reads sfb
@@ -318,13 +337,14 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
                  const int32_t* m_indices, const int32_t* masked_m, const void* C, void* D,
                  int rows_total, int M_logical, int N, int K, int G, long long m_blocks_bound,
                  long long tiles_if_known, cudaStream_t st, const char* name,
-                 long long m_blocks_plan = -1) {
+                 long long m_blocks_plan = -1, bool whole_split = false) {
   int dev = 0, sms = 0;
   dg_status s = device_sms(&dev, &sms);
   if (s != DG_OK) return s;
   // the tile width is planned for the expected number of 128-row blocks
   // (masked: the caller's expected_m hint), the launch for the bound
-  const int bn = choose_bn(m_blocks_plan > 0 ? m_blocks_plan : m_blocks_bound, N, sms);
+  const int bn =
+      whole_split ? 256 : choose_bn(m_blocks_plan > 0 ? m_blocks_plan : m_blocks_bound, N, sms);
   CUtensorMap ta, tb, dummy;
   std::memset(&dummy, 0, sizeof dummy);
   s = make_map_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, rows_total, K, 128, 128,
@@ -371,6 +391,20 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
   // first launch takes the full waves. Both are ordered on the stream.
   int split = 1;
   const long long R = tiles > grid ? tiles % grid : 0;
+  if (MODE == dg::MODE_DENSE && bn == 256 && whole_split && tiles <= grid) {
+    const int k = whole_split_k(tiles, K / 128, sms, dev);
+    if (print_configs())
+      std::fprintf(stderr, "[dg] %s M=%d N=%d K=%d: BM=128 BN=256 tiles=%lld split %d\n", name,
+                   M_logical, N, K, tiles, k);
+    if (k > 1) {
+      args.split_tile0 = 0;
+      args.split = k;
+      args.drop_arrive = 0;
+      return launch_gemm<dg::MODE_SPLITK, 256>(ta, tb, dummy, tsb, td, args,
+                                               static_cast<int>(tiles) * k, st, dev, k);
+    }
+    return launch_gemm<MODE, 256>(ta, tb, dummy, tsb, td, args, static_cast<int>(tiles), st, dev);
+  }
   if (MODE == dg::MODE_DENSE && bn == 256 && tail_split_enabled()) {
     split = tail_split_for(tiles, grid, K / 128);
     if (split > 1 && splitk_clusters(dev, split) < R) split = 1;  // not all at once
@@ -883,6 +917,29 @@ dg_status dispatch_decode(const void* A, const float* sfa, const void* B, const 
   // until all clusters are resident at once (two CTAs per SM pack freely)
   const bool fit = std::getenv("DG_DECODE_SPLITS") == nullptr && p.minb == 1;
   const int clusters = (pair ? (n_tiles + 1) / 2 : n_tiles) * m_tiles;
+  // 65..128 tokens: the swap-AB kernel computes 128 weight rows per CTA and
+  // K-block, the 128 x 256 tile kernel 256 (its MMA's M side holds the
+  // tokens), at about the same per-K-block cadence; the tile kernel has the
+  // larger fixed cost, more so with a split-K exchange. Estimates in us,
+  // fitted to B200 timings of back-to-back launches of the decode shapes
+  // (within ~10%): decode 5.0 + 0.58 x waves x K-blocks per CTA; tiles, per
+  // wave, 8.5 + 0.58 x (K-blocks per part - 4) + 5.6 with a split. Forced
+  // decode plans keep the decode kernel.
+  if (bnp == 128 && !pair && small_m_tiles_env() != 0 && std::getenv("DG_DECODE_SPLITS") == nullptr &&
+      std::getenv("DG_DECODE_MINB") == nullptr) {
+    const int dsplits = fit ? fit_splits<128, 1>(dev, M, clusters, p.splits) : p.splits;
+    const long long dctas = static_cast<long long>(clusters) * dsplits;
+    const double t_dec =
+        5.0 + 0.58 * static_cast<double>((dctas + sms - 1) / sms) * ((KB + dsplits - 1) / dsplits);
+    const long long tiles = (N + 255) / 256;
+    const int k = tiles <= sms ? whole_split_k(tiles, KB, sms, dev) : 1;
+    const int kb_part = (KB + k - 1) / k;
+    const double t_tiles = static_cast<double>((tiles + sms - 1) / sms) *
+                           (8.5 + 0.58 * std::max(0, kb_part - 4) + (k > 1 ? 5.6 : 0.0));
+    if (t_tiles < t_dec)
+      return run_nt<dg::MODE_DENSE>(A, sfa, (M + 3) / 4 * 4, B, sfb, nullptr, nullptr, C, D, M, M,
+                                    N, K, 1, 1, 1, st, "fp8_gemm_nt", -1, true);
+  }
   if (pair)
     return run_decode<128, 1, true>(A, sfa, B, sfb, C, D, M, N, K,
                                     fit ? fit_splits<128, 1, true>(dev, M, clusters, p.splits)
@@ -1386,6 +1443,9 @@ dg_status dg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const f
   const int ld = (M + 3) / 4 * 4;
   const long long mb = (M + 127) / 128;
   if (M <= 128) {
+    if (small_m_tiles_env() == 1)
+      return run_nt<dg::MODE_DENSE>(A, sfa, ld, B, sfb, nullptr, nullptr, C, D, M, M, N, K, 1, mb,
+                                    mb, st, "fp8_gemm_nt", -1, true);
     int dev = 0, sms = 0;
     dg_status s = device_sms(&dev, &sms);
     if (s != DG_OK) return s;

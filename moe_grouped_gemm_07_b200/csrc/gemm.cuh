@@ -747,27 +747,33 @@ __global__ void __launch_bounds__(320, 1)
           const float* slot = sScale + ss * (Cfg::BM + BN);
           const float sav = slot[r_in_tile];
           const float* sbv = slot + Cfg::BM + h * EC;
-          constexpr int KC = 16;  // columns per TMEM load (fewer live registers)
+          // 16-column TMEM loads (fewer live registers), two buffers: the
+          // next chunk's load is in flight while this chunk is scaled
+          constexpr int KC = 16;
+          uint32_t r[2][KC];
+          tmem_ld_32x32b<KC>(t_lane + b * BN + h * EC, r[0]);
+          tmem_ld_wait_regs(r[0]);
 #pragma unroll
           for (int c = 0; c < EC / KC; ++c) {
-            uint32_t r[KC];
-            tmem_ld_32x32b<KC>(t_lane + b * BN + h * EC + c * KC, r);
-            tmem_ld_wait();
-            if (c == EC / KC - 1) {
+            if (c + 1 < EC / KC) {
+              tmem_ld_32x32b<KC>(t_lane + b * BN + h * EC + (c + 1) * KC, r[(c + 1) & 1]);
+            } else {  // every load of this buffer has completed
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&tempty[b]);
             }
+            const uint32_t(&rc)[KC] = r[c & 1];
 #pragma unroll
             for (int i = 0; i < KC; i += 4) {
               // acc += sav * (sb * P): the column-scaled products reuse P's registers
               const float4 sb4 = *reinterpret_cast<const float4*>(sbv + c * KC + i);
               float u0, u1, u2, u3;
-              mul2(u0, u1, sb4.x, sb4.y, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-              mul2(u2, u3, sb4.z, sb4.w, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+              mul2(u0, u1, sb4.x, sb4.y, __uint_as_float(rc[i]), __uint_as_float(rc[i + 1]));
+              mul2(u2, u3, sb4.z, sb4.w, __uint_as_float(rc[i + 2]), __uint_as_float(rc[i + 3]));
               fma2(acc[c * KC + i], acc[c * KC + i + 1], sav, sav, u0, u1);
               fma2(acc[c * KC + i + 2], acc[c * KC + i + 3], sav, sav, u2, u3);
             }
+            if (c + 1 < EC / KC) tmem_ld_wait_regs(r[(c + 1) & 1]);
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&sempty[ss]);

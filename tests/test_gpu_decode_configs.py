@@ -45,3 +45,19 @@ def test_decode_kernel_configs_parity(minb, splits, bnp, pair):
         assert f"BNP={bnp} " in out, "forced token tile did not run:\n" + out[-2000:]
     if pair:
         assert "CTA pairs" in out, "CTA-pair configuration did not run:\n" + out[-2000:]
+
+
+def test_small_m_plan_choice():
+    """65..128 tokens: the cost model sends 128x7168x16384 (28 tiles of 256
+    weight rows, 4-way split-K) to the tile kernel and 128x4096x7168 to the
+    swap-AB decode kernel; the log shows which ran."""
+    env = dict(os.environ, DG_PRINT_CONFIGS="1")
+    env.pop("DG_SMALL_M_TILES", None)
+    cmd = [sys.executable, "bench.py", "--shape", "128,7168,16384;128,4096,7168", "--steps", "1",
+           "--warmup", "1", "--quick", "--no-cpu-baseline", "--no-moe"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    out = r.stdout + r.stderr
+    assert r.returncode == 0, out[-4000:]
+    assert "M=128 N=7168 K=16384: BM=128 BN=256 tiles=28 split 4" in out, out[-2000:]
+    dec = [ln for ln in out.splitlines() if "M=128 N=4096 K=7168" in ln]
+    assert dec and all("CTA/SM" in ln for ln in dec), out[-2000:]

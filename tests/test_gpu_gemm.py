@@ -62,6 +62,9 @@ def test_dense_nt_vs_oracle(M, N, K, with_c):
 
 
 # M <= 128 runs the swap-AB split-K cluster kernel (token widths 16/32/64/128)
+# or, for 65..128 tokens where a cost model expects it to be faster, 128 x 256
+# tiles split along K over a cluster; DG_SMALL_M_TILES=0|1 forces either, and
+# every case runs on both
 DECODE_CASES = [
     (1, 256, 7168, False),
     (16, 2112, 7168, True),
@@ -78,8 +81,10 @@ DECODE_CASES = [
 ]
 
 
+@pytest.mark.parametrize("path", ["0", "1"])
 @pytest.mark.parametrize("M,N,K,with_c", DECODE_CASES)
-def test_dense_decode_path_vs_oracle(M, N, K, with_c):
+def test_dense_decode_path_vs_oracle(M, N, K, with_c, path, monkeypatch):
+    monkeypatch.setenv("DG_SMALL_M_TILES", path)
     w = wl.dense(M, N, K, cfg=88, shape=M + N + K, with_c=with_c)
     Cb = synth.to_bf16_bits(w.C) if with_c else None
     qa, sa, qb, sb = quant_nt_gpu(w.A, w.B)
