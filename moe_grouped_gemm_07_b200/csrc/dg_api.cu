@@ -479,10 +479,43 @@ dg_status run_layout(const void* A, const float* sfa, int ld_sfa, const void* B,
   CUtensorMap tsb = dummy;
   if (MODE == dg::MODE_TT) make_sfb_box_map(&tsb, sfb, N, K, 1, &args);  // B stored [N][K]
   const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(sms, tiles)));
+  // Split-K as for NT: with one wave of tiles (few rows) every tile is split
+  // along K over a cluster when that saves more K-blocks per CTA than the
+  // exchange costs (~10 K-blocks on B200); otherwise a partial last wave runs
+  // as a second, split launch.
+  constexpr int SPLIT_MODE = MODE == dg::MODE_NN   ? dg::MODE_SPLITK_NN
+                             : MODE == dg::MODE_TN ? dg::MODE_SPLITK_TN
+                                                   : dg::MODE_SPLITK_TT;
+  const int KB = K / 128;
+  int k = 1;
+  long long first = tiles;  // tiles of the unsplit launch
+  if (tail_split_enabled()) {
+    if (tiles <= grid) {
+      k = whole_split_k(tiles, KB, sms, dev);
+      if (KB - (KB + k - 1) / k < 10) k = 1;
+      if (k > 1) first = 0;
+    } else if (tiles % grid != 0) {
+      k = tail_split_for(tiles, grid, KB);
+      if (k > 1 && splitk_clusters(dev, k) < tiles % grid) k = 1;
+      if (k > 1) first = tiles - tiles % grid;
+    }
+  }
   if (print_configs())
-    std::fprintf(stderr, "[dg] %s M=%d N=%d K=%d: BM=128 BN=256 tiles=%lld grid=%d\n", name, M, N,
-                 K, tiles, grid);
-  return launch_gemm<MODE, 256>(ta, tb, dummy, tsb, td, args, grid, st, dev);
+    std::fprintf(stderr, "[dg] %s M=%d N=%d K=%d: BM=128 BN=256 tiles=%lld grid=%d split %dx%lld\n",
+                 name, M, N, K, tiles, grid, k, k > 1 ? tiles - first : 0ll);
+  if (first > 0) {
+    GemmArgs full = args;
+    full.total_tiles = static_cast<int>(first);
+    dg_status s1 = launch_gemm<MODE, 256>(ta, tb, dummy, tsb, td, full,
+                                          static_cast<int>(std::min<long long>(grid, first)), st, dev);
+    if (s1 != DG_OK || k == 1) return s1;
+  }
+  args.total_tiles = static_cast<int>(tiles - first);
+  args.split_tile0 = static_cast<int>(first);
+  args.split = k;
+  args.drop_arrive = 0;
+  return launch_gemm<SPLIT_MODE, 256>(ta, tb, dummy, tsb, td, args,
+                                      static_cast<int>(tiles - first) * k, st, dev, k);
 }
 
 // Shared argument checks of the dense entry points. a_mn / b_mn: the operand

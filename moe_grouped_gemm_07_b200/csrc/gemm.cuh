@@ -45,11 +45,21 @@ namespace dg {
 enum GemmMode : int {
   MODE_DENSE = 0, MODE_CONTIG = 1, MODE_MASKED = 2, MODE_KGROUPED = 3, MODE_PAIR = 4,
   MODE_NN = 5, MODE_TN = 6, MODE_TT = 7,
-  // the dense launch's partial last wave, as its own launch: each leftover
-  // tile is split along K over a cluster of `split` CTAs, whose FP32
-  // partials are summed through distributed shared memory
-  MODE_SPLITK = 8
+  // dense tiles split along K over a cluster of `split` CTAs, whose FP32
+  // partials are summed through distributed shared memory (a dense launch's
+  // partial last wave, or every tile of a launch with few rows), for each
+  // operand layout: NT, NN, TN, TT
+  MODE_SPLITK = 8, MODE_SPLITK_NN = 9, MODE_SPLITK_TN = 10, MODE_SPLITK_TT = 11
 };
+
+// The operand layout of a mode (a split-K mode has the layout of its dense mode).
+constexpr int layout_of(int mode) {
+  return mode == MODE_SPLITK      ? MODE_DENSE
+         : mode == MODE_SPLITK_NN ? MODE_NN
+         : mode == MODE_SPLITK_TN ? MODE_TN
+         : mode == MODE_SPLITK_TT ? MODE_TT
+                                  : mode;
+}
 
 constexpr int kMaxKGroups = 256;
 constexpr int kMaxMaskedGroups = 1024;
@@ -96,8 +106,9 @@ struct GemmCfg {
   static constexpr int GROUP_M = 16;       // tile rasterisation group (L2 reuse)
   static constexpr bool KG = MODE == MODE_KGROUPED;
   // operands stored MN-major (K-outer) in global and shared memory
-  static constexpr bool A_MN = KG || MODE == MODE_TN || MODE == MODE_TT;
-  static constexpr bool B_MN = KG || MODE == MODE_NN || MODE == MODE_TN;
+  static constexpr int LAYOUT = layout_of(MODE);
+  static constexpr bool A_MN = KG || LAYOUT == MODE_TN || LAYOUT == MODE_TT;
+  static constexpr bool B_MN = KG || LAYOUT == MODE_NN || LAYOUT == MODE_TN;
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
@@ -195,7 +206,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int*
       tl.b_row = g * a.N + tl.n0;
       tl.rows = Cfg::BM;
     }
-  } else if constexpr (MODE == MODE_SPLITK) {
+  } else if constexpr (MODE >= MODE_SPLITK) {
     // tile split_tile0 + t of the dense rasterisation; CTA `rank` of the
     // cluster takes K-blocks [rank * KB / split, (rank + 1) * KB / split)
     const int tt = a.split_tile0 + t;
@@ -316,7 +327,7 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t lane = lane_id();
   const uint64_t tmo = args.timeout_ns;
   constexpr bool PAIR = Cfg::PAIR;
-  constexpr bool SPLITK = MODE == MODE_SPLITK;
+  constexpr bool SPLITK = MODE >= MODE_SPLITK;
   // pair: 0 = leader of the pair; split-K tail: the part of the K range
   const uint32_t rank = (PAIR || SPLITK) ? cluster_ctarank() : 0u;
   const bool leader = !PAIR || rank == 0;
@@ -675,7 +686,7 @@ __global__ void __launch_bounds__(320, 1)
         half_in = col_first < args.N;
         // sfb is [G][ceil(N/128)][K/128], or [K/128][ceil(N/128)] for B stored [K][N]
         pb = Cfg::B_MN ? col_first / 128 : (tl.g * nbN + col_first / 128) * KBn;
-        if constexpr (SPLITK) pb += tl.kb0;  // this part starts at K-block kb0
+        if constexpr (SPLITK) pb += Cfg::B_MN ? tl.kb0 * nbN : tl.kb0;  // part starts at kb0
         if (half_in && tl.nkb > 0 && (Cfg::B_MN || !args.sfb_tma)) sb_next = sfb_at(0);
       }
 
