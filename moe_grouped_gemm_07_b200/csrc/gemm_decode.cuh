@@ -548,7 +548,6 @@ __global__ void __launch_bounds__(320, MINB)
         const uint32_t mb = dsmem_addr(smem_addr(rbar), orank);
         bulk_copy_to_cluster(dst, stage_out + lo * 128, static_cast<uint32_t>((hi - lo) * 512), mb);
       }
-      bulk_commit();
     }
   }
   bool ok = true;
@@ -556,6 +555,11 @@ __global__ void __launch_bounds__(320, MINB)
     volatile int never = 0;
     ok = mbar_wait(rbar, 0, &never, tmo, SITE_SPLITK_RECV);
   }
+  // The copies complete only on the owners' barriers, so a CTA's staged
+  // partial must stay until every owner has seen its receive slots complete:
+  // each CTA arrives once its own have (or it receives nothing) and waits for
+  // the whole cluster before it exits.
+  if (splits > 1 && !PAIR) cluster_arrive_relaxed();
   if (ok && !*abort_flag) {
     // this CTA's token rows: item = (token m, 8 weight rows), weight rows fastest
     const int items = (m_hi - m_lo) * 16;
@@ -594,9 +598,6 @@ __global__ void __launch_bounds__(320, MINB)
       *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.D) + o) = out;
     }
   }
-  // this CTA's partial must stay until the copies to its peers have read it
-  if (splits > 1 && threadIdx.x == 0) bulk_wait_read0();
-
   if constexpr (PAIR) {
     // the even CTA's MMAs wrote this CTA's TMEM and read its shared memory:
     // neither is released before the whole cluster is here
@@ -606,9 +607,12 @@ __global__ void __launch_bounds__(320, MINB)
       tc_fence_after();
       tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
     }
-  } else if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  } else {
+    if (splits > 1) cluster_wait();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    }
   }
 }
 

@@ -425,8 +425,9 @@ __device__ __forceinline__ void cluster_wait() {
 // Bulk copy of `bytes` bytes (multiple of 16, both addresses 16-byte aligned)
 // from this CTA's shared memory into shared memory of a CTA of the cluster
 // (`dst_cluster`, a shared::cluster address), completing `bytes` transaction
-// bytes on the destination CTA's mbarrier at `mbar_cluster`. Tracked by the
-// issuing thread's bulk async group (bulk_commit / bulk_wait_read0).
+// bytes on the destination CTA's mbarrier at `mbar_cluster`. The copy is in
+// no bulk async group: only the destination's mbarrier tells when it is done
+// (and so when the source may be reused).
 __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, const void* src,
                                                      uint32_t bytes, uint32_t mbar_cluster) {
   asm volatile(
