@@ -353,6 +353,9 @@ uint64_t dg_get_launch_count(void);
  *   DG_DECODE_PF=k       weight K-blocks the FP8 M <= 128 kernel keeps
  *                        requested into L2 ahead of its loads (rounded up to
  *                        a multiple of 8, default 64); read on every call.
+ *   DG_WIDE_EPI=0|1      dense NT tile kernel with a 3-stage ring and
+ *                        whole-tile output staging (default for K <= 1536);
+ *                        read on every call.
  *   DG_SMALL_M_TILES=1   FP8 NT with M <= 128 on the 128 x 256 tile kernel,
  *                        every tile split along K over a cluster, instead of
  *                        the swap-AB decode kernel; read on every call. */

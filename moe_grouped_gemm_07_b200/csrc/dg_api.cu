@@ -243,6 +243,14 @@ int small_m_tiles_env() {
   return e ? (e[0] == '1' ? 1 : 0) : -1;
 }
 
+// Dense NT tiles with few K-blocks spend much of each tile in the epilogue:
+// up to 12 K-blocks run the 3-stage, whole-tile-staging kernel
+// (MODE_DENSE_WIDE). DG_WIDE_EPI=0|1 forces it off or on (read on every call).
+bool wide_epilogue(int KB) {
+  if (const char* e = std::getenv("DG_WIDE_EPI")) return e[0] == '1';
+  return KB <= 12;
+}
+
 // Split-K tail of a dense launch (MODE_SPLITK): DG_TAIL_SPLIT=0 turns it off.
 bool tail_split_enabled() {
   static const bool on = [] {
@@ -424,6 +432,10 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
     tail.drop_arrive = 0;
     return launch_gemm<dg::MODE_SPLITK, 256>(ta, tb, dummy, tsb, td, tail,
                                              static_cast<int>(R) * split, st, dev, split);
+  }
+  if (MODE == dg::MODE_DENSE && bn == 256 && wide_epilogue(K / 128)) {
+    if (print_configs()) std::fprintf(stderr, "[dg] %s: wide epilogue (3 stages)\n", name);
+    return launch_gemm<dg::MODE_DENSE_WIDE, 256>(ta, tb, dummy, tsb, td, args, grid, st, dev);
   }
   if (bn == 256) return launch_gemm<MODE, 256>(ta, tb, dummy, tsb, td, args, grid, st, dev);
   return launch_gemm<MODE, 128>(ta, tb, dummy, tsb, td, args, grid, st, dev);

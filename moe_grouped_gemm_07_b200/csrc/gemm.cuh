@@ -49,12 +49,20 @@ enum GemmMode : int {
   // partials are summed through distributed shared memory (a dense launch's
   // partial last wave, or every tile of a launch with few rows), for each
   // operand layout: NT, NN, TN, TT
-  MODE_SPLITK = 8, MODE_SPLITK_NN = 9, MODE_SPLITK_TN = 10, MODE_SPLITK_TT = 11
+  MODE_SPLITK = 8, MODE_SPLITK_NN = 9, MODE_SPLITK_TN = 10, MODE_SPLITK_TT = 11,
+  // dense NT for short K: a 3-stage ring and a whole-tile output staging (each
+  // warp writes all its chunks, fences once and issues its stores together)
+  MODE_DENSE_WIDE = 12
 };
+
+// Split-K modes (tiles cut along K over a cluster), by layout: 8..11.
+__host__ __device__ constexpr bool is_splitk(int mode) { return mode >= MODE_SPLITK && mode <= MODE_SPLITK_TT; }
+static_assert(!is_splitk(MODE_DENSE_WIDE) && !is_splitk(MODE_TT) && is_splitk(MODE_SPLITK_NN),
+              "split-K mode range");
 
 // The operand layout of a mode (a split-K mode has the layout of its dense mode).
 constexpr int layout_of(int mode) {
-  return mode == MODE_SPLITK      ? MODE_DENSE
+  return mode == MODE_SPLITK || mode == MODE_DENSE_WIDE ? MODE_DENSE
          : mode == MODE_SPLITK_NN ? MODE_NN
          : mode == MODE_SPLITK_TN ? MODE_TN
          : mode == MODE_SPLITK_TT ? MODE_TT
@@ -93,7 +101,8 @@ struct GemmCfg {
   static constexpr int BK = 128;  // FP8 elements (= bytes) per K-block
   static constexpr bool PAIR = MODE == MODE_PAIR;
   // ring depth from the stage size (A + this CTA's B): 48 KB -> 4, 32 KB -> 6, 24 KB -> 8
-  static constexpr int STAGES = PAIR ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6);
+  static constexpr bool WIDE = MODE == MODE_DENSE_WIDE;
+  static constexpr int STAGES = PAIR ? (BN == 256 ? 6 : 8) : WIDE ? 3 : (BN == 256 ? 4 : 6);
   static constexpr int SCALE_SLOTS = 8;  // K-grouped only
   static constexpr int A_BYTES = BM * BK;
   static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * BK;  // this CTA's part of the B tile
@@ -126,7 +135,7 @@ struct GemmCfg {
       ((OFF_SCALE + SCALE_SLOTS * (KG ? SCALE_BYTES : NT_SCALE_BYTES) + 1023) / 1024) * 1024;
   // output staging for the TMA-store epilogue: one 32-row x 64-byte chunk
   // (32 bf16 or 16 fp32 columns) per promotion warp, 64-byte swizzled
-  static constexpr int STAGE_BYTES_PER_WARP = 32 * 64;
+  static constexpr int STAGE_BYTES_PER_WARP = 32 * 64 * (WIDE ? BN / 64 : 1);
   static constexpr int STORE_COLS = KG ? 16 : 32;
   static constexpr int OFF_BAR = OFF_STAGE + 8 * STAGE_BYTES_PER_WARP;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NACC + 2 * SCALE_SLOTS + 1;
@@ -182,7 +191,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int*
     tl.b_row = tl.n0 + rank * (BN / 2);
     tl.rows = min(Cfg::BM, a.M - tl.m0);  // may be <= 0 for the second CTA
     tl.out_row0 = tl.m0;
-  } else if constexpr (MODE == MODE_DENSE || MODE == MODE_CONTIG ||
+  } else if constexpr (MODE == MODE_DENSE || MODE == MODE_DENSE_WIDE || MODE == MODE_CONTIG ||
                        (MODE >= MODE_NN && MODE <= MODE_TT)) {
     const int group_tiles = Cfg::GROUP_M * a.num_n_blocks;
     const int grp = t / group_tiles;
@@ -206,7 +215,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int*
       tl.b_row = g * a.N + tl.n0;
       tl.rows = Cfg::BM;
     }
-  } else if constexpr (MODE >= MODE_SPLITK) {
+  } else if constexpr (is_splitk(MODE)) {
     // tile split_tile0 + t of the dense rasterisation; CTA `rank` of the
     // cluster takes K-blocks [rank * KB / split, (rank + 1) * KB / split)
     const int tt = a.split_tile0 + t;
@@ -327,7 +336,7 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t lane = lane_id();
   const uint64_t tmo = args.timeout_ns;
   constexpr bool PAIR = Cfg::PAIR;
-  constexpr bool SPLITK = MODE >= MODE_SPLITK;
+  constexpr bool SPLITK = is_splitk(MODE);
   // pair: 0 = leader of the pair; split-K tail: the part of the K range
   const uint32_t rank = (PAIR || SPLITK) ? cluster_ctarank() : 0u;
   const bool leader = !PAIR || rank == 0;
@@ -856,13 +865,22 @@ __global__ void __launch_bounds__(320, 1)
         } else if (use_tma) {
           constexpr int CW = Cfg::STORE_COLS;
           uint8_t* stg = sStage + (warp - 2) * Cfg::STAGE_BYTES_PER_WARP;
+          uint8_t* const stg0 = stg;
           const int swz = static_cast<int>((lane >> 1) & 3);  // 64-byte swizzle of row `lane`
+          if constexpr (Cfg::WIDE) {  // the previous tile's stores have left the staging
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
+          }
 #pragma unroll
           for (int c = 0; c < EC / CW; ++c) {
             const int n = col0 + c * CW;
             if (n >= args.N) break;
-            if (lane == 0) bulk_wait_read0();  // previous chunk has left the staging buffer
-            __syncwarp();
+            if constexpr (Cfg::WIDE) {
+              stg = sStage + (warp - 2) * Cfg::STAGE_BYTES_PER_WARP + c * 32 * 64;
+            } else {
+              if (lane == 0) bulk_wait_read0();  // previous chunk has left the staging buffer
+              __syncwarp();
+            }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               uint4 o;
@@ -895,10 +913,25 @@ __global__ void __launch_bounds__(320, 1)
               }
               *reinterpret_cast<uint4*>(stg + lane * 64 + ((j ^ swz) << 4)) = o;
             }
+            if constexpr (!Cfg::WIDE) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tm_d, stg, n, static_cast<int>(tl.out_row0 + q * 32));
+                bulk_commit();
+              }
+            }
+          }
+          if constexpr (Cfg::WIDE) {  // one fence, then every chunk's store
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tm_d, stg, n, static_cast<int>(tl.out_row0 + q * 32));
+#pragma unroll
+              for (int c = 0; c < EC / CW; ++c) {
+                const int n = col0 + c * CW;
+                if (n >= args.N) break;
+                tma_store_2d(&tm_d, stg0 + c * 32 * 64, n, static_cast<int>(tl.out_row0 + q * 32));
+              }
               bulk_commit();
             }
           }
