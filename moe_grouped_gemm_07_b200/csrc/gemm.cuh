@@ -21,7 +21,8 @@
 //   warps 2..9  promotion / epilogue: warp w reads TMEM lane quadrant (w % 4)
 //               and column half ((w - 2) / 4); acc += s * P in registers
 //               (NT: s = sfa from the scale ring x sfb read one K-block
-//               ahead); at tile end adds C, converts and stores D.
+//               ahead, or from a box of sfb in the same ring); at tile end
+//               adds C, converts and stores D.
 // The MMA runs up to 512/BN - 1 K-blocks ahead of the promotion (2 buffers at
 // BN=256, 4 at BN=128); the producer runs up to S K-blocks ahead.
 #pragma once

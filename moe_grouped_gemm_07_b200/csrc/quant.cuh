@@ -336,11 +336,15 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const void* __restrict__
 // to nearest, ties to the even code: the thresholds are the midpoints of
 // neighbouring magnitudes, strict where the lower neighbour has the even code
 // and inclusive where the upper one has; |y| > 6 gives the largest code.
-__device__ __forceinline__ uint32_t e2m1_code(float y) {
-  const float a = fabsf(y);
-  const uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
-                     (a >= 3.5f) + (a > 5.0f);
-  return c | ((__float_as_uint(y) >> 28) & 8u);
+// Two values to E2M1 codes, round to nearest even with saturation to +-6
+// (the hardware conversion; a negative value that rounds to zero keeps its
+// sign bit): `lo` in bits 0..3, `hi` in bits 4..7.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(out)
+      : "f"(hi), "f"(lo));
+  return out;
 }
 
 // Exponent e of the FP4 scale 2^e = 2^ceil(log2 t), t = max(amax, 1e-4f) / 6
@@ -402,7 +406,8 @@ __global__ void __launch_bounds__(256) quant_fp4_kernel(const void* __restrict__
         for (int h = 0; h < 2; ++h) {
           uint32_t acc = 0;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc |= e2m1_code(v[u][h * 8 + j] * rc) << (4 * j);
+          for (int j = 0; j < 4; ++j)
+            acc |= e2m1x2(v[u][h * 8 + 2 * j] * rc, v[u][h * 8 + 2 * j + 1] * rc) << (8 * j);
           w[h] = acc;
         }
         *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(st) * 64 + li * 8) =

@@ -78,6 +78,31 @@ CASES = [
 ]
 
 
+
+
+def test_fp4_quantiser_ties_and_signed_zeros():
+    """Strips whose amax is 6 (scale 1) holding every E2M1 midpoint, values one
+    ulp either side of them, the saturation edge and tiny values of both signs:
+    codes (ties to even, -0 keeps its sign bit) and scales match the oracle."""
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    vals = np.concatenate([mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(7)),
+                           np.array([0.0, 1e-30, 6.0, 5.999999], np.float32)])
+    row = np.concatenate([vals, -vals])          # 52 values
+    row = np.concatenate([row, np.zeros(128 - row.size, np.float32)])
+    row[row.size - 1] = 6.0                      # every 32-strip has amax 6
+    row[31] = 6.0
+    row[63] = -6.0
+    row[95] = 6.0
+    x = np.tile(row, (4, 2)).astype(np.float32)  # 4 x 256
+    x[1] *= np.float32(0.5)                      # scale 2^-1
+    x[2] *= np.float32(8.0)                      # scale 2^3
+    x[3] = -x[3]
+    oc, osc = oracle.quantize_fp4(x)
+    codes, s, packed = dg.dg_quantize_fp4_e2m1(to_dev(x))
+    assert np.array_equal(codes.cpu().numpy(), oc)
+    assert np.array_equal(s.cpu().numpy(), osc)
+
+
 @pytest.mark.parametrize("M,N,K,with_c", CASES)
 def test_fp8_fp4_gemm_vs_oracle(M, N, K, with_c):
     w = wl.dense(M, N, K, cfg=95, shape=M + N + K, with_c=with_c)
