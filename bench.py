@@ -142,11 +142,13 @@ class ClockSampler:
 
 
 def kernel_source_hash():
+    """Hash of the dominant kernel's sources: the tile kernel, its PTX helpers
+    and the host code that plans and launches it (a recorded DRAM traffic is
+    void once any of them changes)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "moe_grouped_gemm_07_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in ("dg_api.cu", "gemm.cuh", "ptx.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
