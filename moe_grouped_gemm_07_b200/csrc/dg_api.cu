@@ -284,8 +284,9 @@ bool no_pending_error() { return cudaPeekAtLastError() == cudaSuccess; }
 
 // How many k-CTA clusters of the split-K kernel the device runs at once
 // (cached per device and k; 0 on error).
+template <int SMODE = dg::MODE_SPLITK>
 int splitk_clusters(int dev, int k) {
-  using Cfg = dg::GemmCfg<dg::MODE_SPLITK, 256>;
+  using Cfg = dg::GemmCfg<SMODE, 256>;
   static std::mutex mu;
   static int cache[kMaxDevices][9];
   static bool done[kMaxDevices][9];
@@ -294,7 +295,7 @@ int splitk_clusters(int dev, int k) {
     if (!no_pending_error()) return 0;
     done[dev][k] = true;
     cache[dev][k] = 0;
-    auto kern = dg::gemm_fp8_kernel<dg::MODE_SPLITK, 256>;
+    auto kern = dg::gemm_fp8_kernel<SMODE, 256>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) ==
         cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
@@ -436,6 +437,32 @@ dg_status run_nt(const void* A, const float* sfa, int ld_sfa, const void* B, con
   if (MODE == dg::MODE_DENSE && bn == 256 && wide_epilogue(K / 128)) {
     if (print_configs()) std::fprintf(stderr, "[dg] %s: wide epilogue (3 stages)\n", name);
     return launch_gemm<dg::MODE_DENSE_WIDE, 256>(ta, tb, dummy, tsb, td, args, grid, st, dev);
+  }
+  if (MODE == dg::MODE_MASKED && bn == 256 && tail_split_enabled()) {
+    // The tile count T is known only on the device. A second launch of
+    // clusters of k CTAs takes the partial last wave (R = T mod grid tiles,
+    // each split along K) when R fits in its clusters; both launches work
+    // out R from the counts, the full-wave launch stops at T - R. Planned
+    // when a split saves at least 16 K-blocks of a tile.
+    const int KB = K / 128;
+    int k = 0;
+    for (int c = 4; c >= 2 && k == 0; c /= 2)
+      if (KB - KB / c >= 16 && KB / c >= 4) k = c;
+    int clusters = k ? std::min(splitk_clusters<dg::MODE_SPLITK_MASKED>(dev, k), grid / k) : 0;
+    if (print_configs())
+      std::fprintf(stderr, "[dg] %s: masked tail split %d x up to %d clusters\n", name, k, clusters);
+    if (k > 1 && clusters > 0) {
+      args.tail_k = k;
+      args.tail_clusters = clusters;
+      args.grid1 = grid;
+      dg_status s1 = launch_gemm<MODE, 256>(ta, tb, dummy, tsb, td, args, grid, st, dev);
+      if (s1 != DG_OK) return s1;
+      GemmArgs tail = args;
+      tail.split = k;
+      tail.drop_arrive = 0;
+      return launch_gemm<dg::MODE_SPLITK_MASKED, 256>(ta, tb, dummy, tsb, td, tail, clusters * k, st,
+                                                      dev, k);
+    }
   }
   if (bn == 256) return launch_gemm<MODE, 256>(ta, tb, dummy, tsb, td, args, grid, st, dev);
   return launch_gemm<MODE, 128>(ta, tb, dummy, tsb, td, args, grid, st, dev);

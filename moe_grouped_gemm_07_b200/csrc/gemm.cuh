@@ -53,17 +53,25 @@ enum GemmMode : int {
   MODE_SPLITK = 8, MODE_SPLITK_NN = 9, MODE_SPLITK_TN = 10, MODE_SPLITK_TT = 11,
   // dense NT for short K: a 3-stage ring and a whole-tile output staging (each
   // warp writes all its chunks, fences once and issues its stores together)
-  MODE_DENSE_WIDE = 12
+  MODE_DENSE_WIDE = 12,
+  // the masked launch's partial last wave (its size known only on the
+  // device), each tile split along K over a cluster
+  MODE_SPLITK_MASKED = 13
 };
 
 // Split-K modes (tiles cut along K over a cluster), by layout: 8..11.
-__host__ __device__ constexpr bool is_splitk(int mode) { return mode >= MODE_SPLITK && mode <= MODE_SPLITK_TT; }
+__host__ __device__ constexpr bool is_splitk(int mode) {
+  return (mode >= MODE_SPLITK && mode <= MODE_SPLITK_TT) || mode == MODE_SPLITK_MASKED;
+}
+__host__ __device__ constexpr bool is_masked(int mode) {
+  return mode == MODE_MASKED || mode == MODE_SPLITK_MASKED;
+}
 static_assert(!is_splitk(MODE_DENSE_WIDE) && !is_splitk(MODE_TT) && is_splitk(MODE_SPLITK_NN),
               "split-K mode range");
 
 // The operand layout of a mode (a split-K mode has the layout of its dense mode).
 constexpr int layout_of(int mode) {
-  return mode == MODE_SPLITK || mode == MODE_DENSE_WIDE ? MODE_DENSE
+  return mode == MODE_SPLITK || mode == MODE_DENSE_WIDE || mode == MODE_SPLITK_MASKED ? MODE_DENSE
          : mode == MODE_SPLITK_NN ? MODE_NN
          : mode == MODE_SPLITK_TN ? MODE_TN
          : mode == MODE_SPLITK_TT ? MODE_TT
@@ -92,6 +100,10 @@ struct GemmArgs {
   const int32_t* ks_dev;        // K-grouped, device sizes: [G] K per group (else null)
   int kb_cap;                   // K-grouped, device sizes: K-blocks the operands hold
   int split_tile0, split;       // MODE_SPLITK: first tail tile, CTAs per tile
+  // masked: split the partial last wave over clusters of tail_k CTAs (0: no)
+  // when its R = T mod grid1 tiles fit in tail_clusters clusters; the
+  // full-wave launch then stops at T - R and MODE_SPLITK_MASKED does the rest
+  int tail_k, tail_clusters, grid1;
   int sfb_tma;                  // NT: sfb comes through the scale ring (tm_sfb), else __ldg
 };
 
@@ -142,7 +154,7 @@ struct GemmCfg {
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NACC + 2 * SCALE_SLOTS + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;       // tmem slot, abort flag
   static constexpr int OFF_PREFIX = OFF_MISC + 16;              // masked: prefix + counts
-  static constexpr int PREFIX_BYTES = MODE == MODE_MASKED     ? (2 * kMaxMaskedGroups + 1) * 4
+  static constexpr int PREFIX_BYTES = is_masked(MODE)         ? (2 * kMaxMaskedGroups + 1) * 4
                                       : MODE == MODE_KGROUPED ? (kMaxKGroups + 1) * 4
                                                               : 0;
   static constexpr int SMEM_BYTES = OFF_PREFIX + PREFIX_BYTES + 1024;  // + alignment slack
@@ -216,7 +228,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int*
       tl.b_row = g * a.N + tl.n0;
       tl.rows = Cfg::BM;
     }
-  } else if constexpr (is_splitk(MODE)) {
+  } else if constexpr (is_splitk(MODE) && MODE != MODE_SPLITK_MASKED) {
     // tile split_tile0 + t of the dense rasterisation; CTA `rank` of the
     // cluster takes K-blocks [rank * KB / split, (rank + 1) * KB / split)
     const int tt = a.split_tile0 + t;
@@ -235,7 +247,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int*
     const int KB = a.K / Cfg::BK;
     tl.kb0 = (rank * KB) / a.split;
     tl.nkb = ((rank + 1) * KB) / a.split - tl.kb0;
-  } else if constexpr (MODE == MODE_MASKED) {
+  } else if constexpr (is_masked(MODE)) {
     // largest g with prefix[g] <= t
     int lo = 0, hi = a.G - 1;
     while (lo < hi) {
@@ -254,6 +266,11 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& a, const int*
     tl.b_row = g * a.N + tl.n0;
     tl.rows = min(Cfg::BM, mm_clamped[g] - tl.m0);
     tl.out_row0 = static_cast<long long>(g) * a.M + tl.m0;
+    if constexpr (MODE == MODE_SPLITK_MASKED) {  // CTA `rank` of the cluster: its part of K
+      const int KB = a.K / Cfg::BK;
+      tl.kb0 = (rank * KB) / a.split;
+      tl.nkb = ((rank + 1) * KB) / a.split - tl.kb0;
+    }
   } else {  // K-grouped
     const int per_g = a.num_m_blocks * a.num_n_blocks;
     const int g = t / per_g;
@@ -396,7 +413,8 @@ __global__ void __launch_bounds__(320, 1)
   // (everything above touched only shared memory, TMEM and kernel params)
   pdl_wait();
   int total_tiles = args.total_tiles;
-  if constexpr (MODE == MODE_MASKED) {
+  int tail0 = 0;  // MODE_SPLITK_MASKED: tile index of its first tile
+  if constexpr (is_masked(MODE)) {
     if (warp == 2) {
       int carry = 0;
       for (int base = 0; base < args.G; base += 32) {
@@ -458,9 +476,18 @@ __global__ void __launch_bounds__(320, 1)
     }
     __syncthreads();
   }
-  if constexpr (MODE == MODE_MASKED) {
+  if constexpr (is_masked(MODE)) {
     __syncthreads();
     total_tiles = prefix[args.G];
+    // the same decision in both launches (same counts, same parameters)
+    const int R = args.tail_k > 1 ? total_tiles % args.grid1 : 0;
+    const bool split = R > 0 && R <= args.tail_clusters;
+    if constexpr (MODE == MODE_MASKED) {
+      if (split) total_tiles -= R;
+    } else {
+      tail0 = total_tiles - R;
+      total_tiles = split ? R : 0;
+    }
   }
 
   // ---------------------------------------------------------------- roles
@@ -472,7 +499,7 @@ __global__ void __launch_bounds__(320, 1)
       uint32_t it = 0, sit = 0;
       int dropped = -1;
       for (int t = cta_first; t < total_tiles; t += cta_step) {
-        const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped, rank);
+        const Tile tl = decode_tile<MODE, BN>(t + tail0, args, prefix, mm_clamped, rank);
         if (!tl.valid) continue;
         for (int kb = 0; kb < tl.nkb; ++kb, ++it) {
           const uint32_t s = it % S;
@@ -553,7 +580,7 @@ __global__ void __launch_bounds__(320, 1)
             float* slot = sScale + ss * Cfg::NT_SLOT_FLOATS;
             if (lane == 3 && bytes > 0) {
               long long off = static_cast<long long>(tl.kb0 + kb) * args.ld_sfa + tl.m0;
-              if constexpr (MODE == MODE_MASKED)
+              if constexpr (is_masked(MODE))
                 off += static_cast<long long>(tl.g) * (args.K / Cfg::BK) * args.ld_sfa;
               bulk_load(slot, args.sfa + off, bytes, &sfull[ss]);
             }
@@ -601,7 +628,7 @@ __global__ void __launch_bounds__(320, 1)
           idesc_e4m3_f32(PAIR ? 2 * Cfg::BM : Cfg::BM, BN, Cfg::A_MN ? 1 : 0, Cfg::B_MN ? 1 : 0);
       uint32_t s = 0, full_ph = 0, b = 0, tmem_ph = 0;
       for (int t = cta_first; t < total_tiles; t += cta_step) {
-        const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped, rank);
+        const Tile tl = decode_tile<MODE, BN>(t + tail0, args, prefix, mm_clamped, rank);
         if (!tl.valid) continue;
         for (int kb = 0; kb < tl.nkb; ++kb) {
           bool ok = mbar_wait(&tempty[b], tmem_ph ^ 1, abort_flag, tmo, SITE_MMA_TMEM_EMPTY);
@@ -671,7 +698,7 @@ __global__ void __launch_bounds__(320, 1)
     const int KBn = args.K / Cfg::BK;  // NT: K-blocks per row of sfb
     const int nbN = (args.N + 127) / 128;
     for (int t = cta_first; t < total_tiles; t += cta_step) {
-      const Tile tl = decode_tile<MODE, BN>(t, args, prefix, mm_clamped, rank);
+      const Tile tl = decode_tile<MODE, BN>(t + tail0, args, prefix, mm_clamped, rank);
       if (!tl.valid) continue;
       float acc[EC];
 #pragma unroll

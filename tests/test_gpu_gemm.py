@@ -198,6 +198,36 @@ def test_masked_vs_oracle(G, max_m, N, K):
         assert np.all(raw[g, w.masked_m[g]:] == SENTINEL), f"group {g}: masked rows written"
 
 
+def test_masked_last_wave_split():
+    """Masked GEMM on a capped grid: 60 tiles of 128 x 256 on 28 CTAs leave a
+    last wave of 4 tiles, which a second launch splits 4 ways along K over
+    clusters (the count is known only on the device). Results match the
+    oracle, repeat bit for bit, and rows past each count stay untouched."""
+    G, max_m, N, K = 3, 256, 3072, 4096
+    w = wl.masked(G=G, max_m=max_m, N=N, K=K, lo=0, hi=max_m, cfg=99, shape=G)
+    w.masked_m[:] = np.array([200, 100, 256], dtype=w.masked_m.dtype)
+    qa, sa = dg.dg_quantize_fp8(to_dev(w.A), dg.DG_QUANT_ROW_1x128)
+    qb, sb = dg.dg_quantize_fp8(to_dev(w.B), dg.DG_QUANT_BLOCK_128x128)
+    outs = []
+    dg.dg_set_num_sms(28)
+    try:
+        for _ in range(2):
+            D = sentinel_bf16((G, max_m, N))
+            dg.dg_m_grouped_fp8_gemm_nt_masked(qa, sa, qb, sb, to_dev(w.masked_m), D)
+            outs.append(D)
+        assert dg.dg_get_last_device_error() == (dg.DG_OK, 0)
+    finally:
+        dg.dg_set_num_sms(0)
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    oqa, osa = oracle.quantize(w.A, oracle.ROW_1x128)
+    oqb, osb = oracle.quantize(w.B, oracle.BLOCK_128x128)
+    R = oracle.m_grouped_masked(oqa, osa, oqb, osb, w.masked_m)
+    check_close(as_f64(outs[0]), R, "masked, split last wave")
+    raw = outs[0].view(torch.int16).cpu().numpy().view(np.uint16)
+    for g in range(G):
+        assert np.all(raw[g, w.masked_m[g]:] == SENTINEL), f"group {g}: masked rows written"
+
+
 def test_masked_expected_m_hint_changes_plan_not_results():
     """expected_m only steers the host's tile-width plan. For 8 groups of up
     to 1024 rows, N=1024, the bound (64 row blocks) plans 128x256 tiles and
