@@ -110,7 +110,7 @@ def quantize(x: np.ndarray, mode: int, ld_scales: int | None = None, bf16: bool 
         scales = np.zeros((batch, cols // 128, ld), dtype=np.float32)
     elif mode in (BLOCK_128x128, BLOCK_128x128_POW2):
         ld = 0
-        scales = np.zeros((batch, (rows + 127) // 128, cols // 128), dtype=np.float32)
+        scales = np.zeros((batch, (rows + 127) // 128, (cols + 127) // 128), dtype=np.float32)
     elif mode == COL_128x1:
         ld = 0
         scales = np.zeros((batch, rows // 128, cols), dtype=np.float32)

@@ -119,24 +119,26 @@ int dgo_quantize(const void* x, int in_is_bf16, int batch, int rows, int cols,
     return 0;
   }
   if (mode == DGO_BLOCK_128x128) {
-    if (cols % 128 != 0) return -1;
-    int kbs = cols / 128, nbs = (rows + 127) / 128;
+    /* a block at the bottom or right edge holds the rows [r0, r1) and the
+       columns [c0, c1) that exist */
+    int kbs = (cols + 127) / 128, nbs = (rows + 127) / 128;
     for (int b = 0; b < batch; ++b) {
       #pragma omp parallel for collapse(2) schedule(static)
       for (int nb = 0; nb < nbs; ++nb) {
         for (int kb = 0; kb < kbs; ++kb) {
           int r0 = nb * 128, r1 = r0 + 128 < rows ? r0 + 128 : rows;
+          int c0 = kb * 128, c1 = c0 + 128 < cols ? c0 + 128 : cols;
           float amax = 0.0f;
           for (int r = r0; r < r1; ++r)
-            for (int j = 0; j < 128; ++j) {
-              float v = fabsf(load_x(x, in_is_bf16, ((size_t)b * rows + r) * cols + kb * 128 + j));
+            for (int c = c0; c < c1; ++c) {
+              float v = fabsf(load_x(x, in_is_bf16, ((size_t)b * rows + r) * cols + c));
               if (v > amax) amax = v;
             }
           float s = pow2 ? pow2_scale_of(amax) : scale_of(amax);
           scales[((size_t)b * nbs + nb) * kbs + kb] = s;
           for (int r = r0; r < r1; ++r)
-            for (int j = 0; j < 128; ++j) {
-              size_t i = ((size_t)b * rows + r) * cols + kb * 128 + j;
+            for (int c = c0; c < c1; ++c) {
+              size_t i = ((size_t)b * rows + r) * cols + c;
               codes[i] = dgo_e4m3_encode(load_x(x, in_is_bf16, i) / s);
             }
         }

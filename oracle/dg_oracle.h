@@ -54,8 +54,10 @@ enum { DGO_ROW_1x128_POW2 = 3, DGO_BLOCK_128x128_POW2 = 4 };
  * otherwise) into E4M3 codes[batch][rows][cols] and FP32 scales:
  *   ROW_1x128    : one scale per (row, 128-column strip); cols % 128 == 0;
  *                  scales[b][cols/128][ld_scales] (transposed, "MN-major").
- *   BLOCK_128x128: one scale per 128x128 block (rows may be ragged);
- *                  scales[b][ceil(rows/128)][cols/128]; cols % 128 == 0.
+ *   BLOCK_128x128: one scale per 128x128 block; blocks at the bottom and
+ *                  right edges cover only the rows and columns that exist
+ *                  (their amax is taken over those elements);
+ *                  scales[b][ceil(rows/128)][ceil(cols/128)].
  *   COL_128x1    : one scale per (128-row strip, column); rows % 128 == 0;
  *                  scales[b][rows/128][cols].
  * scale = max(amax, 1e-4f) / 448.0f and code = E4M3(x / scale), both IEEE

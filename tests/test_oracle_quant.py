@@ -69,6 +69,40 @@ def test_block_scale_positions_ragged():
     assert sf[1, 1] == F32(F32(13.0) / F32(448.0))
 
 
+def test_block_scale_positions_ragged_columns():
+    """Blocks at the right edge (cols % 128 != 0) take their amax over the
+    columns that exist, as blocks at the bottom edge do over their rows."""
+    rows, cols = 200, 328                          # last column block has 72 columns
+    x = np.zeros((rows, cols), dtype=F32)
+    x[5, 300] = -3.0                               # block (0, 2)
+    x[127, 327] = 5.0                              # block (0, 2), its last column: the amax
+    x[150, 256] = -13.0                            # block (1, 2), its first column: the amax
+    x[199, 327] = 11.0                             # block (1, 2), its last row and column
+    x[64, 100] = 2.0                               # block (0, 0)
+    codes, sf = oracle.quantize(x, oracle.BLOCK_128x128)
+    assert sf.shape == (2, 3)
+    assert sf[0, 0] == F32(F32(2.0) / F32(448.0))
+    assert sf[0, 2] == F32(F32(5.0) / F32(448.0))
+    assert sf[1, 2] == F32(F32(13.0) / F32(448.0))
+    floor = F32(F32(1e-4) / F32(448.0))            # all-zero blocks
+    assert sf[0, 1] == floor and sf[1, 0] == floor and sf[1, 1] == floor
+    for (r, c), (br, bc) in {(5, 300): (0, 2), (127, 327): (0, 2), (150, 256): (1, 2),
+                             (199, 327): (1, 2), (64, 100): (0, 0)}.items():
+        assert codes[r, c] == torch_e4m3(np.array([x[r, c] / sf[br, bc]], dtype=F32))[0]
+
+
+def test_block_quantisation_commutes_with_transpose():
+    """A 128x128 block of x holds the same elements as the transposed block of
+    x.T, so BLOCK quantisation of x.T is the transpose of that of x: ragged
+    columns of one are ragged rows of the other."""
+    x = synth.normal((200, 328), synth.seed(9, 13, 0))
+    codes, sf = oracle.quantize(x, oracle.BLOCK_128x128)
+    codes_t, sf_t = oracle.quantize(np.ascontiguousarray(x.T), oracle.BLOCK_128x128)
+    assert sf.shape == (2, 3) and sf_t.shape == (3, 2)
+    assert np.array_equal(sf.view(np.uint32), sf_t.T.view(np.uint32))
+    assert np.array_equal(codes, codes_t.T)
+
+
 def test_col_scale_positions_closed_form():
     rows, cols = 256, 48
     x = np.zeros((rows, cols), dtype=F32)
@@ -245,12 +279,12 @@ def _numpy_scales(x, mode):
         amax = a.reshape(rows // 128, 128, cols).max(axis=1)
         s = (np.maximum(amax, F32(1e-4)).astype(F32) / F32(448.0)).astype(F32)
         return np.repeat(s, 128, axis=0)
-    nb = (rows + 127) // 128
-    pad = np.zeros((nb * 128, cols), dtype=F32)
-    pad[:rows] = a
-    amax = pad.reshape(nb, 128, cols // 128, 128).max(axis=(1, 3))
+    nb, kb = (rows + 127) // 128, (cols + 127) // 128
+    pad = np.zeros((nb * 128, kb * 128), dtype=F32)   # zeros never raise an amax
+    pad[:rows, :cols] = a
+    amax = pad.reshape(nb, 128, kb, 128).max(axis=(1, 3))
     s = (np.maximum(amax, F32(1e-4)).astype(F32) / F32(448.0)).astype(F32)
-    return np.repeat(np.repeat(s, 128, axis=0), 128, axis=1)[:rows]
+    return np.repeat(np.repeat(s, 128, axis=0), 128, axis=1)[:rows, :cols]
 
 
 def _expected_codes(x, s):
@@ -266,7 +300,7 @@ def _check_quotient(x, mode):
     elif mode == oracle.COL_128x1:
         got_s = np.repeat(sf, 128, axis=0)
     else:
-        got_s = np.repeat(np.repeat(sf, 128, axis=0), 128, axis=1)[:x.shape[0]]
+        got_s = np.repeat(np.repeat(sf, 128, axis=0), 128, axis=1)[:x.shape[0], :x.shape[1]]
     assert np.array_equal(got_s.view(np.uint32), s.view(np.uint32))
     assert np.array_equal(codes, _expected_codes(x, s))
 
@@ -280,6 +314,15 @@ def test_quotient_codes_random(mode):
     rows = 200 if mode == oracle.BLOCK_128x128 else 256
     x = synth.normal((rows, 512), synth.seed(9, 10, mode))
     _check_quotient(x, mode)
+
+
+def test_quotient_codes_ragged_block_columns():
+    """BLOCK mode on 200 x 328: ragged blocks at both edges. The first column
+    block is 50x larger, so an amax that strayed past the end of a row (into
+    the next row's first columns) would change the edge blocks' scales."""
+    x = synth.normal((200, 328), synth.seed(9, 14, 0))
+    x[:, :128] *= F32(50.0)
+    _check_quotient(x, oracle.BLOCK_128x128)
 
 
 @pytest.mark.parametrize("mode", MODES3)
