@@ -65,14 +65,16 @@ const char* dg_status_string(dg_status s);
  *                            scales[b][cols/128][ld_scales], transposed
  *                            (MN-major); ld_scales >= rows, ld_scales % 4 == 0.
  *                            This is the sfa layout every NT GEMM below reads.
- *     DG_QUANT_BLOCK_128x128 one per 128x128 block, rows may be ragged:
- *                            scales[b][ceil(rows/128)][cols/128]; cols % 128
- *                            == 0; ld_scales ignored. This is the sfb layout.
+ *     DG_QUANT_BLOCK_128x128 one per 128x128 block, rows and columns may
+ *                            be ragged: scales[b][ceil(rows/128)]
+ *                            [ceil(cols/128)]; cols % 4 == 0; ld_scales
+ *                            ignored. This is the sfb layout (of B [N][K],
+ *                            and of B [K][N] for the NN / TN layouts).
  *     DG_QUANT_COL_128x1     one per (128-row strip, column): rows % 128 == 0;
  *                            scales[b][rows/128][cols]; ld_scales ignored.
  *                            This is the layout the K-grouped TN GEMM reads.
  *   amax is taken over the elements that exist (a ragged last block reads only
- *   its real rows).
+ *   its real rows and columns).
  * ------------------------------------------------------------------------- */
 enum { DG_IN_F32 = 0, DG_IN_BF16 = 1 };
 enum { DG_QUANT_ROW_1x128 = 0, DG_QUANT_BLOCK_128x128 = 1, DG_QUANT_COL_128x1 = 2 };

@@ -144,7 +144,7 @@ def dg_quantize_fp8(x, mode, codes=None, scales=None, ld_scales=None, stream=Non
         sshape = (batch, cols // 128, ld)
     elif mode == DG_QUANT_BLOCK_128x128:
         ld = 0
-        sshape = (batch, (rows + 127) // 128, cols // 128)
+        sshape = (batch, (rows + 127) // 128, (cols + 127) // 128)
     elif mode == DG_QUANT_COL_128x1:
         ld = 0
         sshape = (batch, rows // 128, cols)

@@ -1332,8 +1332,10 @@ dg_status dg_quantize_fp8(const void* x, int in_dtype, int batch, int rows, int 
   if (batch < 0 || rows < 0 || cols < 0) return DG_ERR_INVALID_ARG;
   if (in_dtype != DG_IN_F32 && in_dtype != DG_IN_BF16) return DG_ERR_INVALID_ARG;
   if (mode < DG_QUANT_ROW_1x128 || mode > DG_QUANT_COL_128x1) return DG_ERR_INVALID_ARG;
-  if (mode == DG_QUANT_ROW_1x128 || mode == DG_QUANT_BLOCK_128x128) {
+  if (mode == DG_QUANT_ROW_1x128) {
     if (cols % 128 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+  } else if (mode == DG_QUANT_BLOCK_128x128) {
+    if (cols % 4 != 0) return DG_ERR_UNSUPPORTED_SHAPE;  // a lane's 4 columns
   } else {
     if (rows % 128 != 0 || cols % 4 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
   }
@@ -1359,7 +1361,8 @@ dg_status dg_quantize_fp8(const void* x, int in_dtype, int batch, int rows, int 
            : launch(dg::quant_row_kernel<false>, dim3(grid), dim3(256), 0, st, 1, x, batch, rows,
                     cols, q, scales, ld_scales, none);
   } else if (mode == DG_QUANT_BLOCK_128x128) {
-    const long long blocks = static_cast<long long>(batch) * ((rows + 127) / 128) * (cols / 128);
+    const long long blocks =
+        static_cast<long long>(batch) * ((rows + 127) / 128) * ((cols + 127) / 128);
     if (blocks > 0x7fffffffll) return DG_ERR_UNSUPPORTED_SHAPE;
     uint8_t* none = nullptr;
     e = bf ? launch(dg::quant_block_kernel<true>, dim3(static_cast<int>(blocks)), dim3(256), 0, st,

@@ -5,7 +5,7 @@
 // IEEE division would round it (see quotient()); this file must not be built
 // with --use_fast_math. Three scale granularities:
 //   ROW   one scale per (row, 128-column strip), stored transposed [cols/128][ld]
-//   BLOCK one scale per 128x128 block, [ceil(rows/128)][cols/128]
+//   BLOCK one scale per 128x128 block, [ceil(rows/128)][ceil(cols/128)]
 //   COL   one scale per (128-row strip, column), [rows/128][cols]
 // All three are single-pass, HBM-bound kernels: every input byte is read once,
 // every code and scale written once.
@@ -210,11 +210,13 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
 }
 
 // BLOCK_128x128: one 256-thread CTA per 128x128 block; warp w holds rows
-// [16w, 16w+16) of the block, lane l columns [4l, 4l+4).
+// [16w, 16w+16) of the block, lane l columns [4l, 4l+4). Blocks at the
+// bottom and right edges hold only the rows and columns that exist
+// (cols % 4 == 0, so a lane's four columns are all in or all out).
 // POW2: power-of-two scales; the block's UE8M0 byte is written for all 128
 // rows of the block into `packed` (batch 1), and `scales` may be null.
 template <bool BF16, bool POW2 = false>
-__global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict__ x, int batch,
+__global__ void __launch_bounds__(256, 2) quant_block_kernel(const void* __restrict__ x, int batch,
                                                           int rows, int cols,
                                                           uint8_t* __restrict__ codes,
                                                           float* __restrict__ scales,
@@ -223,17 +225,19 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
   pdl_trigger();  // the next launch's PDL wait still waits for this grid
   pdl_wait();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int kbs = cols >> 7, nbs = (rows + 127) >> 7;
+  const int kbs = (cols + 127) >> 7, nbs = (rows + 127) >> 7;
   const int64_t blk = blockIdx.x;
   const int kb = static_cast<int>(blk % kbs);
   const int nb = static_cast<int>((blk / kbs) % nbs);
   const int64_t b = blk / (static_cast<int64_t>(kbs) * nbs);
+  // rows this lane reads: none where its four columns lie past the right edge
+  const int lane_rows = (kb << 7) + (lane << 2) < cols ? rows : 0;
   In4 v[16];
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int r = (nb << 7) + (w << 4) + i;
-    if (r < rows) {
+    if (r < lane_rows) {
       v[i] = load4<BF16>(x, (b * rows + r) * cols + (kb << 7) + (lane << 2));
       amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].v[0]), fabsf(v[i].v[1])),
                                fmaxf(fabsf(v[i].v[2]), fabsf(v[i].v[3]))));
@@ -258,7 +262,7 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int r = (nb << 7) + (w << 4) + i;
-    if (r < rows)
+    if (r < lane_rows)
       *reinterpret_cast<uint32_t*>(codes + (b * rows + r) * cols + (kb << 7) + (lane << 2)) =
           encode4(v[i].v, sc, rc);
   }

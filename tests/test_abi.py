@@ -106,6 +106,11 @@ def test_host_validation_before_any_cuda_call():
         dg.DG_ERR_UNSUPPORTED_SHAPE
     assert L.dg_quantize_fp8(fake, 0, 1, 100, 128, 2, fake, fake, 0, None) == \
         dg.DG_ERR_UNSUPPORTED_SHAPE
+    # BLOCK mode takes ragged columns in whole groups of four
+    assert L.dg_quantize_fp8(fake, 0, 1, 128, 130, 1, fake, fake, 0, None) == \
+        dg.DG_ERR_UNSUPPORTED_SHAPE
+    assert L.dg_quantize_fp8(fake, 0, 1, 128, 132, 1, vp(0x1002), fake, 0, None) == \
+        dg.DG_ERR_MISALIGNED
     assert L.dg_quantize_fp8(fake, 7, 1, 128, 128, 0, fake, fake, 128, None) == \
         dg.DG_ERR_INVALID_ARG
     assert L.dg_quantize_fp8(fake, 0, 1, 128, 128, 0, fake, fake, 126, None) == \

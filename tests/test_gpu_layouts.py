@@ -21,7 +21,8 @@ pytestmark = pytest.mark.gpu
 
 FN = {"nn": dg.dg_fp8_gemm_nn, "tn": dg.dg_fp8_gemm_tn, "tt": dg.dg_fp8_gemm_tt}
 CASES = [(256, 256, 512, True), (144, 384, 640, False), (64, 512, 1024, True),
-         (1024, 2048, 2048, False), (128, 128, 128, True)]
+         (1024, 2048, 2048, False), (128, 128, 128, True),
+         (256, 2112, 1024, True)]   # N % 128 == 64: ragged last 128x128 block of B
 
 
 def run_layout_case(layout, M, N, K, with_c, cfg, sms=0, reps=1):
@@ -76,6 +77,7 @@ def test_dense_layouts_vs_oracle(layout, M, N, K, with_c):
 SPLIT_CASES = [
     (64, 1024, 4096, True, 0),      # 4 tiles, 8 parts each
     (128, 2176, 2048, False, 0),    # 9 tiles (ragged N), 4 parts each
+    (128, 2112, 2048, False, 0),    # 9 tiles, the last B block 64 wide
     (48, 512, 2048, True, 0),       # 2 tiles of 48 rows
     (384, 768, 8192, True, 8),      # 9 tiles on 8 CTAs: 1 tail tile x 8 parts
     (608, 1024, 12288, False, 16),  # 20 tiles on 16: 4 tail tiles x 4 parts

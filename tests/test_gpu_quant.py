@@ -49,6 +49,16 @@ def test_quant_random_bit_exact(mode, shape):
     assert_bit_exact(*run_both(x, mode))
 
 
+@pytest.mark.parametrize("shape", [(200, 328), (7168, 2112), (3, 130, 196), (64, 4)])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_quant_block_ragged_columns_bit_exact(shape, bf16):
+    """BLOCK mode with cols % 128 != 0 (B stored [K][N] for NN / TN, e.g.
+    N = 2112): the right-edge blocks cover only the existing columns."""
+    x = synth.normal(shape, synth.seed(70, zlib.crc32(repr(("ragged", shape)).encode()) % 997))
+    x[..., : min(128, shape[-1])] *= np.float32(50.0)   # an amax past a row's end would show
+    assert_bit_exact(*run_both(x, "block", bf16=bf16))
+
+
 @pytest.mark.parametrize("mode", ["row", "block", "col"])
 def test_quant_bf16_bit_exact(mode):
     x = synth.normal((256, 512), synth.seed(71, 1))
