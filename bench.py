@@ -418,7 +418,8 @@ def run_grouped(args):
 # ----------------------------------------------------------------- operand layouts
 def run_layouts(args):
     """--workload layouts: the dense GEMM in its four operand layouts (NT, NN,
-    TN, TT) at M in {64, 128, 4096} on two weight shapes, GEMM launches back
+    TN, TT) at M in {64, 128, 4096} on three weight shapes (N = 2112 has a
+    ragged last 128x128 block of B in the NN / TN storage), GEMM launches back
     to back over rotating weight copies (>= 3x L2) in a CUDA graph. NT routes
     M <= 128 to the swap-AB decode kernel; NN / TN / TT run the persistent
     kernel at every M. One GPU."""
@@ -432,7 +433,7 @@ def run_layouts(args):
     fns = {"nt": dg.dg_fp8_gemm_nt, "nn": dg.dg_fp8_gemm_nn, "tn": dg.dg_fp8_gemm_tn,
            "tt": dg.dg_fp8_gemm_tt}
     rows = []
-    for (N, K) in ((7168, 16384), (4096, 7168)):
+    for (N, K) in ((7168, 16384), (4096, 7168), (2112, 7168)):
         Bf = torch.from_numpy(synth.normal((N, K), synth.seed(2, nk_index(N, K), 1))).to(dev)
         for layout in ("nt", "nn", "tn", "tt"):
             b_mn = layout[1] == "n"
