@@ -944,7 +944,7 @@ def run_ours(args):
     return 0
 
 
-def main():
+def make_parser():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -965,7 +965,11 @@ def main():
                     help="dense (the bench line) or one MoE variant at its benchmark size")
     ap.add_argument("--masked-index", type=int, default=0,
                     help="masked workload: index into the (N, K) pairs")
-    args = ap.parse_args()
+    return ap
+
+
+def main():
+    args = make_parser().parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
